@@ -1,0 +1,14 @@
+"""Float64 CPU oracle (test infrastructure only; see attn64 for the header)."""
+from .attn64 import (  # noqa: F401
+    attn_bwd,
+    attn_fwd,
+    attn_fwd_online,
+    attn_partial,
+    attn_with_kvcache,
+    combine_splits,
+    effective_window,
+    gather_cache,
+    kvcache_append,
+    split_token_ranges,
+    visible,
+)

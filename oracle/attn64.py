@@ -1,0 +1,387 @@
+"""Float64 CPU oracle for exact scaled-dot-product attention.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the library imports, links or calls this
+module; only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` do.  It shares no code, header, table
+or constant with the CUDA path: every function here is the plain definition,
+written with NumPy in float64, and it materialises the whole score matrix on
+purpose.
+
+Sources (three web pages about FlashAttention; formulas are never written out
+there, so each function states the reading it implements):
+
+* "FlashAttention 实战指南" (mhpq.cn), section on why long sequences run out of
+  memory: standard scaled dot-product attention is QK^T, then softmax, then a
+  product with V; the method's output is numerically the same as that standard
+  attention ("exact").  -> :func:`attn_fwd` is that definition.
+* same page, section on advanced parameters: ``window_size=(left, right)`` with
+  (-1, -1) meaning an unbounded window; ``softcap`` bounds the logits to
+  [-softcap, softcap]; K/V may have fewer heads than Q as long as the Q head
+  count is an integer multiple (MQA/GQA); ``deterministic`` backward.
+* same page, section on incremental decoding: ``flash_attn_with_kvcache``
+  appends the new K/V into the existing cache and attends in place,
+  ``cache_seqlens`` marks each sample's valid length, ``block_table`` pages the
+  cache, ``num_splits`` splits the KV range.  -> :func:`attn_with_kvcache`.
+* same page, the three techniques: tiling, online softmax (running row max and
+  running sum updated block by block), recomputation in the backward.
+  -> :func:`attn_fwd_online` (used only to pin :func:`attn_fwd`).
+
+Readings where the pages are silent (each is listed in the design doc):
+
+* softcap: ``s = softcap * tanh(u / softcap)`` applied after the scale and
+  before the mask; ``softcap <= 0`` switches it off.
+* window: key j is visible to query i iff
+  ``i+off-left <= j <= i+off+right`` (inclusive), a negative extent is
+  unbounded; ``causal`` is the same as ``right = 0`` and intersects with a
+  given window.  ``off = Sk - Sq`` (bottom-right alignment).
+* GQA: q-head h reads kv-head ``h // (Hq // Hkv)``.
+* LSE is the natural-log row log-sum-exp, layout (B, Hq, Sq).
+* a row with no visible key has O = 0 and LSE = -inf.
+* ``cache_seqlens`` is the length before the append; the call attends over
+  ``cache_seqlens[b] + Snew`` keys and does not update ``cache_seqlens``.
+* split s of a sequence with P pages covers pages
+  ``ceil(s*P/n) .. ceil((s+1)*P/n) - 1``.
+
+Layouts follow the pages' (batch, seqlen, nheads, headdim) convention.
+"""
+
+import math
+
+import numpy as np
+
+# -inf arithmetic on masked entries is intended; the results are selected away.
+np.seterr(invalid="ignore", divide="ignore")
+
+NEG_INF = -np.inf
+
+
+# ---------------------------------------------------------------------------
+# visibility (mask) rule
+# ---------------------------------------------------------------------------
+
+def effective_window(causal, window_left, window_right):
+    """Return (left, right) extents after folding ``causal`` in.
+
+    Negative means unbounded.  Causal attention is the window with right
+    extent 0; when a window is also given the two are intersected.
+    """
+    left = int(window_left) if window_left is not None and window_left >= 0 else -1
+    right = int(window_right) if window_right is not None and window_right >= 0 else -1
+    if causal:
+        right = 0 if right < 0 else min(right, 0)
+    return left, right
+
+
+def visible(Sq, Sk, causal=False, window_left=-1, window_right=-1, key_offset=0, n_keys=None):
+    """Boolean (Sq, n_keys) matrix: may query i see key (key_offset + j)?
+
+    Query i sits at absolute position ``i + Sk - Sq``.  ``key_offset`` and
+    ``n_keys`` select a sub-range of the Sk keys (used for KV splits).
+    """
+    if n_keys is None:
+        n_keys = Sk - key_offset
+    left, right = effective_window(causal, window_left, window_right)
+    qpos = np.arange(Sq)[:, None] + (Sk - Sq)
+    kpos = np.arange(key_offset, key_offset + n_keys)[None, :]
+    ok = np.broadcast_to((kpos >= 0) & (kpos < Sk), (Sq, n_keys)).copy()
+    if right >= 0:
+        ok &= kpos <= qpos + right
+    if left >= 0:
+        ok &= kpos >= qpos - left
+    return ok
+
+
+# ---------------------------------------------------------------------------
+# forward: the plain definition
+# ---------------------------------------------------------------------------
+
+def _check_heads(Hq, Hkv):
+    if Hkv <= 0 or Hq % Hkv != 0:
+        raise ValueError(f"Hq={Hq} must be an integer multiple of Hkv={Hkv}")
+    return Hq // Hkv
+
+
+def raw_scores(q, k, scale, h, g):
+    """u[b, i, j] = scale * sum_d q[b,i,h,d] * k[b,j,g,d]  (float64)."""
+    return scale * np.einsum("bid,bjd->bij", q[:, :, h, :], k[:, :, g, :])
+
+
+def transform_scores(u, softcap):
+    """Apply the soft cap ``softcap * tanh(u / softcap)`` (off when <= 0)."""
+    if softcap is not None and softcap > 0:
+        return softcap * np.tanh(u / softcap)
+    return u
+
+
+def attn_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1,
+             softcap=0.0, return_probs=False):
+    """Exact attention O = softmax(transform(scale * Q K^T) + mask) V.
+
+    q: (B, Sq, Hq, D); k, v: (B, Sk, Hkv, D), any float dtype (upcast to f64).
+    Returns O (B, Sq, Hq, D) f64 and LSE (B, Hq, Sq) f64 (natural log).
+    With ``return_probs`` also returns P (B, Hq, Sq, Sk) and the raw
+    scores u (B, Hq, Sq, Sk).
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    G = _check_heads(Hq, Hkv)
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(D)
+    vis = visible(Sq, Sk, causal, window_left, window_right)
+    out = np.zeros((B, Sq, Hq, D))
+    lse = np.full((B, Hq, Sq), NEG_INF)
+    P_all = np.zeros((B, Hq, Sq, Sk)) if return_probs else None
+    U_all = np.zeros((B, Hq, Sq, Sk)) if return_probs else None
+    for h in range(Hq):
+        g = h // G
+        u = raw_scores(q, k, scale, h, g)              # (B, Sq, Sk)
+        s = transform_scores(u, softcap)
+        s = np.where(vis[None], s, NEG_INF)
+        any_vis = vis.any(axis=1)                       # (Sq,)
+        m = np.where(any_vis[None], s.max(axis=2), 0.0)  # row max over visible keys
+        e = np.where(vis[None], np.exp(s - m[:, :, None]), 0.0)
+        l = e.sum(axis=2)
+        row_lse = np.where(any_vis[None], m + np.log(np.where(l > 0, l, 1.0)), NEG_INF)
+        P = np.where(vis[None], np.exp(s - row_lse[:, :, None]), 0.0)
+        out[:, :, h, :] = np.einsum("bij,bjd->bid", P, v[:, :, g, :])
+        lse[:, h, :] = row_lse
+        if return_probs:
+            P_all[:, h] = P
+            U_all[:, h] = u
+    if return_probs:
+        return out, lse, P_all, U_all
+    return out, lse
+
+
+# ---------------------------------------------------------------------------
+# forward: the tiled online-softmax algorithm (pins attn_fwd, never the GPU)
+# ---------------------------------------------------------------------------
+
+def attn_fwd_online(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1,
+                    softcap=0.0, block=16):
+    """Same result as :func:`attn_fwd`, reached block by block.
+
+    Follows the page's description of the online softmax: walk the keys in
+    blocks, keep a running row maximum m and running sum l, and rescale the
+    partial output by exp(m_old - m_new) whenever the maximum grows.  The full
+    score matrix of a row is never formed.
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    G = _check_heads(Hq, Hkv)
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(D)
+    out = np.zeros((B, Sq, Hq, D))
+    lse = np.full((B, Hq, Sq), NEG_INF)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            m = np.full(Sq, NEG_INF)
+            l = np.zeros(Sq)
+            acc = np.zeros((Sq, D))
+            for j0 in range(0, Sk, block):
+                j1 = min(Sk, j0 + block)
+                vis = visible(Sq, Sk, causal, window_left, window_right, key_offset=j0, n_keys=j1 - j0)
+                u = scale * (q[b, :, h, :] @ k[b, j0:j1, g, :].T)
+                s = np.where(vis, transform_scores(u, softcap), NEG_INF)
+                m_blk = s.max(axis=1)
+                m_new = np.maximum(m, m_blk)
+                safe = np.isfinite(m_new)
+                alpha = np.where(safe & np.isfinite(m), np.exp(np.where(safe, m - m_new, 0.0)), 0.0)
+                p = np.where(vis & safe[:, None], np.exp(s - np.where(safe, m_new, 0.0)[:, None]), 0.0)
+                l = alpha * l + p.sum(axis=1)
+                acc = alpha[:, None] * acc + p @ v[b, j0:j1, g, :]
+                m = m_new
+            has = l > 0
+            out[b, :, h, :] = np.where(has[:, None], acc / np.where(has, l, 1.0)[:, None], 0.0)
+            lse[b, h, :] = np.where(has, m + np.log(np.where(has, l, 1.0)), NEG_INF)
+    return out, lse
+
+
+# ---------------------------------------------------------------------------
+# backward: chain rule on the materialised tensors
+# ---------------------------------------------------------------------------
+
+def attn_bwd(dout, q, k, v, scale=None, causal=False, window_left=-1, window_right=-1,
+             softcap=0.0):
+    """Gradients of L = sum(dout * O) with respect to q, k, v.
+
+    Steps (per q-head h reading kv-head g):
+      dV_g += P^T dO ; dP = dO V^T ; Delta_i = sum_j P_ij dP_ij ;
+      dS = P * (dP - Delta) ; dU = dS * (1 - tanh^2(u/softcap)) when capped ;
+      dQ = scale * dU K ; dK_g += scale * dU^T Q.
+    Returns dq, dk, dv (f64, shapes of q, k, v) and Delta (B, Hq, Sq).
+    """
+    dout = np.asarray(dout, np.float64)
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    G = _check_heads(Hq, Hkv)
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(D)
+    _, _, P, U = attn_fwd(q, k, v, scale, causal, window_left, window_right, softcap,
+                          return_probs=True)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    delta = np.zeros((B, Hq, Sq))
+    for h in range(Hq):
+        g = h // G
+        Ph = P[:, h]                                    # (B, Sq, Sk)
+        dO = dout[:, :, h, :]                           # (B, Sq, D)
+        dv[:, :, g, :] += np.einsum("bij,bid->bjd", Ph, dO)
+        dP = np.einsum("bid,bjd->bij", dO, v[:, :, g, :])
+        dl = (Ph * dP).sum(axis=2)                      # Delta
+        dS = Ph * (dP - dl[:, :, None])
+        if softcap is not None and softcap > 0:
+            t = np.tanh(U[:, h] / softcap)
+            dS = dS * (1.0 - t * t)
+        dq[:, :, h, :] = scale * np.einsum("bij,bjd->bid", dS, k[:, :, g, :])
+        dk[:, :, g, :] += scale * np.einsum("bij,bid->bjd", dS, q[:, :, h, :])
+        delta[:, h, :] = dl
+    return dq, dk, dv, delta
+
+
+# ---------------------------------------------------------------------------
+# incremental decoding with a (paged) KV cache
+# ---------------------------------------------------------------------------
+
+def cache_slot(b, pos, block_table, page_size):
+    """(page, slot) that holds token ``pos`` of sequence ``b``.
+
+    Without a block table the cache is contiguous per sequence and the
+    "page" is the sequence index itself.
+    """
+    if block_table is None:
+        return b, pos
+    return int(block_table[b, pos // page_size]), pos % page_size
+
+
+def kvcache_append(k_cache, v_cache, k_new, v_new, cache_seqlens, block_table=None,
+                   page_size=None):
+    """Write k_new/v_new (B, Snew, Hkv, D) at positions cache_seqlens[b] + t.
+
+    Returns new (k_cache, v_cache) arrays; the inputs are not modified.  The
+    caches are (num_pages, page_size, Hkv, D) with a block table, else
+    (B, max_seqlen, Hkv, D).
+    """
+    kc = np.array(k_cache, copy=True)
+    vc = np.array(v_cache, copy=True)
+    if k_new is None:
+        return kc, vc
+    B, Snew = k_new.shape[0], k_new.shape[1]
+    for b in range(B):
+        for t in range(Snew):
+            page, slot = cache_slot(b, int(cache_seqlens[b]) + t, block_table, page_size)
+            kc[page, slot] = k_new[b, t]
+            vc[page, slot] = v_new[b, t]
+    return kc, vc
+
+
+def gather_cache(cache, b, L, block_table=None, page_size=None):
+    """Contiguous (L, Hkv, D) view of the first L tokens of sequence b."""
+    rows = [cache[cache_slot(b, pos, block_table, page_size)] for pos in range(L)]
+    if not rows:
+        return np.zeros((0,) + cache.shape[2:], dtype=np.float64)
+    return np.stack(rows).astype(np.float64)
+
+
+def attn_with_kvcache(q, k_cache, v_cache, k_new=None, v_new=None, cache_seqlens=None,
+                      block_table=None, page_size=None, scale=None, causal=False,
+                      window_left=-1, window_right=-1, softcap=0.0):
+    """Append then attend: q (B, Sq, Hq, D) against each sequence's cache.
+
+    Sequence b attends over L_b = cache_seqlens[b] + Snew keys (Snew = 0 when
+    no new K/V is given), with the bottom-right alignment of
+    :func:`visible`.  Returns O (B, Sq, Hq, D), LSE (B, Hq, Sq) and the
+    updated caches.
+    """
+    q = np.asarray(q, np.float64)
+    B, Sq, Hq, D = q.shape
+    Snew = 0 if k_new is None else k_new.shape[1]
+    kc, vc = kvcache_append(k_cache, v_cache, k_new, v_new, cache_seqlens, block_table, page_size)
+    out = np.zeros((B, Sq, Hq, D))
+    lse = np.full((B, Hq, Sq), NEG_INF)
+    for b in range(B):
+        L = int(cache_seqlens[b]) + Snew
+        Kb = gather_cache(kc, b, L, block_table, page_size)[None]
+        Vb = gather_cache(vc, b, L, block_table, page_size)[None]
+        o, s = attn_fwd(q[b:b + 1], Kb, Vb, scale, causal, window_left, window_right, softcap)
+        out[b] = o[0]
+        lse[b] = s[0]
+    return out, lse, kc, vc
+
+
+# ---------------------------------------------------------------------------
+# KV splits and their combination
+# ---------------------------------------------------------------------------
+
+def split_token_ranges(L, unit, num_splits):
+    """Token range [t0, t1) of each of ``num_splits`` splits of L keys.
+
+    The keys are grouped in units of ``unit`` tokens (the cache page); split
+    s takes units ceil(s*P/n) .. ceil((s+1)*P/n) - 1 with P = ceil(L/unit).
+    Splits may be empty.
+    """
+    P = -(-L // unit)
+    out = []
+    for s in range(num_splits):
+        u0 = -(-(s * P) // num_splits)
+        u1 = -(-((s + 1) * P) // num_splits)
+        out.append((min(L, u0 * unit), min(L, u1 * unit)))
+    return out
+
+
+def attn_partial(q, K, V, t0, t1, scale, causal=False, window_left=-1, window_right=-1,
+                 softcap=0.0):
+    """Attention of q (Sq, Hq, D) over keys [t0, t1) of K, V (L, Hkv, D).
+
+    Masks use absolute positions in the full length L.  Returns the
+    split-normalised partial output (Sq, Hq, D) and its LSE (Hq, Sq); an
+    empty or fully masked split gives O = 0, LSE = -inf.
+    """
+    Sq, Hq, D = q.shape
+    L, Hkv = K.shape[0], K.shape[1]
+    G = _check_heads(Hq, Hkv)
+    o = np.zeros((Sq, Hq, D))
+    lse = np.full((Hq, Sq), NEG_INF)
+    if t1 <= t0:
+        return o, lse
+    vis = visible(Sq, L, causal, window_left, window_right, key_offset=t0, n_keys=t1 - t0)
+    for h in range(Hq):
+        g = h // G
+        u = scale * (q[:, h, :] @ K[t0:t1, g, :].T)
+        s = np.where(vis, transform_scores(u, softcap), NEG_INF)
+        anyv = vis.any(axis=1)
+        m = np.where(anyv, s.max(axis=1), 0.0)
+        e = np.where(vis, np.exp(s - m[:, None]), 0.0)
+        l = e.sum(axis=1)
+        o[:, h, :] = np.where(anyv[:, None], (e @ V[t0:t1, g, :]) / np.where(anyv, l, 1.0)[:, None], 0.0)
+        lse[h] = np.where(anyv, m + np.log(np.where(anyv, l, 1.0)), NEG_INF)
+    return o, lse
+
+
+def combine_splits(o_parts, lse_parts):
+    """Merge split results: LSE = ln sum_s e^{LSE_s}; O = sum_s e^{LSE_s-LSE} O_s.
+
+    o_parts (n, Sq, Hq, D); lse_parts (n, Hq, Sq).  All-empty rows give
+    O = 0, LSE = -inf.
+    """
+    o_parts = np.asarray(o_parts, np.float64)
+    lse_parts = np.asarray(lse_parts, np.float64)
+    m = lse_parts.max(axis=0)                               # (Hq, Sq)
+    finite = np.isfinite(m)
+    w = np.where(finite[None], np.exp(lse_parts - np.where(finite, m, 0.0)[None]), 0.0)
+    tot = w.sum(axis=0)
+    lse = np.where(finite, np.where(finite, m, 0.0) + np.log(np.where(finite, tot, 1.0)), NEG_INF)
+    wn = np.where(finite[None], w / np.where(finite, tot, 1.0)[None], 0.0)  # (n, Hq, Sq)
+    o = np.einsum("nhi,nihd->ihd", wn, o_parts)
+    return o, lse

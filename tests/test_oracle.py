@@ -1,0 +1,408 @@
+"""Pins for the float64 oracle, against what the pages and the mathematics fix.
+
+None of these compares the oracle with itself: each check is a closed form, a
+brute-force index rule, an invariant of the method (online softmax, GQA as
+repeated KV, paging, splits) or central finite differences.
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import attn64
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_examples.json")
+
+_NS = {"ln": math.log, "tanh": math.tanh, "atanh": math.atanh, "sqrt": math.sqrt,
+       "inf": math.inf, "__builtins__": {}}
+
+
+def _ev(x):
+    if isinstance(x, list):
+        return [_ev(e) for e in x]
+    return float(eval(x, _NS))  # expressions are fixture text: numbers, ln, tanh, atanh
+
+
+def _arr(x):
+    return np.array(_ev(x), dtype=np.float64)
+
+
+def _load():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+def _rand(shape, rng, amp=1.0):
+    return amp * rng.standard_normal(shape)
+
+
+# ---------------------------------------------------------------------------
+# hand-derived closed forms (tests/golden/hand_examples.json)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("ex", _load()["examples"], ids=lambda e: e["name"])
+def test_hand_examples_forward(ex):
+    q, k, v = _arr(ex["q"]), _arr(ex["k"]), _arr(ex["v"])
+    o, lse = oracle.attn_fwd(q, k, v, scale=_ev(ex["scale"]), causal=ex["causal"],
+                             window_left=ex["window"][0], window_right=ex["window"][1],
+                             softcap=_ev(ex["softcap"]))
+    np.testing.assert_allclose(o, _arr(ex["out"]), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse, _arr(ex["lse"]), rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("ex", _load()["backward"], ids=lambda e: e["name"])
+def test_hand_examples_backward(ex):
+    q, k, v, do = _arr(ex["q"]), _arr(ex["k"]), _arr(ex["v"]), _arr(ex["dout"])
+    kw = dict(scale=_ev(ex["scale"]), causal=ex["causal"], window_left=ex["window"][0],
+              window_right=ex["window"][1], softcap=_ev(ex["softcap"]))
+    o, _ = oracle.attn_fwd(q, k, v, **kw)
+    np.testing.assert_allclose(o, _arr(ex["out"]), atol=1e-13)
+    dq, dk, dv, delta = oracle.attn_bwd(do, q, k, v, **kw)
+    np.testing.assert_allclose(dq, _arr(ex["dq"]), atol=1e-13)
+    np.testing.assert_allclose(dk, _arr(ex["dk"]), atol=1e-13)
+    np.testing.assert_allclose(dv, _arr(ex["dv"]), atol=1e-13)
+    np.testing.assert_allclose(delta, _arr(ex["delta"]), atol=1e-13)
+
+
+@pytest.mark.parametrize("ex", _load()["kvcache"], ids=lambda e: e["name"])
+def test_hand_examples_kvcache(ex):
+    o, lse, kc, vc = oracle.attn_with_kvcache(
+        _arr(ex["q"]), _arr(ex["k_cache"]), _arr(ex["v_cache"]), _arr(ex["k_new"]),
+        _arr(ex["v_new"]), np.array(ex["cache_seqlens"]), np.array(ex["block_table"]),
+        ex["page_size"], scale=_ev(ex["scale"]), causal=ex["causal"])
+    np.testing.assert_allclose(o, _arr(ex["out"]), atol=1e-13)
+    np.testing.assert_allclose(lse, _arr(ex["lse"]), atol=1e-13)
+    np.testing.assert_array_equal(vc, _arr(ex["v_cache_after"]))
+
+
+# ---------------------------------------------------------------------------
+# softmax rows, masks
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal,wl,wr,cap", [(False, -1, -1, 0.0), (True, -1, -1, 0.0),
+                                              (True, 5, 0, 3.0), (False, 3, 2, 0.0)])
+def test_probability_rows(causal, wl, wr, cap):
+    rng = np.random.default_rng(0)
+    q, k, v = _rand((2, 13, 4, 8), rng), _rand((2, 13, 2, 8), rng), _rand((2, 13, 2, 8), rng)
+    _, lse, P, _ = oracle.attn_fwd(q, k, v, 0.3, causal, wl, wr, cap, return_probs=True)
+    vis = attn64.visible(13, 13, causal, wl, wr)
+    assert (P >= 0).all()
+    assert (P[..., ~vis] == 0).all()
+    np.testing.assert_allclose(P.sum(-1), 1.0, atol=1e-12)
+    assert np.isfinite(lse).all()
+
+
+def _brute_visible(Sq, Sk, causal, wl, wr):
+    """Index rule written out element by element, independent of numpy masks."""
+    off = Sk - Sq
+    out = set()
+    for i in range(Sq):
+        for j in range(Sk):
+            lo = -10**9 if wl < 0 else i + off - wl
+            hi = 10**9 if wr < 0 else i + off + wr
+            if causal:
+                hi = min(hi, i + off)
+            if lo <= j <= hi:
+                out.add((i, j))
+    return out
+
+
+@pytest.mark.parametrize("Sq,Sk", [(7, 7), (3, 9), (9, 3), (1, 5)])
+@pytest.mark.parametrize("causal,wl,wr", [(False, -1, -1), (True, -1, -1), (False, 2, 0),
+                                          (False, 1, 3), (True, 4, 5), (False, 0, 0),
+                                          (False, 100, 100)])
+def test_visible_matches_brute_force(Sq, Sk, causal, wl, wr):
+    m = attn64.visible(Sq, Sk, causal, wl, wr)
+    got = {(i, j) for i in range(Sq) for j in range(Sk) if m[i, j]}
+    assert got == _brute_visible(Sq, Sk, causal, wl, wr)
+
+
+def test_window_special_cases():
+    S = 11
+    none = attn64.visible(S, S)
+    assert none.all()
+    np.testing.assert_array_equal(attn64.visible(S, S, False, -1, -1), none)
+    np.testing.assert_array_equal(attn64.visible(S, S, False, S, S), none)
+    np.testing.assert_array_equal(attn64.visible(S, S, True), attn64.visible(S, S, False, -1, 0))
+    np.testing.assert_array_equal(attn64.visible(S, S, True), np.tril(np.ones((S, S), bool)))
+
+
+# ---------------------------------------------------------------------------
+# online softmax == two-pass
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("block", [16, 32, 128])
+@pytest.mark.parametrize("causal,wl,wr,cap", [(False, -1, -1, 0.0), (True, -1, -1, 0.0),
+                                              (True, 20, 0, 5.0), (False, 7, 9, 0.0)])
+def test_online_softmax_equals_two_pass(block, causal, wl, wr, cap):
+    rng = np.random.default_rng(1)
+    q = _rand((2, 40, 4, 16), rng, 2.0)
+    k = _rand((2, 77, 2, 16), rng, 2.0)
+    v = _rand((2, 77, 2, 16), rng)
+    o1, l1 = oracle.attn_fwd(q, k, v, 0.25, causal, wl, wr, cap)
+    o2, l2 = oracle.attn_fwd_online(q, k, v, 0.25, causal, wl, wr, cap, block=block)
+    np.testing.assert_allclose(o2, o1, rtol=0, atol=1e-12)
+    fin = np.isfinite(l1)
+    np.testing.assert_array_equal(fin, np.isfinite(l2))
+    np.testing.assert_allclose(l2[fin], l1[fin], rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# special cases with closed forms
+# ---------------------------------------------------------------------------
+
+def test_single_key():
+    rng = np.random.default_rng(2)
+    q, k, v = _rand((1, 5, 2, 8), rng), _rand((1, 1, 2, 8), rng), _rand((1, 1, 2, 8), rng)
+    o, lse = oracle.attn_fwd(q, k, v, 0.7)
+    np.testing.assert_allclose(o, np.broadcast_to(v, o.shape), atol=1e-14)
+    s00 = 0.7 * np.einsum("bihd,bjhd->bhi", q, k)
+    np.testing.assert_allclose(lse, s00, atol=1e-14)
+
+
+def test_identical_keys_give_uniform_weights():
+    rng = np.random.default_rng(3)
+    n = 9
+    q = _rand((1, 4, 1, 8), rng)
+    k = np.repeat(_rand((1, 1, 1, 8), rng), n, axis=1)
+    v = _rand((1, n, 1, 8), rng)
+    o, lse = oracle.attn_fwd(q, k, v, 0.5)
+    np.testing.assert_allclose(o[0, :, 0], np.broadcast_to(v[0, :, 0].mean(0), (4, 8)), atol=1e-14)
+    s = 0.5 * (q[0, :, 0] @ k[0, 0, 0])
+    np.testing.assert_allclose(lse[0, 0], s + math.log(n), atol=1e-13)
+
+
+def test_zero_query_is_uniform():
+    rng = np.random.default_rng(4)
+    k, v = _rand((1, 6, 1, 4), rng), _rand((1, 6, 1, 4), rng)
+    o, lse = oracle.attn_fwd(np.zeros((1, 2, 1, 4)), k, v, 1.0)
+    np.testing.assert_allclose(o[0, 0, 0], v[0, :, 0].mean(0), atol=1e-14)
+    np.testing.assert_allclose(lse, math.log(6), atol=1e-14)
+
+
+def test_softcap_limit_and_bound():
+    rng = np.random.default_rng(5)
+    q, k, v = _rand((1, 6, 2, 8), rng), _rand((1, 6, 2, 8), rng), _rand((1, 6, 2, 8), rng)
+    o0, l0, _, U = oracle.attn_fwd(q, k, v, 0.5, return_probs=True)
+    c = 1e4
+    o1, l1 = oracle.attn_fwd(q, k, v, 0.5, softcap=c)
+    # c*tanh(u/c) = u - u^3/(3c^2) + ...: scores move by at most max|u|^3/(3c^2)
+    bound = np.abs(U).max() ** 3 / (3 * c * c)
+    np.testing.assert_allclose(l1, l0, atol=4 * bound + 1e-14)
+    assert not np.allclose(oracle.attn_fwd(q, k, v, 0.5, softcap=0.5)[0], o0, atol=1e-3)
+    # capped scores stay inside [-c, c]
+    _, _, P, _ = oracle.attn_fwd(q * 50, k, v, 1.0, softcap=2.0, return_probs=True)
+    assert np.isfinite(P).all()
+
+
+def test_fully_masked_rows():
+    rng = np.random.default_rng(6)
+    q, k, v = _rand((1, 5, 1, 4), rng), _rand((1, 3, 1, 4), rng), _rand((1, 3, 1, 4), rng)
+    o, lse = oracle.attn_fwd(q, k, v, 1.0, causal=True)   # Sq > Sk: first 2 rows see nothing
+    assert np.isneginf(lse[0, 0, :2]).all() and np.isfinite(lse[0, 0, 2:]).all()
+    np.testing.assert_array_equal(o[0, :2], 0.0)
+    o2, l2 = oracle.attn_fwd_online(q, k, v, 1.0, causal=True, block=2)
+    np.testing.assert_allclose(o2, o, atol=1e-13)
+
+
+def test_gqa_requires_integer_multiple():
+    with pytest.raises(ValueError):
+        oracle.attn_fwd(np.zeros((1, 2, 3, 4)), np.zeros((1, 2, 2, 4)), np.zeros((1, 2, 2, 4)))
+
+
+# ---------------------------------------------------------------------------
+# GQA == MHA on repeated K/V (forward and backward)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 1), (8, 2), (6, 3)])
+def test_gqa_equals_repeated_kv(Hq, Hkv):
+    rng = np.random.default_rng(7)
+    G = Hq // Hkv
+    q, do = _rand((2, 9, Hq, 8), rng), _rand((2, 9, Hq, 8), rng)
+    k, v = _rand((2, 11, Hkv, 8), rng), _rand((2, 11, Hkv, 8), rng)
+    kr, vr = np.repeat(k, G, axis=2), np.repeat(v, G, axis=2)
+    kw = dict(scale=0.4, causal=True, window_left=5, window_right=0, softcap=2.0)
+    o, l = oracle.attn_fwd(q, k, v, **kw)
+    o_r, l_r = oracle.attn_fwd(q, kr, vr, **kw)
+    np.testing.assert_allclose(o, o_r, atol=1e-14)
+    np.testing.assert_allclose(l, l_r, atol=1e-14)
+    dq, dk, dv, _ = oracle.attn_bwd(do, q, k, v, **kw)
+    dq_r, dk_r, dv_r, _ = oracle.attn_bwd(do, q, kr, vr, **kw)
+    np.testing.assert_allclose(dq, dq_r, atol=1e-13)
+    np.testing.assert_allclose(dk, dk_r.reshape(2, 11, Hkv, G, 8).sum(3), atol=1e-13)
+    np.testing.assert_allclose(dv, dv_r.reshape(2, 11, Hkv, G, 8).sum(3), atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# gradients: central finite differences
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("S", [3, 5])
+@pytest.mark.parametrize("causal,wl,wr,cap", [(False, -1, -1, 0.0), (True, -1, -1, 0.0),
+                                              (False, 1, 1, 0.0), (True, 2, 0, 1.5)])
+def test_gradients_match_finite_differences(S, causal, wl, wr, cap):
+    rng = np.random.default_rng(10 + S)
+    q, k, v = _rand((1, S, 2, 4), rng), _rand((1, S, 1, 4), rng), _rand((1, S, 1, 4), rng)
+    do = _rand((1, S, 2, 4), rng)
+    kw = dict(scale=0.6, causal=causal, window_left=wl, window_right=wr, softcap=cap)
+
+    def loss(qq, kk, vv):
+        return float((oracle.attn_fwd(qq, kk, vv, **kw)[0] * do).sum())
+
+    dq, dk, dv, _ = oracle.attn_bwd(do, q, k, v, **kw)
+    h = 1e-6
+    for x, g in ((q, dq), (k, dk), (v, dv)):
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = [xp if x is t else t for t in (q, k, v)]
+            args_m = [xm if x is t else t for t in (q, k, v)]
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        err = np.linalg.norm(num - g) / max(np.linalg.norm(g), 1e-30)
+        assert err <= 1e-6, err
+
+
+def test_delta_identity():
+    rng = np.random.default_rng(20)
+    q, k, v = _rand((2, 7, 4, 8), rng), _rand((2, 7, 2, 8), rng), _rand((2, 7, 2, 8), rng)
+    do = _rand((2, 7, 4, 8), rng)
+    o, _ = oracle.attn_fwd(q, k, v, 0.3, True, 3, 0, 2.0)
+    _, _, _, delta = oracle.attn_bwd(do, q, k, v, 0.3, True, 3, 0, 2.0)
+    np.testing.assert_allclose(delta, np.einsum("bihd,bihd->bhi", do, o), atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# KV cache: paged == contiguous, append-then-attend == full attention
+# ---------------------------------------------------------------------------
+
+def _paged_setup(rng, B=3, Hq=4, Hkv=2, D=8, page=4, pps=5, Snew=2):
+    num_pages = B * pps + 3
+    bt = rng.permutation(num_pages)[: B * pps].reshape(B, pps)
+    seqlens = np.array([0, 7, pps * page - Snew])[:B]
+    kc = _rand((num_pages, page, Hkv, D), rng)
+    vc = _rand((num_pages, page, Hkv, D), rng)
+    kn, vn = _rand((B, Snew, Hkv, D), rng), _rand((B, Snew, Hkv, D), rng)
+    q = _rand((B, Snew, Hq, D), rng)
+    return q, kc, vc, kn, vn, seqlens, bt, page
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_paged_equals_contiguous(causal):
+    rng = np.random.default_rng(30)
+    q, kc, vc, kn, vn, seqlens, bt, page = _paged_setup(rng)
+    B, pps = bt.shape
+    # contiguous copy of every sequence's pages
+    kcc = np.stack([np.concatenate([kc[p] for p in bt[b]]) for b in range(B)])
+    vcc = np.stack([np.concatenate([vc[p] for p in bt[b]]) for b in range(B)])
+    o1, l1, kc1, _ = oracle.attn_with_kvcache(q, kc, vc, kn, vn, seqlens, bt, page, 0.5, causal)
+    o2, l2, kc2, _ = oracle.attn_with_kvcache(q, kcc, vcc, kn, vn, seqlens, None, None, 0.5, causal)
+    np.testing.assert_allclose(o1, o2, atol=1e-14)
+    np.testing.assert_allclose(l1, l2, atol=1e-14)
+    kcc1 = np.stack([np.concatenate([kc1[p] for p in bt[b]]) for b in range(B)])
+    np.testing.assert_array_equal(kcc1, kc2)
+
+
+def test_append_then_attend_equals_full_attention():
+    rng = np.random.default_rng(31)
+    q, kc, vc, kn, vn, seqlens, bt, page = _paged_setup(rng)
+    o, l, _, _ = oracle.attn_with_kvcache(q, kc, vc, kn, vn, seqlens, bt, page, 0.5, True, 3, 0, 1.5)
+    for b in range(bt.shape[0]):
+        L0 = int(seqlens[b])
+        Kold = np.array([kc[bt[b, t // page], t % page] for t in range(L0)]).reshape(L0, *kc.shape[2:])
+        Vold = np.array([vc[bt[b, t // page], t % page] for t in range(L0)]).reshape(L0, *vc.shape[2:])
+        Kfull = np.concatenate([Kold, kn[b]])
+        Vfull = np.concatenate([Vold, vn[b]])
+        # full self-attention over the concatenation; keep its last Snew rows
+        qfull = np.concatenate([np.zeros((L0,) + q.shape[2:]), q[b]])[None]
+        of, lf = oracle.attn_fwd(qfull, Kfull[None], Vfull[None], 0.5, True, 3, 0, 1.5)
+        np.testing.assert_allclose(o[b], of[0, L0:], atol=1e-14)
+        np.testing.assert_allclose(l[b], lf[0, :, L0:], atol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# splits: combine(partials) == unsplit
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("L", [1, 5, 37, 64])
+@pytest.mark.parametrize("n", [1, 4, 16])
+def test_split_combine_equals_unsplit(L, n):
+    rng = np.random.default_rng(40 + L)
+    q = _rand((2, 4, 8), rng)
+    K, V = _rand((L, 2, 8), rng), _rand((L, 2, 8), rng)
+    ranges = oracle.split_token_ranges(L, 4, n)
+    assert ranges[0][0] == 0 and ranges[-1][1] == L
+    assert all(ranges[i][1] == ranges[i + 1][0] for i in range(n - 1))
+    parts = [oracle.attn_partial(q, K, V, t0, t1, 0.5, True, 9, 0, 2.0) for t0, t1 in ranges]
+    o, lse = oracle.combine_splits([p[0] for p in parts], [p[1] for p in parts])
+    of, lf = oracle.attn_fwd(q[None], K[None], V[None], 0.5, True, 9, 0, 2.0)
+    np.testing.assert_allclose(o, of[0], atol=1e-12)
+    np.testing.assert_allclose(lse, lf[0], atol=1e-12)
+
+
+def test_split_ranges_page_aligned_with_empty_splits():
+    r = oracle.split_token_ranges(1, 256, 16)
+    assert sum(t1 - t0 for t0, t1 in r) == 1
+    assert sum(1 for t0, t1 in r if t1 > t0) == 1
+    r = oracle.split_token_ranges(32769, 256, 16)
+    assert all(t0 % 256 == 0 for t0, _ in r)
+    assert r[-1][1] == 32769
+
+
+# ---------------------------------------------------------------------------
+# planted mistakes: each must be caught by one of the pins above
+# ---------------------------------------------------------------------------
+
+def _hand(name, section="examples"):
+    return next(e for e in _load()[section] if e["name"] == name)
+
+
+def test_planted_clamp_softcap_is_caught(monkeypatch):
+    monkeypatch.setattr(attn64, "transform_scores",
+                        lambda u, c: np.clip(u, -c, c) if c and c > 0 else u)
+    with pytest.raises(AssertionError):
+        test_hand_examples_forward(_hand("softcap_tanh"))
+
+
+def test_planted_gqa_modulo_mapping_is_caught(monkeypatch):
+    orig = attn64.raw_scores
+
+    def bad_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1, softcap=0.0,
+                return_probs=False):
+        # q-head h reads kv-head h % Hkv instead of h // G
+        Hq, Hkv = q.shape[2], k.shape[2]
+        idx = [h % Hkv for h in range(Hq)]
+        return orig_fwd(q, k[:, :, idx], v[:, :, idx], scale, causal, window_left, window_right,
+                        softcap, return_probs)
+
+    orig_fwd = attn64.attn_fwd
+    assert orig is attn64.raw_scores
+    monkeypatch.setattr(oracle, "attn_fwd", bad_fwd)
+    with pytest.raises(AssertionError):
+        test_hand_examples_forward(_hand("gqa_head_mapping"))
+
+
+def test_planted_missing_scale_is_caught(monkeypatch):
+    monkeypatch.setattr(attn64, "raw_scores",
+                        lambda q, k, scale, h, g: np.einsum("bid,bjd->bij", q[:, :, h, :], k[:, :, g, :]))
+    with pytest.raises(AssertionError):
+        test_hand_examples_forward(_hand("rectangular_noncausal"))
+
+
+def test_planted_exclusive_window_is_caught(monkeypatch):
+    orig = attn64.visible
+
+    def excl(Sq, Sk, causal=False, window_left=-1, window_right=-1, key_offset=0, n_keys=None):
+        wl = window_left - 1 if window_left is not None and window_left > 0 else window_left
+        return orig(Sq, Sk, causal, wl, window_right, key_offset, n_keys)
+
+    monkeypatch.setattr(attn64, "visible", excl)
+    with pytest.raises(AssertionError):
+        test_hand_examples_forward(_hand("window_left1"))
