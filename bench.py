@@ -1,0 +1,518 @@
+#!/usr/bin/env python
+"""Throughput of the attention hot path on B200, one JSON line on rank 0.
+
+A step is one pass of the whole hot path over one batch of synthetic inputs:
+  * the seqlen sweep at hidden 2048 (H=32,D=64 and H=16,D=128; S = 512..16k,
+    B = 16384/S; causal and non-causal; bf16): forward + backward of each point;
+  * the GQA + local-attention workload (B=2, S=4096, Hq=32, Hkv=8, D=128,
+    window (1024,0), softcap 30): forward + backward;
+  * the paged KV-cache decode (B=8, Hq=32, Hkv=8, D=128, lengths U[1,32768],
+    page 256): append + split-KV attention + combine.
+``value`` is algorithmic attention TFLOP/s of the whole step (4*D flops per
+visible (query, key) pair forward, 10*D backward; decode flops counted the
+same way) with inputs resident in HBM.  Every tensor of a sweep point, the GQA
+workload and the KV cache is larger than L2 (126 MB per step working set far
+exceeds it), so L2 is not flushed.  Multi-GPU: every rank runs its own replica
+of the step (the work units are independent), value sums all ranks' flops
+over the max time across ranks.
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "attention TFLOPs/s fwd+bwd (seqlen sweep 512-16k d64/d128, GQA+local, paged decode)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work
+# ---------------------------------------------------------------------------
+
+def visible_pairs(Sq, Sk, causal, wl, wr):
+    """Number of visible (query, key) pairs of one head (bottom-right aligned)."""
+    if causal:
+        wr = 0
+    i = np.arange(Sq, dtype=np.int64) + (Sk - Sq)
+    lo = np.maximum(0, i - wl) if wl >= 0 else np.zeros_like(i)
+    hi = np.minimum(Sk - 1, i + wr) if wr >= 0 else np.full_like(i, Sk - 1)
+    return int(np.maximum(0, hi - lo + 1).sum())
+
+
+def attn_flops(cfg):
+    pairs = visible_pairs(cfg["Sq"], cfg["Sk"], cfg["causal"], cfg["window"][0], cfg["window"][1])
+    n = pairs * cfg["B"] * cfg["Hq"]
+    return 4 * cfg["D"] * n, 10 * cfg["D"] * n
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"fa_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                                          "-lms", "200", "-i", str(self.gpu_index)],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1].split()[0]), smax=float(parts[2].split()[0]),
+                                     power=float(parts[3].split()[0]) if parts[3][0].isdigit() else 0.0,
+                                     hw=parts[5], hwt=parts[6], swt=parts[7], swp=parts[8]))
+                except (ValueError, IndexError):
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("swp", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["smax"] for r in rows),
+                "samples": len(rows), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# workload units
+# ---------------------------------------------------------------------------
+
+class AttnUnit:
+    kind = "attn"
+
+    def __init__(self, cfg, dev, deterministic=False):
+        from exact_attention_121_b200 import api, inputs
+        self.api = api
+        self.cfg = cfg
+        self.det = deterministic
+        q, k, v, do = inputs.attention_inputs(cfg["B"], cfg["Sq"], cfg["Sk"], cfg["Hq"], cfg["Hkv"], cfg["D"],
+                                              cfg["dtype"], seed=cfg["seed"], amp=cfg.get("amp", 1.0))
+        self.host_in = (q, k, v, do)
+        self.q, self.k, self.v, self.do = (t.to(dev) for t in (q, k, v, do))
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty(cfg["B"], cfg["Hq"], cfg["Sq"], device=dev)
+        self.dq, self.dk, self.dv = torch.empty_like(self.q), torch.empty_like(self.k), torch.empty_like(self.v)
+        n = api.fa_bwd_workspace_size(cfg["B"], cfg["Sq"], cfg["Sk"], cfg["Hq"], cfg["Hkv"], cfg["D"], self.det)
+        self.ws = torch.empty(n, dtype=torch.uint8, device=dev)
+        self.flops_fwd, self.flops_bwd = attn_flops(cfg)
+        self.kw = dict(scale=cfg["scale"], causal=cfg["causal"], window=cfg["window"], softcap=cfg["softcap"])
+
+    def name(self):
+        c = self.cfg
+        return "H%dD%dS%d%s" % (c["Hq"], c["D"], c["Sq"], "c" if c["causal"] else "n")
+
+    def run(self, tracer):
+        api = self.api
+        tracer.arm("fwd", self)
+        api.fa_fwd(self.q, self.k, self.v, out=self.out, lse=self.lse, **self.kw)
+        n = api.fa_last_launch_count()
+        tracer.arm("bwd", self)
+        api.fa_bwd(self.do, self.q, self.k, self.v, self.out, self.lse, self.dq, self.dk, self.dv,
+                   deterministic=self.det, workspace=self.ws, **self.kw)
+        tracer.disarm()
+        return n + api.fa_last_launch_count()
+
+    def flops(self):
+        return self.flops_fwd + self.flops_bwd
+
+    # end-to-end: inputs from pinned host memory, outputs back to pinned host memory
+    def setup_e2e(self, pinned):
+        self.pin_in = [pinned.get(t, i) for i, t in enumerate(self.host_in)]
+        self.pin_out = [pinned.get_like(t) for t in (self.out, self.dq, self.dk, self.dv)]
+
+    def run_e2e(self, tracer):
+        for dst, src in zip((self.q, self.k, self.v, self.do), self.pin_in):
+            dst.copy_(src, non_blocking=True)
+        n = self.run(tracer)
+        for dst, src in zip(self.pin_out, (self.out, self.dq, self.dk, self.dv)):
+            dst.copy_(src, non_blocking=True)
+        return n
+
+    def e2e_bytes(self):
+        return (sum(t.numel() * t.element_size() for t in (self.q, self.k, self.v, self.do)),
+                sum(t.numel() * t.element_size() for t in (self.out, self.dq, self.dk, self.dv)))
+
+
+class DecodeUnit:
+    kind = "decode"
+
+    def __init__(self, cfg, dev, num_splits=0):
+        from exact_attention_121_b200 import api, inputs
+        self.api = api
+        self.cfg = cfg
+        self.num_splits = num_splits
+        d = inputs.kvcache_inputs(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["D"], cfg["page_size"],
+                                  cfg["pages_per_seq"], cfg["max_len"], Sq=1, Snew=1, dtype=cfg["dtype"],
+                                  seed=cfg["seed"])
+        self.host_in = (d["q"], d["k_new"], d["v_new"])
+        self.q, self.kn, self.vn = (t.to(dev) for t in self.host_in)
+        self.kc, self.vc = d["k_cache"].to(dev), d["v_cache"].to(dev)
+        self.sl, self.bt = d["cache_seqlens"].to(dev), d["block_table"].to(dev)
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty(cfg["B"], cfg["Hq"], 1, device=dev)
+        n = api.fa_kvcache_workspace_size(cfg["B"], 1, cfg["Hq"], cfg["D"], num_splits)
+        self.ws = torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
+        lens = d["cache_seqlens"].numpy().astype(np.int64) + 1
+        # algorithmic bytes: every attended K and V row once, plus q/out/new rows and the block table
+        row = cfg["Hkv"] * cfg["D"] * 2
+        self.bytes = int(2 * lens.sum() * row + 2 * self.q.numel() * 2 + 2 * self.kn.numel() * 2
+                         + d["block_table"].numel() * 4 + lens.size * 4)
+        self.flops_dec = int(4 * cfg["D"] * cfg["Hq"] * lens.sum())
+
+    def name(self):
+        return "decode"
+
+    def run(self, tracer):
+        tracer.arm("decode", self)
+        self.api.fa_fwd_kvcache(self.q, self.kc, self.vc, self.kn, self.vn, self.sl, self.bt,
+                                page_size=self.cfg["page_size"], out=self.out, lse=self.lse,
+                                scale=self.cfg["scale"], causal=True, num_splits=self.num_splits,
+                                workspace=self.ws)
+        tracer.disarm()
+        return self.api.fa_last_launch_count()
+
+    def flops(self):
+        return self.flops_dec
+
+    def setup_e2e(self, pinned):
+        self.pin_in = [pinned.get(t, i) for i, t in enumerate(self.host_in)]
+        self.pin_out = [pinned.get_like(self.out)]
+
+    def run_e2e(self, tracer):
+        for dst, src in zip((self.q, self.kn, self.vn), self.pin_in):
+            dst.copy_(src, non_blocking=True)
+        n = self.run(tracer)
+        self.pin_out[0].copy_(self.out, non_blocking=True)
+        return n
+
+    def e2e_bytes(self):
+        return (sum(t.numel() * t.element_size() for t in (self.q, self.kn, self.vn)),
+                self.out.numel() * self.out.element_size())
+
+
+class Pinned:
+    """Pinned host staging buffers, shared between units of equal byte size."""
+
+    def __init__(self):
+        self.pool = {}
+
+    def _buf(self, nbytes, tag):
+        key = (nbytes, tag)
+        if key not in self.pool:
+            self.pool[key] = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+        return self.pool[key]
+
+    def get(self, t, slot):
+        nb = t.numel() * t.element_size()
+        buf = self._buf(nb, "in%d" % slot)
+        view = buf.view(t.dtype).view(t.shape)
+        view.copy_(t)
+        return view
+
+    def get_like(self, t):
+        nb = t.numel() * t.element_size()
+        return self._buf(nb, "out%d" % nb).view(t.dtype).view(t.shape)
+
+
+class Tracer:
+    """Per-call CUDA event pairs around each call's dominant kernel (set through
+    fa_set_trace_events), accumulated per kernel class over the timed region."""
+
+    def __init__(self, lib, enabled=False):
+        self.lib = lib
+        self.enabled = enabled
+        self.pending = []
+        self.totals = {}
+
+    def arm(self, cls, unit):
+        if not self.enabled:
+            return
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        b.record()
+        self.lib.fa_set_trace_events(a.cuda_event, b.cuda_event)
+        work = {"fwd": getattr(unit, "flops_fwd", 0), "bwd": getattr(unit, "flops_bwd", 0),
+                "decode": getattr(unit, "bytes", 0)}[cls]
+        self.pending.append((cls, a, b, work))
+
+    def disarm(self):
+        if self.enabled:
+            self.lib.fa_set_trace_events(None, None)
+
+    def collect(self):
+        for cls, a, b, work in self.pending:
+            ms = a.elapsed_time(b)
+            t = self.totals.setdefault(cls, [0.0, 0, 0])
+            t[0] += ms
+            t[1] += 1
+            t[2] += work
+        self.pending = []
+        return self.totals
+
+
+# ---------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------
+
+def build_units(dev, workload):
+    from exact_attention_121_b200 import inputs
+    units = []
+    if workload in ("full", "sweep"):
+        for cfg in inputs.seqlen_sweep_configs():
+            units.append(AttnUnit(cfg, dev))
+    if workload in ("full", "gqa"):
+        units.append(AttnUnit(inputs.gqa_local_config(), dev))
+    if workload in ("full", "decode"):
+        units.append(DecodeUnit(inputs.paged_decode_config(), dev))
+    if workload == "small":
+        units.append(AttnUnit(inputs.fwd_bwd_512_config(), dev))
+    return units
+
+
+def time_steps(units, steps, warmup, tracer, e2e=False, barrier=None):
+    stream = torch.cuda.current_stream()
+    launches = 0
+    for _ in range(warmup):
+        for u in units:
+            (u.run_e2e if e2e else u.run)(Tracer(tracer.lib))
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        for u in units:
+            launches += (u.run_e2e if e2e else u.run)(tracer)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    return start.elapsed_time(stop), launches
+
+
+def cpu_oracle_sample(budget_s=12.0):
+    """Time the float64 oracle on head slices of the seqlen-sweep point S=2048,
+    D=128 (forward + backward) for about budget_s seconds; TFLOP/s."""
+    import oracle
+    from exact_attention_121_b200 import inputs
+    cfg = next(c for c in inputs.seqlen_sweep_configs() if c["Sq"] == 2048 and c["D"] == 128 and c["causal"])
+    q, k, v, do = inputs.attention_inputs(cfg["B"], cfg["Sq"], cfg["Sk"], cfg["Hq"], cfg["Hkv"], cfg["D"],
+                                          cfg["dtype"], seed=cfg["seed"])
+    f = lambda t, b, h: t[b:b + 1, :, h:h + 1].double().numpy()
+    one = dict(cfg, B=1, Hq=1, Hkv=1)
+    flops = sum(attn_flops(one))
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        b, h = n % cfg["B"], (n // cfg["B"]) % cfg["Hq"]
+        oracle.attn_fwd(f(q, b, h), f(k, b, h), f(v, b, h), cfg["scale"], cfg["causal"])
+        oracle.attn_bwd(f(do, b, h), f(q, b, h), f(k, b, h), f(v, b, h), cfg["scale"], cfg["causal"])
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:  # noqa: BLE001
+        cores = os.cpu_count()
+    return dict(value=n * flops / el / 1e12, unit="TFLOP/s", cores=int(cores), kind="oracle",
+                sample=f"{n} (batch, head) slices of the S=2048 D=128 causal sweep point, fwd+bwd in float64, "
+                       f"{el:.1f} s", elapsed_s=el, flops=n * flops)
+
+
+def reference_arm(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    for _ in range(args.warmup):
+        cpu_oracle_sample(budget_s=0.0)
+    samples = [cpu_oracle_sample(budget_s=0.0) for _ in range(args.steps)]
+    total_s = sum(s["elapsed_s"] for s in samples)
+    value = sum(s["flops"] for s in samples) / total_s / 1e12
+    cb = {k: samples[0][k] for k in ("unit", "cores", "kind")}
+    cb["value"] = value
+    cb["sample"] = f"each step: one (batch, head) slice of the S=2048 D=128 causal sweep point, fwd+bwd in float64"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total_s / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": "oracle on sampled slices of the step's workload"},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="full", choices=["full", "sweep", "gqa", "decode", "small"])
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--detail", action="store_true", help="also print per-unit times")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    def barrier():
+        if pg:
+            pg.barrier()
+
+    from exact_attention_121_b200 import _lib
+    lib = _lib.load()
+    units = build_units(dev, args.workload)
+    flops_step = sum(u.flops() for u in units)
+    peaks, peak_src = load_peaks()
+
+    # device-resident timing with per-kernel trace events
+    tracer = Tracer(lib, enabled=True)
+    gidx = os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local] if "CUDA_VISIBLE_DEVICES" in os.environ else str(local)
+    clocks = ClockSampler(gidx)
+    clocks.start()
+    ms, launches = time_steps(units, args.steps, args.warmup, tracer, barrier=barrier)
+    clk = clocks.stop()
+    totals = tracer.collect()
+    ms_max = ms
+    if pg:
+        t = torch.tensor([ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms_max = float(t.item())
+    value = world * flops_step * args.steps / (ms_max / 1e3) / 1e12
+
+    # per-unit detail (untimed for the headline; separate short pass)
+    detail = {}
+    if args.detail and rank == 0:
+        for u in units:
+            tr = Tracer(lib, enabled=True)
+            t_ms, _ = time_steps([u], 3, 1, tr)
+            tt = tr.collect()
+            d = {"ms": t_ms / 3, "tflops": u.flops() / (t_ms / 3 / 1e3) / 1e12}
+            for cls, (kms, cnt, work) in tt.items():
+                d[cls + "_ms"] = kms / cnt
+                d[cls + ("_gbs" if cls == "decode" else "_tflops")] = (work / cnt) / (kms / cnt / 1e3) / (1e9 if cls == "decode" else 1e12)
+            detail[u.name()] = d
+
+    # end to end through the C ABI with pinned host buffers
+    pinned = Pinned()
+    for u in units:
+        u.setup_e2e(pinned)
+    h2d = sum(u.e2e_bytes()[0] for u in units)
+    d2h = sum(u.e2e_bytes()[1] for u in units)
+    ms_e2e, _ = time_steps(units, args.e2e_steps, 1, Tracer(lib), e2e=True, barrier=barrier)
+    if pg:
+        t = torch.tensor([ms_e2e], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    e2e_value = world * flops_step * args.e2e_steps / (ms_e2e / 1e3) / 1e12
+
+    # roofline of the dominant kernel class (largest traced time)
+    dom = max(totals.items(), key=lambda kv: kv[1][0])
+    cls, (kms, cnt, work) = dom
+    if cls == "decode":
+        achieved = work / (kms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None}
+    else:
+        achieved = work / (kms / 1e3) / 1e12
+        pk = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
+                "frac": achieved / pk, "traffic": None}
+    roof["kernel"] = {"fwd": "forward attention kernel", "bwd": "main backward kernel (dK/dV/dQ)",
+                      "decode": "split-KV decode kernel"}[cls]
+    roof["peak_source"] = f"{peak_src} ({'bf16_tflops_sustained' if cls != 'decode' else 'hbm_gbs'})"
+    kernels = {c: {"ms_total": v[0], "launches": v[1],
+                   ("gbs" if c == "decode" else "tflops"): v[2] / (v[0] / 1e3) / (1e9 if c == "decode" else 1e12)}
+               for c, v in totals.items()}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_sample()
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": args.workload + ": " + ", ".join(u.name() for u in units),
+                           "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}",
+                           "flops_per_step": flops_step},
+                "gpu_launches": launches,
+                "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h, "steps": args.e2e_steps},
+                "roofline": roof, "kernels": kernels, "cpu_baseline": cpu,
+                "clocks": clk}
+        if detail:
+            line["detail"] = detail
+        print(json.dumps(line))
+    if pg:
+        pg.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

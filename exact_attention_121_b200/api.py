@@ -1,0 +1,162 @@
+"""Thin PyTorch-facing binding of libfa.so with the C entry points' names.
+
+PyTorch supplies device memory and the current CUDA stream; every step of the
+computation runs in the library's kernels.  Tensors are (batch, seqlen,
+nheads, headdim), contiguous, fp16 or bf16, on one CUDA device.  There is no
+CPU or fallback path: if libfa.so is missing, the import of ``_lib`` fails.
+"""
+
+import ctypes
+
+import torch
+
+from . import _lib
+
+_DT = {torch.float16: _lib.FA_FP16, torch.bfloat16: _lib.FA_BF16}
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_tensor(t, name, dtype=None, device=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _window(window):
+    wl, wr = (-1, -1) if window is None else window
+    return int(wl), int(wr)
+
+
+def fa_status_string(code):
+    return _lib.load().fa_status_string(int(code)).decode()
+
+
+def fa_set_fwd_kernel(which):
+    """0 = automatic (tcgen05 where it applies), 1 = force the mma.sync kernel."""
+    _lib.load().fa_set_fwd_kernel(int(which))
+
+
+def fa_last_launch_count():
+    return int(_lib.load().fa_last_launch_count())
+
+
+def fa_fwd(q, k, v, out=None, lse=None, scale=None, causal=False, window=(-1, -1), softcap=0.0,
+           stream=None):
+    """Forward attention; returns (out, lse).  lse is fp32 (B, Hq, Sq)."""
+    lib = _lib.load()
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    dt = q.dtype
+    if dt not in _DT:
+        raise ValueError(f"unsupported dtype {dt}")
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _check_tensor(t, n, dt, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    _check_tensor(lse, "lse", torch.float32, q.device)
+    wl, wr = _window(window)
+    code = lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq, Sk, Hq, Hkv, D, _DT[dt],
+                      float(scale or 0.0), int(bool(causal)), wl, wr, float(softcap or 0.0),
+                      _stream(stream))
+    _lib.check(code, "fa_fwd")
+    return out, lse
+
+
+def fa_bwd_workspace_size(B, Sq, Sk, Hq, Hkv, D, deterministic=False):
+    return int(_lib.load().fa_bwd_workspace_size(B, Sq, Sk, Hq, Hkv, D, int(bool(deterministic))))
+
+
+def fa_bwd(dout, q, k, v, out, lse, dq=None, dk=None, dv=None, scale=None, causal=False,
+           window=(-1, -1), softcap=0.0, deterministic=False, workspace=None, stream=None):
+    """Backward attention; returns (dq, dk, dv)."""
+    lib = _lib.load()
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    dt = q.dtype
+    for t, n in ((dout, "dout"), (q, "q"), (k, "k"), (v, "v"), (out, "out"), (dq, "dq"), (dk, "dk"),
+                 (dv, "dv")):
+        _check_tensor(t, n, dt, q.device)
+    _check_tensor(lse, "lse", torch.float32, q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = fa_bwd_workspace_size(B, Sq, Sk, Hq, Hkv, D, deterministic)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    wl, wr = _window(window)
+    code = lib.fa_bwd(_ptr(dout), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dq), _ptr(dk),
+                      _ptr(dv), B, Sq, Sk, Hq, Hkv, D, _DT[dt], float(scale or 0.0),
+                      int(bool(causal)), wl, wr, float(softcap or 0.0), int(bool(deterministic)),
+                      _ptr(workspace), workspace.numel(), _stream(stream))
+    _lib.check(code, "fa_bwd")
+    return dq, dk, dv
+
+
+def fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits):
+    return int(_lib.load().fa_kvcache_workspace_size(B, Sq, Hq, D, int(num_splits)))
+
+
+def fa_fwd_kvcache(q, k_cache, v_cache, k_new=None, v_new=None, cache_seqlens=None, block_table=None,
+                   page_size=256, out=None, lse=None, scale=None, causal=False, window=(-1, -1),
+                   softcap=0.0, num_splits=0, workspace=None, stream=None, return_lse=True):
+    """Append k_new/v_new into the cache (in place), then attend; returns (out, lse).
+
+    Paged when ``block_table`` (B, max_pages_per_seq) int32 is given: caches
+    are (num_pages, page_size, Hkv, D).  Otherwise caches are
+    (B, max_seqlen, Hkv, D).  ``cache_seqlens`` (B,) int32 is the length
+    before the append and is not modified.
+    """
+    lib = _lib.load()
+    B, Sq, Hq, D = q.shape
+    Hkv = k_cache.shape[2]
+    dt = q.dtype
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (k_new, "k_new"),
+                 (v_new, "v_new"), (out, "out")):
+        _check_tensor(t, n, dt, q.device)
+    _check_tensor(cache_seqlens, "cache_seqlens", torch.int32, q.device)
+    _check_tensor(block_table, "block_table", torch.int32, q.device)
+    Snew = 0 if k_new is None else k_new.shape[1]
+    if block_table is not None:
+        max_pages_per_seq = block_table.shape[1]
+        cap = k_cache.shape[0]
+        page_size = k_cache.shape[1]
+    else:
+        max_pages_per_seq = 0
+        cap = k_cache.shape[1]
+    out = torch.empty_like(q) if out is None else out
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    need = fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wl, wr = _window(window)
+    code = lib.fa_fwd_kvcache(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_new), _ptr(v_new),
+                              _ptr(cache_seqlens), _ptr(block_table), int(page_size), int(max_pages_per_seq),
+                              int(cap), _ptr(out), _ptr(lse), B, Sq, Snew, Hq, Hkv, D, _DT[dt],
+                              float(scale or 0.0), int(bool(causal)), wl, wr, float(softcap or 0.0),
+                              int(num_splits), _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                              _stream(stream))
+    _lib.check(code, "fa_fwd_kvcache")
+    return out, lse
+
+
+def fa_last_device_status(stream=None):
+    """Wait for the stream; return and clear the device status word (an int)."""
+    return int(_lib.load().fa_last_device_status(_stream(stream)))

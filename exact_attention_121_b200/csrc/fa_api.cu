@@ -1,0 +1,287 @@
+// Host side of the C ABI declared in include/fa.h: argument validation,
+// workspace sizing and carving, the device status word, and kernel dispatch.
+// Nothing here allocates, frees or synchronises (except fa_last_device_status,
+// whose job is to wait and read the status word).
+#include <math.h>
+#include <stdint.h>
+
+#include "fa.h"
+#include "fa_common.cuh"
+#include "fa_kernels.h"
+
+namespace fa {
+int bwd_num_qblocks(int Sq);
+}
+
+namespace {
+
+// Device status word: bounded waits and device-side argument checks record
+// their failure here; fa_last_device_status reads and clears it.
+__device__ int g_fa_status = 0;
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {nullptr};
+int g_fwd_kernel_choice = 0;
+cudaEvent_t g_trace_start = nullptr, g_trace_stop = nullptr;
+thread_local int g_last_launches = 0;
+
+int* status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fa_status) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+fa_status check_common(int B, int Sq, int Hq, int Hkv, int D, fa_dtype dt, float scale, float softcap) {
+  if (B < 0 || Sq < 0 || Hq <= 0 || Hkv <= 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (dt != FA_FP16 && dt != FA_BF16) return FA_ERR_INVALID_ARG;
+  if (isnan(scale) || isinf(scale) || isnan(softcap) || isinf(softcap)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (B > 65535 || Hq > 65535) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+void fold_window(int causal, int window_left, int window_right, int* wl, int* wr) {
+  *wl = window_left < 0 ? -1 : window_left;
+  *wr = window_right < 0 ? -1 : window_right;
+  if (causal) *wr = 0;
+}
+
+float resolve_scale(float scale, int D) { return scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(D)); }
+
+void fill_cap(float scale, float softcap, float* cap, float* cap_in, float* cap_log2, float* scale_log2) {
+  const float log2e = 1.4426950408889634f;
+  *scale_log2 = scale * log2e;
+  if (softcap > 0.f) {
+    *cap = softcap;
+    *cap_in = scale / softcap;
+    *cap_log2 = softcap * log2e;
+  } else {
+    *cap = 0.f;
+    *cap_in = 0.f;
+    *cap_log2 = 0.f;
+  }
+}
+
+// Waits (bounded) for *flag == expected with the same helper the ordered
+// backward uses; records FA_ERR_TIMEOUT in the status word when it runs out.
+__global__ void selftest_wait_kernel(const int* flag, int expected, unsigned long long limit_ns, int* status) {
+  if (threadIdx.x == 0 && !fa::wait_eq_bounded(flag, expected, limit_ns)) fa::report_status(status, FA_ERR_TIMEOUT);
+}
+
+}  // namespace
+
+namespace fa {
+void trace_begin(cudaStream_t s) {
+  if (g_trace_start) cudaEventRecord(g_trace_start, s);
+}
+void trace_end(cudaStream_t s) {
+  if (g_trace_stop) cudaEventRecord(g_trace_stop, s);
+}
+}  // namespace fa
+
+extern "C" {
+
+void fa_set_trace_events(void* start_event, void* stop_event) {
+  g_trace_start = static_cast<cudaEvent_t>(start_event);
+  g_trace_stop = static_cast<cudaEvent_t>(stop_event);
+}
+
+fa_status fa_selftest_bounded_wait(const int* flag, int expected, long long limit_ns, fa_stream_t stream) {
+  g_last_launches = 0;
+  if (!flag || limit_ns < 0 || (reinterpret_cast<uintptr_t>(flag) & 3u)) return FA_ERR_INVALID_ARG;
+  int* st = status_ptr();
+  if (!st) return FA_ERR_CUDA;
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(flag, expected, static_cast<unsigned long long>(limit_ns), st);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  g_last_launches = 1;
+  return FA_OK;
+}
+
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+  }
+  return "FA_ERR_UNKNOWN";
+}
+
+void fa_set_fwd_kernel(int which) { g_fwd_kernel_choice = which; }
+
+int fa_last_launch_count(void) { return g_last_launches; }
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk,
+                 int Hq, int Hkv, int D, fa_dtype dt, float scale, int causal, int window_left, int window_right,
+                 float softcap, fa_stream_t stream) {
+  g_last_launches = 0;
+  fa_status st = check_common(B, Sq, Hq, Hkv, D, dt, scale, softcap);
+  if (st != FA_OK) return st;
+  if (Sk < 0) return FA_ERR_INVALID_ARG;
+  if (B == 0 || Sq == 0) return FA_OK;
+  if (!q || !out || !lse) return FA_ERR_INVALID_ARG;
+  if (Sk > 0 && (!k || !v)) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return FA_ERR_INVALID_ARG;
+  fa::FwdParams p{};
+  p.q = q; p.k = k; p.v = v; p.o = out; p.lse = lse;
+  p.B = B; p.Sq = Sq; p.Sk = Sk; p.Hq = Hq; p.Hkv = Hkv; p.D = D; p.G = Hq / Hkv;
+  fold_window(causal, window_left, window_right, &p.wl, &p.wr);
+  scale = resolve_scale(scale, D);
+  fill_cap(scale, softcap, &p.softcap, &p.cap_in, &p.cap_log2, &p.scale_log2);
+  p.status = status_ptr();
+  if (!p.status) return FA_ERR_CUDA;
+  int launches = 0;
+  cudaError_t e;
+  if (g_fwd_kernel_choice == 0 && fa::fwd_tc_supported(p))
+    e = fa::launch_fwd_tc(p, dt, stream, &launches);
+  else
+    e = fa::launch_fwd_mma(p, dt, stream, &launches);
+  g_last_launches = launches;
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_bwd_workspace_size(int B, int Sq, int Sk, int Hq, int Hkv, int D, int deterministic) {
+  if (B < 0 || Sq < 0 || Sk < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || (D != 64 && D != 128)) return 0;
+  size_t n = round256((size_t)B * Sq * Hq * D * sizeof(float));   // dQ accumulator
+  n += round256((size_t)B * Hq * Sq * sizeof(float));               // Delta
+  if (deterministic) n += round256(((size_t)B * Hq * fa::bwd_num_qblocks(Sq) + 1) * sizeof(int));
+  return n;
+}
+
+fa_status fa_bwd(const void* dout, const void* q, const void* k, const void* v, const void* out, const float* lse,
+                 void* dq, void* dk, void* dv, int B, int Sq, int Sk, int Hq, int Hkv, int D, fa_dtype dt,
+                 float scale, int causal, int window_left, int window_right, float softcap, int deterministic,
+                 void* workspace, size_t ws_bytes, fa_stream_t stream) {
+  g_last_launches = 0;
+  fa_status st = check_common(B, Sq, Hq, Hkv, D, dt, scale, softcap);
+  if (st != FA_OK) return st;
+  if (Sk < 0) return FA_ERR_INVALID_ARG;
+  if (B == 0 || (Sq == 0 && Sk == 0)) return FA_OK;
+  const void* ptrs[] = {dout, q, k, v, out, lse, dq, dk, dv, workspace};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return FA_ERR_INVALID_ARG;
+  if (Sq > 0 && (!dout || !q || !out || !lse || !dq)) return FA_ERR_INVALID_ARG;
+  if (Sk > 0 && (!k || !v || !dk || !dv)) return FA_ERR_INVALID_ARG;
+  const size_t need = fa_bwd_workspace_size(B, Sq, Sk, Hq, Hkv, D, deterministic);
+  if (ws_bytes < need || (need > 0 && !workspace)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
+  fa::BwdParams p{};
+  p.dout = dout; p.q = q; p.k = k; p.v = v; p.o = out; p.lse = lse; p.dq = dq; p.dk = dk; p.dv = dv;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.dq_accum = reinterpret_cast<float*>(ws);
+  ws += round256((size_t)B * Sq * Hq * D * sizeof(float));
+  p.delta = reinterpret_cast<float*>(ws);
+  ws += round256((size_t)B * Hq * Sq * sizeof(float));
+  if (deterministic) {
+    p.sem = reinterpret_cast<int*>(ws);
+    p.work_counter = p.sem + (size_t)B * Hq * fa::bwd_num_qblocks(Sq);
+  }
+  p.B = B; p.Sq = Sq; p.Sk = Sk; p.Hq = Hq; p.Hkv = Hkv; p.D = D; p.G = Hq / Hkv;
+  fold_window(causal, window_left, window_right, &p.wl, &p.wr);
+  scale = resolve_scale(scale, D);
+  p.scale = scale;
+  fill_cap(scale, softcap, &p.softcap, &p.cap_in, &p.cap_log2, &p.scale_log2);
+  p.deterministic = deterministic ? 1 : 0;
+  p.status = status_ptr();
+  if (!p.status) return FA_ERR_CUDA;
+  int launches = 0;
+  cudaError_t e = fa::launch_bwd(p, dt, stream, &launches);
+  g_last_launches = launches;
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_kvcache_workspace_size(int B, int Sq, int Hq, int D, int num_splits) {
+  if (B < 0 || Sq < 0 || Hq <= 0 || (D != 64 && D != 128)) return 0;
+  if (num_splits <= 0 || num_splits > FA_MAX_SPLITS) num_splits = FA_MAX_SPLITS;
+  if (num_splits == 1) return 0;
+  const size_t rows = (size_t)num_splits * B * Hq * Sq;
+  return round256(rows * D * sizeof(float)) + round256(rows * sizeof(float));
+}
+
+fa_status fa_fwd_kvcache(const void* q, void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                         const int* cache_seqlens, const int* block_table, int page_size, int max_pages_per_seq,
+                         int num_pages_or_max_seqlen, void* out, float* lse, int B, int Sq, int Snew, int Hq,
+                         int Hkv, int D, fa_dtype dt, float scale, int causal, int window_left, int window_right,
+                         float softcap, int num_splits, void* workspace, size_t ws_bytes, fa_stream_t stream) {
+  g_last_launches = 0;
+  fa_status st = check_common(B, Sq, Hq, Hkv, D, dt, scale, softcap);
+  if (st != FA_OK) return st;
+  if (Snew < 0 || page_size <= 0 || num_pages_or_max_seqlen < 0) return FA_ERR_INVALID_ARG;
+  if (num_splits > FA_MAX_SPLITS) return FA_ERR_INVALID_ARG;
+  if (B == 0 || Sq == 0) return FA_OK;
+  if (!q || !k_cache || !v_cache || !cache_seqlens || !out) return FA_ERR_INVALID_ARG;
+  if (Snew > 0 && (!k_new || !v_new)) return FA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k_cache, v_cache, k_new, v_new, out, lse};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cache_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(block_table) & 3u))
+    return FA_ERR_INVALID_ARG;
+  const bool paged = block_table != nullptr;
+  if (paged && max_pages_per_seq <= 0) return FA_ERR_INVALID_ARG;
+  fa::DecodeParams p{};
+  p.q = q; p.k_cache = k_cache; p.v_cache = v_cache; p.k_new = k_new; p.v_new = v_new;
+  p.cache_seqlens = cache_seqlens; p.block_table = block_table;
+  p.page_size = page_size; p.paged = paged ? 1 : 0;
+  p.max_pages_per_seq = paged ? max_pages_per_seq : 0;
+  p.capacity_pages = paged ? num_pages_or_max_seqlen : 0;
+  p.max_seqlen = paged ? 0 : num_pages_or_max_seqlen;
+  p.out = out; p.lse = lse;
+  p.B = B; p.Sq = Sq; p.Snew = Snew; p.Hq = Hq; p.Hkv = Hkv; p.D = D; p.G = Hq / Hkv;
+  fold_window(causal, window_left, window_right, &p.wl, &p.wr);
+  scale = resolve_scale(scale, D);
+  fill_cap(scale, softcap, &p.softcap, &p.cap_in, &p.cap_log2, &p.scale_log2);
+  // Split count: explicit, else enough (b, kv-head, split) work items for two
+  // waves over the SMs, never more splits than pages of the longest sequence.
+  const int cap_tokens = paged ? max_pages_per_seq * page_size : num_pages_or_max_seqlen;
+  const int max_units = (cap_tokens + page_size - 1) / page_size;
+  if (num_splits <= 0) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int nrt = (Sq * p.G + 15) / 16;
+    const long long units = (long long)B * Hkv * nrt;
+    long long n = (2LL * sms + units - 1) / units;
+    if (n > FA_MAX_SPLITS) n = FA_MAX_SPLITS;
+    if (n > max_units) n = max_units;
+    num_splits = n < 1 ? 1 : (int)n;
+  }
+  p.num_splits = num_splits;
+  if (num_splits > 1) {
+    const size_t rows = (size_t)num_splits * B * Hq * Sq;
+    const size_t need = round256(rows * D * sizeof(float)) + round256(rows * sizeof(float));
+    if (!workspace || ws_bytes < need) return FA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
+    p.o_part = static_cast<float*>(workspace);
+    p.lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round256(rows * D * sizeof(float)));
+  }
+  p.status = status_ptr();
+  if (!p.status) return FA_ERR_CUDA;
+  int launches = 0;
+  cudaError_t e = fa::launch_decode(p, dt, stream, &launches);
+  g_last_launches = launches;
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_last_device_status(fa_stream_t stream) {
+  int* ptr = status_ptr();
+  if (!ptr) return FA_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return FA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_fa_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_fa_status, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  return static_cast<fa_status>(v);
+}
+
+}  // extern "C"

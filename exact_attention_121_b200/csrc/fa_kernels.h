@@ -1,0 +1,87 @@
+// Parameter blocks and launchers shared between the host layer (fa_api.cu)
+// and the kernel translation units.  Host code only; no torch types.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fa.h"
+
+namespace fa {
+
+// Forward problem after validation: window extents already have causal folded
+// in (negative = unbounded), scale already resolved.
+struct FwdParams {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  int B, Sq, Sk, Hq, Hkv, D, G;
+  int wl, wr;            // effective window extents, -1 = unbounded
+  float scale_log2;      // scale * log2(e)
+  float softcap;         // > 0 enables the tanh cap
+  float cap_in;          // scale / softcap: raw dot product -> tanh argument
+  float cap_log2;        // softcap * log2(e)
+  int* status;           // device status word
+};
+
+struct BwdParams {
+  const void* dout;
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;
+  const float* lse;
+  void* dq;
+  void* dk;
+  void* dv;
+  float* dq_accum;       // (B, Sq, Hq, D) fp32
+  float* delta;          // (B, Hq, Sq) fp32
+  int* sem;              // (B, Hq, n_qblocks) ordering counters (deterministic)
+  int* work_counter;     // dynamic work index (deterministic)
+  int B, Sq, Sk, Hq, Hkv, D, G;
+  int wl, wr;
+  float scale;
+  float scale_log2;
+  float softcap, cap_in, cap_log2;
+  int deterministic;
+  int* status;
+};
+
+struct DecodeParams {
+  const void* q;
+  void* k_cache;
+  void* v_cache;
+  const void* k_new;
+  const void* v_new;
+  const int* cache_seqlens;
+  const int* block_table;
+  int page_size, max_pages_per_seq, capacity_pages;  // paged layout
+  int max_seqlen;                                    // contiguous layout
+  int paged;
+  void* out;
+  float* lse;
+  float* o_part;   // (splits, B, Hq, Sq, D)
+  float* lse_part; // (splits, B, Hq, Sq)
+  int B, Sq, Snew, Hq, Hkv, D, G;
+  int num_splits;
+  int wl, wr;
+  float scale_log2, softcap, cap_in, cap_log2;
+  int* status;
+};
+
+// Optional timing hooks around the dominant kernel of each call (events set
+// with fa_set_trace_events; no-ops when unset).
+void trace_begin(cudaStream_t s);
+void trace_end(cudaStream_t s);
+
+// Launchers: return the first CUDA error (cudaSuccess on success) and add the
+// number of kernels launched to *launches.
+cudaError_t launch_fwd_mma(const FwdParams& p, fa_dtype dt, cudaStream_t s, int* launches);
+bool fwd_tc_supported(const FwdParams& p);
+cudaError_t launch_fwd_tc(const FwdParams& p, fa_dtype dt, cudaStream_t s, int* launches);
+cudaError_t launch_bwd(const BwdParams& p, fa_dtype dt, cudaStream_t s, int* launches);
+cudaError_t launch_decode(const DecodeParams& p, fa_dtype dt, cudaStream_t s, int* launches);
+
+}  // namespace fa

@@ -1,0 +1,195 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact-attention library libfa.so.
+ *
+ * The library computes exact scaled dot-product attention
+ *     O = softmax(transform(scale * Q K^T) + mask) V
+ * tile by tile with an online softmax, so the Sq x Sk score matrix never
+ * reaches device memory; the backward recomputes the probabilities from the
+ * saved row log-sum-exp instead of storing them.  Sources: "FlashAttention
+ * 实战指南" (mhpq.cn), sections "why long sequences run out of memory" (the
+ * three steps of standard attention, tiling, online softmax, recomputation,
+ * exact result), "advanced parameters" (causal, window_size, softcap,
+ * deterministic, MQA/GQA) and "incremental decoding" (flash_attn_with_kvcache:
+ * append then attend, cache_seqlens, block_table, num_splits).
+ *
+ * Conventions shared by every entry point
+ * --------------------------------------
+ * Layout.   Q, K, V, O and their gradients are dense row-major tensors in the
+ *           pages' (batch, seqlen, nheads, headdim) order: element
+ *           [b][s][h][d] sits at ((b*S + s)*H + h)*D + d.  Every pointer must
+ *           be 16-byte aligned.  LSE is float32 (B, Hq, Sq), natural log.
+ * Types.    FA_FP16 or FA_BF16 for all 16-bit tensors of one call; every
+ *           accumulation is float32.
+ * Heads.    Hq must be an integer multiple of Hkv (MQA/GQA); q-head h reads
+ *           kv-head h / (Hq/Hkv).  D must be 64 or 128.
+ * Scale.    scale <= 0 selects 1/sqrt(D).
+ * Softcap.  softcap > 0 replaces each scaled score u by softcap*tanh(u/softcap)
+ *           before masking; softcap <= 0 disables it.
+ * Masks.    Query i sits at key position i + Sk - Sq (bottom-right
+ *           alignment).  Key j is visible iff
+ *               j >= i + Sk - Sq - window_left   (when window_left  >= 0)
+ *               j <= i + Sk - Sq + window_right  (when window_right >= 0)
+ *           bounds inclusive, a negative extent is unbounded; causal != 0 is
+ *           the same as window_right = 0 and is intersected with the window.
+ *           A query with no visible key gets O = 0 and LSE = -inf.
+ * Memory.   The caller owns every buffer, including workspaces; the library
+ *           never allocates or frees device memory and never synchronises the
+ *           stream (fa_last_device_status is the one exception, by design).
+ *           Every call is asynchronous on `stream` (NULL = legacy default).
+ * Errors.   Argument errors are returned before anything is launched.  A
+ *           launch failure returns FA_ERR_CUDA.  Waits inside kernels are
+ *           bounded; one that runs out records FA_ERR_TIMEOUT in a device
+ *           status word that fa_last_device_status() reads.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared here so that the header needs no CUDA
+ * include. */
+typedef struct CUstream_st* fa_stream_t;
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment or Hq % Hkv != 0 */
+  FA_ERR_UNSUPPORTED = 2, /* valid request this build does not implement (e.g. D=96) */
+  FA_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+  FA_ERR_TIMEOUT = 4      /* a bounded device wait ran out (device status word) */
+} fa_status;
+
+typedef enum { FA_FP16 = 0, FA_BF16 = 1 } fa_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fa_status_string(fa_status s);
+
+/*
+ * Forward attention ("FlashAttention 实战指南", minimal example with
+ * flash_attn_func and the advanced parameters).
+ *   q   (B, Sq, Hq, D)  16-bit, read
+ *   k,v (B, Sk, Hkv, D) 16-bit, read
+ *   out (B, Sq, Hq, D)  16-bit, written
+ *   lse (B, Hq, Sq)     float32, written (natural-log row log-sum-exp)
+ * Sq, Sk >= 1 (Sq or Sk = 0 or B = 0 is a no-op returning FA_OK).
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                 int B, int Sq, int Sk, int Hq, int Hkv, int D, fa_dtype dt,
+                 float scale, int causal, int window_left, int window_right, float softcap,
+                 fa_stream_t stream);
+
+/*
+ * Bytes of workspace fa_bwd needs: the float32 dQ accumulator (B, Sq, Hq, D),
+ * the row terms Delta = rowsum(dO * O) (B, Hq, Sq) and, when deterministic,
+ * one int32 ordering counter per (b, q-head, 64-row query block) plus a work
+ * counter.  Linear in the sequence length.  Returns 0 for invalid sizes.
+ */
+size_t fa_bwd_workspace_size(int B, int Sq, int Sk, int Hq, int Hkv, int D, int deterministic);
+
+/*
+ * Backward attention by recomputation ("FlashAttention 实战指南", the three
+ * techniques: the backward pass recomputes the attention matrix; and the
+ * `deterministic` parameter).
+ *   dout, q, out (B, Sq, Hq, D) 16-bit, read;  k, v (B, Sk, Hkv, D) read
+ *   lse          (B, Hq, Sq) float32 from fa_fwd with the same arguments
+ *   dq (B, Sq, Hq, D), dk, dv (B, Sk, Hkv, D) 16-bit, written (overwritten,
+ *   not accumulated into).  dK/dV of a kv-head sum over its q-heads.
+ *   workspace: >= fa_bwd_workspace_size(...) bytes, 256-byte aligned,
+ *   contents on entry ignored.
+ *   deterministic != 0: dQ contributions are added in ascending key-block
+ *   order behind bounded counters, so repeated calls give bit-identical
+ *   results; otherwise they are added with float32 atomics.
+ */
+fa_status fa_bwd(const void* dout, const void* q, const void* k, const void* v,
+                 const void* out, const float* lse, void* dq, void* dk, void* dv,
+                 int B, int Sq, int Sk, int Hq, int Hkv, int D, fa_dtype dt,
+                 float scale, int causal, int window_left, int window_right, float softcap,
+                 int deterministic, void* workspace, size_t ws_bytes, fa_stream_t stream);
+
+/* Largest split count fa_fwd_kvcache accepts; num_splits <= 0 picks one. */
+#define FA_MAX_SPLITS 64
+
+/*
+ * Bytes of workspace fa_fwd_kvcache needs for `num_splits` KV splits: the
+ * float32 partial outputs (splits, B, Hq, Sq, D) and partial LSEs
+ * (splits, B, Hq, Sq).  num_splits <= 0 returns the size for FA_MAX_SPLITS.
+ * Returns 0 when one split needs no workspace.
+ */
+size_t fa_kvcache_workspace_size(int B, int Sq, int Hq, int D, int num_splits);
+
+/*
+ * Incremental decoding with a KV cache ("FlashAttention 实战指南", section on
+ * flash_attn_with_kvcache): append the new keys/values into the cache, then
+ * attend in place.
+ *   q (B, Sq, Hq, D) 16-bit, read.
+ *   Paged (block_table != NULL): k_cache, v_cache (num_pages, page_size, Hkv,
+ *     D); block_table (B, max_pages_per_seq) int32 physical page ids in
+ *     [0, num_pages_or_max_seqlen); logical token t of sequence b lives in
+ *     page block_table[b][t / page_size], slot t % page_size.
+ *   Contiguous (block_table == NULL): k_cache, v_cache (B,
+ *     num_pages_or_max_seqlen, Hkv, D); page_size still sets the split unit.
+ *   k_new, v_new (B, Snew, Hkv, D) or NULL when Snew == 0; written into the
+ *     cache at logical positions cache_seqlens[b] .. cache_seqlens[b]+Snew-1.
+ *   cache_seqlens (B) int32 device: valid length of each sequence BEFORE the
+ *     append; not modified.  Sequence b attends over cache_seqlens[b] + Snew
+ *     keys, which must fit the cache (checked on the device: an overflowing
+ *     sequence is skipped and FA_ERR_INVALID_ARG is recorded in the status
+ *     word).
+ *   out (B, Sq, Hq, D) 16-bit written; lse (B, Hq, Sq) float32 or NULL.
+ *   num_splits: KV range of each sequence split into this many page-aligned
+ *     parts (<= 0: chosen from B, Hkv and the capacity); partials are merged
+ *     by a log-sum-exp combine.  workspace >= fa_kvcache_workspace_size(B, Sq,
+ *     Hq, D, num_splits) bytes, 256-byte aligned (may be NULL when that is 0).
+ */
+fa_status fa_fwd_kvcache(const void* q, void* k_cache, void* v_cache, const void* k_new,
+                         const void* v_new, const int* cache_seqlens, const int* block_table,
+                         int page_size, int max_pages_per_seq, int num_pages_or_max_seqlen,
+                         void* out, float* lse, int B, int Sq, int Snew, int Hq, int Hkv, int D,
+                         fa_dtype dt, float scale, int causal, int window_left, int window_right,
+                         float softcap, int num_splits, void* workspace, size_t ws_bytes,
+                         fa_stream_t stream);
+
+/*
+ * Waits for `stream`, then returns and clears the device status word of the
+ * current device: FA_OK, FA_ERR_TIMEOUT (a bounded wait ran out) or
+ * FA_ERR_INVALID_ARG (a device-side argument check failed, e.g. a cache
+ * overflow).  Returns FA_ERR_CUDA if the synchronisation itself fails.
+ */
+fa_status fa_last_device_status(fa_stream_t stream);
+
+/*
+ * Which forward kernel fa_fwd runs: 0 = automatic (tensor-memory tcgen05
+ * kernel where it applies), 1 = force the warp-level mma.sync kernel.  Process
+ * wide; meant for tests and benchmarks that compare the two.
+ */
+void fa_set_fwd_kernel(int which);
+
+/*
+ * Diagnostic for the failure-detection path: one kernel spins (bounded, with
+ * the same helper the ordered backward uses) until the int32 at device
+ * address `flag` equals `expected` or `limit_ns` nanoseconds pass; on timeout
+ * it records FA_ERR_TIMEOUT in the status word and returns.  Never faults or
+ * hangs: the wait always ends.
+ */
+fa_status fa_selftest_bounded_wait(const int* flag, int expected, long long limit_ns, fa_stream_t stream);
+
+/*
+ * Timing hook: when set (non-NULL cudaEvent_t handles), every later fa_fwd,
+ * fa_bwd and fa_fwd_kvcache call records `start_event` immediately before its
+ * dominant kernel (the forward kernel, the main backward kernel, the split
+ * decode kernel) and `stop_event` immediately after it, on the call's stream.
+ * Pass NULL, NULL to switch it off.  The events stay owned by the caller.
+ */
+void fa_set_trace_events(void* start_event, void* stop_event);
+
+/* Number of kernels the last fa_* call launched (for launch accounting). */
+int fa_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

@@ -2,6 +2,7 @@
 from .attn64 import (  # noqa: F401
     attn_bwd,
     attn_fwd,
+    attn_fwd_rows,
     attn_fwd_online,
     attn_partial,
     attn_with_kvcache,
@@ -11,4 +12,5 @@ from .attn64 import (  # noqa: F401
     kvcache_append,
     split_token_ranges,
     visible,
+    visible_rows,
 )

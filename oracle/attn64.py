@@ -72,23 +72,31 @@ def effective_window(causal, window_left, window_right):
     return left, right
 
 
-def visible(Sq, Sk, causal=False, window_left=-1, window_right=-1, key_offset=0, n_keys=None):
-    """Boolean (Sq, n_keys) matrix: may query i see key (key_offset + j)?
+def visible_rows(rows, Sq, Sk, causal=False, window_left=-1, window_right=-1, key_offset=0,
+                 n_keys=None):
+    """Boolean (len(rows), n_keys): may query ``rows[r]`` see key (key_offset + j)?
 
-    Query i sits at absolute position ``i + Sk - Sq``.  ``key_offset`` and
-    ``n_keys`` select a sub-range of the Sk keys (used for KV splits).
+    Query i sits at absolute position ``i + Sk - Sq`` (bottom-right
+    alignment).  ``key_offset`` and ``n_keys`` select a sub-range of the Sk
+    keys (used for KV splits).
     """
     if n_keys is None:
         n_keys = Sk - key_offset
+    rows = np.asarray(rows)
     left, right = effective_window(causal, window_left, window_right)
-    qpos = np.arange(Sq)[:, None] + (Sk - Sq)
+    qpos = rows[:, None] + (Sk - Sq)
     kpos = np.arange(key_offset, key_offset + n_keys)[None, :]
-    ok = np.broadcast_to((kpos >= 0) & (kpos < Sk), (Sq, n_keys)).copy()
+    ok = np.broadcast_to((kpos >= 0) & (kpos < Sk), (len(rows), n_keys)).copy()
     if right >= 0:
         ok &= kpos <= qpos + right
     if left >= 0:
         ok &= kpos >= qpos - left
     return ok
+
+
+def visible(Sq, Sk, causal=False, window_left=-1, window_right=-1, key_offset=0, n_keys=None):
+    """Boolean (Sq, n_keys) matrix for all queries; see :func:`visible_rows`."""
+    return visible_rows(np.arange(Sq), Sq, Sk, causal, window_left, window_right, key_offset, n_keys)
 
 
 # ---------------------------------------------------------------------------
@@ -103,7 +111,7 @@ def _check_heads(Hq, Hkv):
 
 def raw_scores(q, k, scale, h, g):
     """u[b, i, j] = scale * sum_d q[b,i,h,d] * k[b,j,g,d]  (float64)."""
-    return scale * np.einsum("bid,bjd->bij", q[:, :, h, :], k[:, :, g, :])
+    return scale * np.matmul(q[:, :, h, :], k[:, :, g, :].transpose(0, 2, 1))
 
 
 def transform_scores(u, softcap):
@@ -146,7 +154,7 @@ def attn_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1,
         l = e.sum(axis=2)
         row_lse = np.where(any_vis[None], m + np.log(np.where(l > 0, l, 1.0)), NEG_INF)
         P = np.where(vis[None], np.exp(s - row_lse[:, :, None]), 0.0)
-        out[:, :, h, :] = np.einsum("bij,bjd->bid", P, v[:, :, g, :])
+        out[:, :, h, :] = np.matmul(P, v[:, :, g, :])
         lse[:, h, :] = row_lse
         if return_probs:
             P_all[:, h] = P
@@ -154,6 +162,39 @@ def attn_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1,
     if return_probs:
         return out, lse, P_all, U_all
     return out, lse
+
+
+def attn_fwd_rows(q, k, v, b, h, rows, scale=None, causal=False, window_left=-1, window_right=-1,
+                  softcap=0.0):
+    """O and LSE of selected query rows of one (batch b, q-head h).
+
+    Each row is the plain definition on its own: its scores against every
+    key, the visibility rule at its absolute position, a softmax over the
+    visible keys and the weighted sum of V.  Returns O (len(rows), D) and LSE
+    (len(rows),).  Used to check outputs of problems too large to evaluate
+    whole.
+    """
+    q = np.asarray(q)
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    G = _check_heads(Hq, Hkv)
+    g = h // G
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(D)
+    rows = np.asarray(rows)
+    Kg = np.asarray(k[b, :, g, :], np.float64)
+    Vg = np.asarray(v[b, :, g, :], np.float64)
+    u = scale * (np.asarray(q[b, rows, h, :], np.float64) @ Kg.T)   # (R, Sk)
+    s = transform_scores(u, softcap)
+    vis = visible_rows(rows, Sq, Sk, causal, window_left, window_right)
+    s = np.where(vis, s, NEG_INF)
+    anyv = vis.any(axis=1)
+    m = np.where(anyv, s.max(axis=1), 0.0)
+    e = np.where(vis, np.exp(s - m[:, None]), 0.0)
+    l = e.sum(axis=1)
+    lse = np.where(anyv, m + np.log(np.where(anyv, l, 1.0)), NEG_INF)
+    o = np.where(anyv[:, None], (e @ Vg) / np.where(anyv, l, 1.0)[:, None], 0.0)
+    return o, lse
 
 
 # ---------------------------------------------------------------------------
@@ -227,25 +268,28 @@ def attn_bwd(dout, q, k, v, scale=None, causal=False, window_left=-1, window_rig
     G = _check_heads(Hq, Hkv)
     if scale is None or scale <= 0:
         scale = 1.0 / math.sqrt(D)
-    _, _, P, U = attn_fwd(q, k, v, scale, causal, window_left, window_right, softcap,
-                          return_probs=True)
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
     delta = np.zeros((B, Hq, Sq))
     for h in range(Hq):
         g = h // G
-        Ph = P[:, h]                                    # (B, Sq, Sk)
+        # forward of this head alone (same definition as attn_fwd)
+        _, _, P, U = attn_fwd(q[:, :, h:h + 1], k[:, :, g:g + 1], v[:, :, g:g + 1], scale, causal,
+                              window_left, window_right, softcap, return_probs=True)
+        Ph, Uh = P[:, 0], U[:, 0]                       # (B, Sq, Sk)
+        del P, U
         dO = dout[:, :, h, :]                           # (B, Sq, D)
-        dv[:, :, g, :] += np.einsum("bij,bid->bjd", Ph, dO)
-        dP = np.einsum("bid,bjd->bij", dO, v[:, :, g, :])
+        dv[:, :, g, :] += np.matmul(Ph.transpose(0, 2, 1), dO)
+        dP = np.matmul(dO, v[:, :, g, :].transpose(0, 2, 1))
         dl = (Ph * dP).sum(axis=2)                      # Delta
         dS = Ph * (dP - dl[:, :, None])
+        del dP
         if softcap is not None and softcap > 0:
-            t = np.tanh(U[:, h] / softcap)
+            t = np.tanh(Uh / softcap)
             dS = dS * (1.0 - t * t)
-        dq[:, :, h, :] = scale * np.einsum("bij,bjd->bid", dS, k[:, :, g, :])
-        dk[:, :, g, :] += scale * np.einsum("bij,bid->bjd", dS, q[:, :, h, :])
+        dq[:, :, h, :] = scale * np.matmul(dS, k[:, :, g, :])
+        dk[:, :, g, :] += scale * np.matmul(dS.transpose(0, 2, 1), q[:, :, h, :])
         delta[:, h, :] = dl
     return dq, dk, dv, delta
 

@@ -8,3 +8,6 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+    # libfa.so is built in-tree (incremental: a no-op when it is up to date).
+    from exact_attention_121_b200 import build
+    build.build()

@@ -1,0 +1,111 @@
+"""The C ABI without a GPU: libfa.so loads, exports every symbol include/fa.h
+declares with the declared arity, and rejects bad arguments on the host
+before touching CUDA.  Workspace sizes are linear in the sequence length."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_attention_121_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+
+def _declarations():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    decls = {}
+    for m in re.finditer(r"^\s*(?:const\s+char\s*\*|fa_status|size_t|void|int)\s+(fa_\w+)\s*\(([^)]*)\)\s*;",
+                         text, flags=re.M):
+        args = m.group(2).strip()
+        n = 0 if args in ("", "void") else len(args.split(","))
+        decls[m.group(1)] = n
+    return decls
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return _lib.load()
+
+
+def test_header_declares_entry_points():
+    d = _declarations()
+    for name in ("fa_fwd", "fa_bwd", "fa_fwd_kvcache", "fa_bwd_workspace_size",
+                 "fa_kvcache_workspace_size", "fa_status_string", "fa_last_device_status"):
+        assert name in d
+
+
+def test_every_declared_symbol_is_exported_with_its_arity(lib):
+    d = _declarations()
+    assert set(d) == set(_lib.SIGNATURES), set(d) ^ set(_lib.SIGNATURES)
+    for name, nargs in d.items():
+        assert hasattr(lib, name), name
+        assert len(_lib.SIGNATURES[name][1]) == nargs, name
+
+
+def test_status_strings(lib):
+    assert lib.fa_status_string(0) == b"FA_OK"
+    assert lib.fa_status_string(4) == b"FA_ERR_TIMEOUT"
+    assert lib.fa_status_string(99) == b"FA_ERR_UNKNOWN"
+
+
+def _fwd(lib, ptr=0x1000, B=1, Sq=8, Sk=8, Hq=2, Hkv=2, D=64, dt=1, scale=0.0, softcap=0.0):
+    p = ctypes.c_void_p(ptr)
+    return lib.fa_fwd(p, p, p, p, p, B, Sq, Sk, Hq, Hkv, D, dt, scale, 0, -1, -1, softcap, None)
+
+
+def test_host_validation_rejects_before_launch(lib):
+    assert _fwd(lib, Hq=3, Hkv=2) == _lib.FA_ERR_INVALID_ARG      # GQA needs Hq % Hkv == 0
+    assert _fwd(lib, D=96) == _lib.FA_ERR_UNSUPPORTED
+    assert _fwd(lib, dt=7) == _lib.FA_ERR_INVALID_ARG
+    assert _fwd(lib, ptr=0x1008) == _lib.FA_ERR_INVALID_ARG       # not 16-byte aligned
+    assert _fwd(lib, ptr=0) == _lib.FA_ERR_INVALID_ARG            # null pointers
+    assert _fwd(lib, scale=float("nan")) == _lib.FA_ERR_INVALID_ARG
+    assert _fwd(lib, B=-1) == _lib.FA_ERR_INVALID_ARG
+    assert _fwd(lib, B=0) == _lib.FA_OK                            # empty batch: no-op
+    assert _fwd(lib, Sq=0) == _lib.FA_OK
+
+
+def test_bwd_rejects_short_workspace(lib):
+    p = ctypes.c_void_p(0x1000)
+    need = lib.fa_bwd_workspace_size(1, 64, 64, 2, 2, 64, 0)
+    assert need > 0
+    code = lib.fa_bwd(p, p, p, p, p, p, p, p, p, 1, 64, 64, 2, 2, 64, 1, 0.0, 0, -1, -1, 0.0, 0,
+                      ctypes.c_void_p(0x10000), need - 1, None)
+    assert code == _lib.FA_ERR_INVALID_ARG
+
+
+def test_kvcache_rejects_bad_split_count_and_pages(lib):
+    p = ctypes.c_void_p(0x1000)
+    args = [p, p, p, p, p, p, p, 256, 4, 8, p, p, 2, 1, 1, 8, 2, 128, 1, 0.0, 1, -1, -1, 0.0]
+    assert lib.fa_fwd_kvcache(*args, _lib.FA_MAX_SPLITS + 1, p, 0, None) == _lib.FA_ERR_INVALID_ARG
+    bad = list(args)
+    bad[7] = 0  # page_size
+    assert lib.fa_fwd_kvcache(*bad, 1, p, 0, None) == _lib.FA_ERR_INVALID_ARG
+    gqa = list(args)
+    gqa[15] = 3  # Hkv does not divide Hq=8
+    assert lib.fa_fwd_kvcache(*gqa, 1, p, 0, None) == _lib.FA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("det", [0, 1])
+def test_bwd_workspace_is_linear_in_seqlen(lib, det):
+    sizes = [lib.fa_bwd_workspace_size(2, S, S, 16, 16, 128, det) for S in (1024, 2048, 4096, 8192)]
+    for a, b in zip(sizes, sizes[1:]):
+        assert abs(b / a - 2.0) < 0.01
+    # the attention matrix would be B*H*S*S*2 bytes: the workspace is far below it
+    assert sizes[-1] < 2 * 16 * 8192 * 8192 * 2 / 20
+
+
+def test_kvcache_workspace(lib):
+    assert lib.fa_kvcache_workspace_size(8, 1, 32, 128, 1) == 0
+    n4 = lib.fa_kvcache_workspace_size(8, 1, 32, 128, 4)
+    n16 = lib.fa_kvcache_workspace_size(8, 1, 32, 128, 16)
+    assert n4 >= 4 * 8 * 32 * 128 * 4 and n16 >= 4 * n4 - 1024
+    assert lib.fa_kvcache_workspace_size(8, 1, 32, 128, 0) == lib.fa_kvcache_workspace_size(8, 1, 32, 128, 64)
+
+
+def test_selftest_rejects_null_flag(lib):
+    assert lib.fa_selftest_bounded_wait(None, 1, 1000, None) == _lib.FA_ERR_INVALID_ARG

@@ -1,0 +1,120 @@
+"""Backward parity: CUDA dQ/dK/dV vs the float64 oracle's chain rule, atomic
+and deterministic (ordered) dQ modes; bit-identity of the deterministic mode."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from _parity import check_grad, check_lse, check_out, f64
+from exact_attention_121_b200 import api, inputs
+
+pytestmark = pytest.mark.gpu
+
+DT = {"fp16": torch.float16, "bf16": torch.bfloat16}
+
+# (B, Sq, Sk, Hq, Hkv, D, dtype, causal, window, softcap, scale, amp)
+SMALL = [
+    (2, 77, 77, 4, 4, 64, "bf16", True, (-1, -1), 0.0, None, 1.0),
+    (1, 130, 200, 4, 2, 128, "fp16", False, (-1, -1), 5.0, None, 1.0),
+    (2, 200, 130, 8, 2, 64, "bf16", True, (-1, -1), 0.0, None, 1.0),
+    (1, 257, 257, 2, 1, 128, "bf16", False, (32, 16), 0.0, None, 1.0),
+    (1, 1, 300, 4, 4, 64, "fp16", True, (-1, -1), 0.0, None, 1.0),
+    (1, 300, 1, 2, 2, 128, "bf16", False, (-1, -1), 0.0, None, 1.0),
+    (3, 190, 190, 6, 3, 128, "fp16", True, (50, 0), 10.0, None, 2.0),
+    (1, 512, 512, 4, 1, 128, "bf16", True, (-1, -1), 30.0, 0.3, 2.0),
+]
+
+
+def _fwd_bwd(q, k, v, do, det, **kw):
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    out, lse = api.fa_fwd(qd, kd, vd, **kw)
+    dq, dk, dv = api.fa_bwd(dod, qd, kd, vd, out, lse, deterministic=det, **kw)
+    torch.cuda.synchronize()
+    assert api.fa_last_device_status() == 0
+    return out, lse, dq, dk, dv
+
+
+@pytest.mark.parametrize("det", [False, True], ids=["atomic", "ordered"])
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: "B%dSq%dSk%dH%d-%dD%d%s%s" % (
+    c[0], c[1], c[2], c[3], c[4], c[5], c[6], "c" if c[7] else ""))
+def test_bwd_small_full_compare(case, det):
+    B, Sq, Sk, Hq, Hkv, D, dt, causal, window, cap, scale, amp = case
+    q, k, v, do = inputs.attention_inputs(B, Sq, Sk, Hq, Hkv, D, dt, seed=21, amp=amp)
+    kw = dict(scale=scale, causal=causal, window=window, softcap=cap)
+    out, lse, dq, dk, dv = _fwd_bwd(q, k, v, do, det, **kw)
+    sc = scale or 1 / math.sqrt(D)
+    dq_r, dk_r, dv_r, _ = oracle.attn_bwd(f64(do), f64(q), f64(k), f64(v), sc, causal, window[0], window[1], cap)
+    check_grad(dq, dq_r, "dQ")
+    check_grad(dk, dk_r, "dK")
+    check_grad(dv, dv_r, "dV")
+
+
+@pytest.mark.parametrize("det", [False, True], ids=["atomic", "ordered"])
+def test_fwd_bwd_512_full(det):
+    cfg = inputs.fwd_bwd_512_config()
+    q, k, v, do = inputs.attention_inputs(cfg["B"], cfg["Sq"], cfg["Sk"], cfg["Hq"], cfg["Hkv"], cfg["D"],
+                                          cfg["dtype"], seed=cfg["seed"])
+    out, lse, dq, dk, dv = _fwd_bwd(q, k, v, do, det, scale=cfg["scale"], causal=True)
+    o_r, l_r = oracle.attn_fwd(f64(q), f64(k), f64(v), cfg["scale"], True)
+    check_out(out, o_r, torch.float16)
+    check_lse(lse, l_r)
+    dq_r, dk_r, dv_r, _ = oracle.attn_bwd(f64(do), f64(q), f64(k), f64(v), cfg["scale"], True)
+    check_grad(dq, dq_r, "dQ")
+    check_grad(dk, dk_r, "dK")
+    check_grad(dv, dv_r, "dV")
+
+
+@pytest.mark.parametrize("det", [False, True], ids=["atomic", "ordered"])
+def test_gqa_local_full_size_slices(det):
+    """Full-size GQA + window + softcap workload; gradients of two kv-head groups
+    (all their q-heads) in both batches are compared with the oracle."""
+    cfg = inputs.gqa_local_config()
+    q, k, v, do = inputs.attention_inputs(cfg["B"], cfg["Sq"], cfg["Sk"], cfg["Hq"], cfg["Hkv"], cfg["D"],
+                                          cfg["dtype"], seed=cfg["seed"], amp=cfg["amp"])
+    kw = dict(scale=cfg["scale"], causal=True, window=cfg["window"], softcap=cfg["softcap"])
+    out, lse, dq, dk, dv = _fwd_bwd(q, k, v, do, det, **kw)
+    G = cfg["Hq"] // cfg["Hkv"]
+    for b in (0, 1):
+        for g in (0, cfg["Hkv"] - 1):
+            hs = slice(g * G, (g + 1) * G)
+            sl = lambda t, heads: f64(t[b:b + 1, :, heads])
+            dq_r, dk_r, dv_r, _ = oracle.attn_bwd(sl(do, hs), sl(q, hs), sl(k, slice(g, g + 1)),
+                                                  sl(v, slice(g, g + 1)), cfg["scale"], True,
+                                                  cfg["window"][0], 0, cfg["softcap"])
+            check_grad(dq[b:b + 1, :, hs], dq_r, f"dQ b{b} g{g}")
+            check_grad(dk[b:b + 1, :, g:g + 1], dk_r, f"dK b{b} g{g}")
+            check_grad(dv[b:b + 1, :, g:g + 1], dv_r, f"dV b{b} g{g}")
+
+
+def test_deterministic_is_bit_identical():
+    cfg = inputs.gqa_local_config()
+    q, k, v, do = inputs.attention_inputs(cfg["B"], cfg["Sq"], cfg["Sk"], cfg["Hq"], cfg["Hkv"], cfg["D"],
+                                          cfg["dtype"], seed=cfg["seed"], amp=cfg["amp"])
+    kw = dict(scale=cfg["scale"], causal=True, window=cfg["window"], softcap=cfg["softcap"])
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    out, lse = api.fa_fwd(qd, kd, vd, **kw)
+    runs = []
+    for _ in range(3):
+        runs.append([t.clone() for t in api.fa_bwd(dod, qd, kd, vd, out, lse, deterministic=True, **kw)])
+    torch.cuda.synchronize()
+    for r in runs[1:]:
+        for a, b in zip(runs[0], r):
+            assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert api.fa_last_device_status() == 0
+
+
+@pytest.mark.parametrize("cfg", [c for c in inputs.seqlen_sweep_configs() if c["Sq"] <= 2048],
+                         ids=lambda c: "H%dD%dS%d%s" % (c["Hq"], c["D"], c["Sq"], "c" if c["causal"] else "n"))
+def test_bwd_seqlen_sweep_head_slices(cfg):
+    q, k, v, do = inputs.attention_inputs(cfg["B"], cfg["Sq"], cfg["Sk"], cfg["Hq"], cfg["Hkv"], cfg["D"],
+                                          cfg["dtype"], seed=cfg["seed"])
+    out, lse, dq, dk, dv = _fwd_bwd(q, k, v, do, False, scale=cfg["scale"], causal=cfg["causal"])
+    for b, h in ((0, 0), (cfg["B"] - 1, cfg["Hq"] - 1)):
+        sl = lambda t: f64(t[b:b + 1, :, h:h + 1])
+        dq_r, dk_r, dv_r, _ = oracle.attn_bwd(sl(do), sl(q), sl(k), sl(v), cfg["scale"], cfg["causal"])
+        check_grad(dq[b:b + 1, :, h:h + 1], dq_r, "dQ")
+        check_grad(dk[b:b + 1, :, h:h + 1], dk_r, "dK")
+        check_grad(dv[b:b + 1, :, h:h + 1], dv_r, "dV")

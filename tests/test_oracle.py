@@ -406,3 +406,16 @@ def test_planted_exclusive_window_is_caught(monkeypatch):
     monkeypatch.setattr(attn64, "visible", excl)
     with pytest.raises(AssertionError):
         test_hand_examples_forward(_hand("window_left1"))
+
+
+def test_rows_equal_full_forward():
+    rng = np.random.default_rng(50)
+    q, k, v = _rand((2, 37, 4, 8), rng), _rand((2, 41, 2, 8), rng), _rand((2, 41, 2, 8), rng)
+    kw = dict(scale=0.3, causal=True, window_left=9, window_right=0, softcap=2.0)
+    o, lse = oracle.attn_fwd(q, k, v, **kw)
+    rows = np.array([0, 5, 17, 36])
+    for b in range(2):
+        for h in range(4):
+            orow, lrow = oracle.attn_fwd_rows(q, k, v, b, h, rows, **kw)
+            np.testing.assert_allclose(orow, o[b, rows, h], atol=1e-14)
+            np.testing.assert_allclose(lrow, lse[b, h, rows], atol=1e-14)
