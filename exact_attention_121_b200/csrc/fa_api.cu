@@ -22,6 +22,8 @@ __device__ int g_fa_status = 0;
 constexpr int kMaxDevices = 64;
 int* g_status_ptr[kMaxDevices] = {nullptr};
 int g_fwd_kernel_choice = 0;
+// Whether the automatic choice uses the tcgen05 forward kernel.
+constexpr bool kTcAuto = false;
 cudaEvent_t g_trace_start = nullptr, g_trace_stop = nullptr;
 thread_local int g_last_launches = 0;
 
@@ -144,10 +146,13 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* 
   if (!p.status) return FA_ERR_CUDA;
   int launches = 0;
   cudaError_t e;
-  if (g_fwd_kernel_choice == 0 && fa::fwd_tc_supported(p))
+  const bool tc = (g_fwd_kernel_choice == 2) || (g_fwd_kernel_choice == 0 && kTcAuto);
+  if (tc && fa::fwd_tc_supported(p)) {
     e = fa::launch_fwd_tc(p, dt, stream, &launches);
-  else
+  } else {
+    if (g_fwd_kernel_choice == 2) return FA_ERR_UNSUPPORTED;
     e = fa::launch_fwd_mma(p, dt, stream, &launches);
+  }
   g_last_launches = launches;
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

@@ -161,9 +161,10 @@ fa_status fa_fwd_kvcache(const void* q, void* k_cache, void* v_cache, const void
 fa_status fa_last_device_status(fa_stream_t stream);
 
 /*
- * Which forward kernel fa_fwd runs: 0 = automatic (tensor-memory tcgen05
- * kernel where it applies), 1 = force the warp-level mma.sync kernel.  Process
- * wide; meant for tests and benchmarks that compare the two.
+ * Which forward kernel fa_fwd runs: 0 = automatic, 1 = the warp-level
+ * mma.sync kernel, 2 = the tensor-memory tcgen05 kernel (fa_fwd returns
+ * FA_ERR_UNSUPPORTED where it does not apply).  Process wide; meant for tests
+ * and benchmarks that compare the two.
  */
 void fa_set_fwd_kernel(int which);
 
