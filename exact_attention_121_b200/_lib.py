@@ -28,6 +28,8 @@ SIGNATURES = {
     "fa_kvcache_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "fa_fwd_kvcache": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _I, _I, _I, _I, _I, _I,
                             _I, _F, _I, _I, _I, _F, _I, _P, _Z, _P]),
+    "fa_fwd_kvcache_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _I, _I, _I, _I, _I, _I,
+                                    _I, _F, _I, _I, _I, _F, _I, _P]),
     "fa_last_device_status": (_I, [_P]),
     "fa_set_fwd_kernel": (None, [_I]),
     "fa_selftest_bounded_wait": (_I, [_P, _I, ctypes.c_longlong, _P]),

@@ -152,6 +152,40 @@ fa_status fa_fwd_kvcache(const void* q, void* k_cache, void* v_cache, const void
                          float softcap, int num_splits, void* workspace, size_t ws_bytes,
                          fa_stream_t stream);
 
+/* Size of the fixed device scratch array behind fa_fwd_kvcache_noalloc. */
+#define FA_STATIC_SCRATCH_BYTES (8u * 1024u * 1024u)
+
+/*
+ * fa_fwd_kvcache without a workspace argument, for callers that cannot
+ * allocate device memory: e.g. a plugin inside a host runtime that owns all
+ * device allocations, or a serving loop whose device footprint is fixed after
+ * start-up.  The pages have no counterpart to this entry point; it exists for
+ * those callers only.
+ *   Arguments: as fa_fwd_kvcache, minus workspace and ws_bytes.  The caller
+ *   still owns and passes every input and output buffer.
+ *   Scratch: the split-KV partials go to one file-scope device array of
+ *   FA_STATIC_SCRATCH_BYTES (8 MiB) per GPU, part of the library's device
+ *   image and held until the process exits.  That fits
+ *   num_splits * B * Hq * Sq <= 16,256 partial rows at D=128 (32,263 at D=64);
+ *   larger requests return FA_ERR_INVALID_ARG before anything is launched.
+ *   The call allocates nothing: no cudaMalloc, cudaFree or allocating library
+ *   routine.
+ *   Set-up: the first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call before any stream capture.
+ *   Sharing: every call on a device uses the same array, which keeps the last
+ *   call's partials (nothing in it needs to start at zero: every partial row
+ *   is written before it is read).  Calls whose executions overlap on the GPU
+ *   (other streams, other host threads) race on the array and must be
+ *   serialised by the caller.
+ */
+fa_status fa_fwd_kvcache_noalloc(const void* q, void* k_cache, void* v_cache, const void* k_new,
+                                 const void* v_new, const int* cache_seqlens, const int* block_table,
+                                 int page_size, int max_pages_per_seq, int num_pages_or_max_seqlen,
+                                 void* out, float* lse, int B, int Sq, int Snew, int Hq, int Hkv, int D,
+                                 fa_dtype dt, float scale, int causal, int window_left, int window_right,
+                                 float softcap, int num_splits, fa_stream_t stream);
+
 /*
  * Waits for `stream`, then returns and clears the device status word of the
  * current device: FA_OK, FA_ERR_TIMEOUT (a bounded wait ran out) or

@@ -1,0 +1,81 @@
+"""fa_fwd_kvcache_noalloc, the decode entry point for callers that cannot
+allocate device memory (a plugin inside a runtime that owns all device
+memory, a serving loop with a fixed footprint): its split-KV partials live in
+a fixed device array inside libfa.so instead of a caller workspace.
+
+Checked through the C ABI against fa_fwd_kvcache (the workspace entry point)
+on two calls in a row with different inputs and split counts, since the array
+keeps the previous call's contents.  Collected last so that a stop-at-first-
+failure run has already run every other test; it also passes alone.
+"""
+
+import ctypes
+
+import pytest
+import torch
+
+from _parity import check_lse, check_out, f64
+from exact_attention_121_b200 import _lib, api, inputs
+
+pytestmark = pytest.mark.gpu
+
+SCRATCH_BYTES = 8 * 1024 * 1024
+DT = {torch.float16: _lib.FA_FP16, torch.bfloat16: _lib.FA_BF16}
+
+
+def _device_case(seed, dtype="bf16"):
+    d = inputs.kvcache_inputs(4, 32, 8, 128, 64, 6, 380, Sq=1, Snew=1, dtype=dtype, seed=seed)
+    return {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+
+
+def _noalloc(lib, d, num_splits, out, lse):
+    q = d["q"]
+    B, Sq, Hq, D = q.shape
+    stream = torch.cuda.current_stream().cuda_stream
+    return lib.fa_fwd_kvcache_noalloc(
+        q.data_ptr(), d["k_cache"].data_ptr(), d["v_cache"].data_ptr(), d["k_new"].data_ptr(),
+        d["v_new"].data_ptr(), d["cache_seqlens"].data_ptr(), d["block_table"].data_ptr(), d["page_size"],
+        d["block_table"].shape[1], d["k_cache"].shape[0], out.data_ptr(), lse.data_ptr(), B, Sq,
+        d["k_new"].shape[1], Hq, d["k_cache"].shape[2], D, DT[q.dtype], 0.0, 1, -1, -1, 0.0, num_splits,
+        ctypes.c_void_p(stream))
+
+
+def _reference(d, num_splits):
+    return api.fa_fwd_kvcache(d["q"], d["k_cache"], d["v_cache"], d["k_new"], d["v_new"], d["cache_seqlens"],
+                              d["block_table"], page_size=d["page_size"], causal=True, num_splits=num_splits)
+
+
+def test_noalloc_matches_workspace_entry_point_on_two_calls():
+    lib = _lib.load()
+    for seed, splits in ((31, 4), (32, 7)):
+        d = _device_case(seed)
+        ref_out, ref_lse = _reference(d, splits)
+        out = torch.empty_like(d["q"])
+        lse = torch.empty_like(ref_lse)
+        torch.cuda.synchronize()
+        before = torch.cuda.memory_allocated()
+        code = _noalloc(lib, d, splits, out, lse)
+        torch.cuda.synchronize()
+        assert code == _lib.FA_OK, api.fa_status_string(code)
+        assert api.fa_last_device_status() == 0
+        assert torch.cuda.memory_allocated() == before
+        check_out(out, f64(ref_out), torch.bfloat16)
+        check_lse(lse, f64(ref_lse))
+
+
+def test_noalloc_refuses_requests_beyond_the_array():
+    lib = _lib.load()
+    d = _device_case(33)
+    out = torch.empty_like(d["q"])
+    lse = torch.empty(4, 32, 1, device="cuda")
+    # 64 splits x 4 x 32 x 1 rows of 128 fp32 partials = 4 MiB + 32 KiB: fits
+    assert _noalloc(lib, d, 64, out, lse) == _lib.FA_OK
+    # 16,384 rows x 516 bytes > 8 MiB: refused before any launch
+    big = dict(d, q=torch.zeros(4, 2, 32, 128, dtype=torch.bfloat16, device="cuda"),
+               k_new=torch.zeros(4, 2, 8, 128, dtype=torch.bfloat16, device="cuda"),
+               v_new=torch.zeros(4, 2, 8, 128, dtype=torch.bfloat16, device="cuda"))
+    out2 = torch.empty_like(big["q"])
+    lse2 = torch.empty(4, 32, 2, device="cuda")
+    assert _noalloc(lib, big, 64, out2, lse2) == _lib.FA_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert api.fa_last_device_status() == 0
