@@ -304,11 +304,14 @@ class Tracer:
 # arms
 # ---------------------------------------------------------------------------
 
-def build_units(dev, workload):
+def build_units(dev, workload, point=None):
     from exact_attention_121_b200 import inputs
     units = []
-    if workload in ("full", "sweep"):
+    if workload in ("full", "sweep", "point"):
         for cfg in inputs.seqlen_sweep_configs():
+            u_name = "H%dD%dS%d%s" % (cfg["Hq"], cfg["D"], cfg["Sq"], "c" if cfg["causal"] else "n")
+            if workload == "point" and u_name != point:
+                continue
             units.append(AttnUnit(cfg, dev))
     if workload in ("full", "gqa"):
         units.append(AttnUnit(inputs.gqa_local_config(), dev))
@@ -400,7 +403,8 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="full", choices=["full", "sweep", "gqa", "decode", "small"])
+    ap.add_argument("--workload", default="full", choices=["full", "sweep", "gqa", "decode", "small", "point"])
+    ap.add_argument("--point", default="H16D128S4096n", help="sweep point for --workload point")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--detail", action="store_true", help="also print per-unit times")
@@ -426,7 +430,7 @@ def main():
 
     from exact_attention_121_b200 import _lib
     lib = _lib.load()
-    units = build_units(dev, args.workload)
+    units = build_units(dev, args.workload, args.point)
     flops_step = sum(u.flops() for u in units)
     peaks, peak_src = load_peaks()
 

@@ -32,6 +32,7 @@ SIGNATURES = {
                                     _I, _F, _I, _I, _I, _F, _I, _P]),
     "fa_last_device_status": (_I, [_P]),
     "fa_set_fwd_kernel": (None, [_I]),
+    "fa_set_bwd_kernel": (None, [_I]),
     "fa_selftest_bounded_wait": (_I, [_P, _I, ctypes.c_longlong, _P]),
     "fa_last_launch_count": (_I, []),
     "fa_set_trace_events": (None, [_P, _P]),

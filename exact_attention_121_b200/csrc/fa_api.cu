@@ -22,8 +22,9 @@ __device__ int g_fa_status = 0;
 constexpr int kMaxDevices = 64;
 int* g_status_ptr[kMaxDevices] = {nullptr};
 int g_fwd_kernel_choice = 0;
+int g_bwd_kernel_choice = 0;
 // Whether the automatic choice uses the tcgen05 forward kernel.
-constexpr bool kTcAuto = false;
+constexpr bool kTcAuto = true;
 cudaEvent_t g_trace_start = nullptr, g_trace_stop = nullptr;
 thread_local int g_last_launches = 0;
 
@@ -122,6 +123,8 @@ const char* fa_status_string(fa_status s) {
 
 void fa_set_fwd_kernel(int which) { g_fwd_kernel_choice = which; }
 
+void fa_set_bwd_kernel(int which) { g_bwd_kernel_choice = which; }
+
 int fa_last_launch_count(void) { return g_last_launches; }
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk,
@@ -199,6 +202,7 @@ fa_status fa_bwd(const void* dout, const void* q, const void* k, const void* v, 
   p.scale = scale;
   fill_cap(scale, softcap, &p.softcap, &p.cap_in, &p.cap_log2, &p.scale_log2);
   p.deterministic = deterministic ? 1 : 0;
+  p.kernel_choice = g_bwd_kernel_choice;
   p.status = status_ptr();
   if (!p.status) return FA_ERR_CUDA;
   int launches = 0;

@@ -393,7 +393,12 @@ cudaError_t launch_bwd_t(const BwdParams& p, cudaStream_t s, int* launches) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   ++*launches;
-  e = (p.D == 64) ? launch_main_d<T, 64>(p, s) : launch_main_d<T, 128>(p, s);
+  const bool tc = (p.kernel_choice == 0 || p.kernel_choice == 2) && bwd_tc_supported(p);
+  if (p.kernel_choice == 2 && !tc) return cudaErrorNotSupported;
+  if (tc)
+    e = launch_bwd_main_tc(p, Elem<T>::kBf16 ? FA_BF16 : FA_FP16, s);
+  else
+    e = (p.D == 64) ? launch_main_d<T, 64>(p, s) : launch_main_d<T, 128>(p, s);
   if (e != cudaSuccess) return e;
   ++*launches;
   bwd_convert_kernel<T><<<148 * 8, 256, 0, s>>>(p);

@@ -1,0 +1,467 @@
+// Backward attention on the Blackwell tensor-memory path (tcgen05 + TMA),
+// head dim 128, float32 atomic-style dQ accumulation through bulk reductions.
+//
+// The method: "FlashAttention 实战指南" (mhpq.cn), the three techniques — the
+// backward pass recomputes the attention probabilities from the saved row
+// log-sum-exp instead of reading a stored matrix.
+//
+// One CTA owns 128 keys of one (batch, kv-head) and walks every q-head of the
+// GQA group and every 64-row query block that can see those keys.  Per
+// iteration i (query block Q_i, dO_i, LSE_i, Delta_i):
+//   S^T  = K Q_i^T        (M=128 keys, N=64 queries, K=D)      -> TMEM
+//   dP^T = V dO_i^T                                            -> TMEM
+//   P^T  = exp(S^T - LSE), dS^T = P^T (dP^T - Delta) [* (1 - tanh^2)]
+//          (warps 0-3, thread = key = TMEM lane; P^T and dS^T go back to
+//           TMEM in 16 bits, dS^T also to shared memory)
+//   dV  += P^T dO_i       (A = P^T from TMEM)                  -> TMEM
+//   dK  += dS^T Q_i       (A = dS^T from TMEM)                 -> TMEM
+//   dQ^T = K^T dS^T       (M=128 head dims, N=64 queries)      -> TMEM
+//   dQ  += dQ^T^T         (warps 4-7, thread = head-dim index: TMEM ->
+//                          shared memory -> bulk fp32 add into the dQ
+//                          accumulator in global memory)
+// S^T/dP^T live in two TMEM buffers, so the elementwise work of iteration i
+// overlaps the products of iteration i+1.  TMEM (512 columns): buffer x at
+// [128x, 128x+128) holds S^T | dP^T, then P^T | dS^T | dQ^T; dV [256,384),
+// dK [384,512).  Warp 8 loads (TMA for K, V, Q_i, dO_i; plain loads for
+// LSE/Delta), warp 9 issues the MMAs.  Every wait is bounded.
+#include <math.h>
+
+#include "fa_common.cuh"
+#include "fa_kernels.h"
+#include "fa_sm100.cuh"
+#include "fa_tma.h"
+
+namespace fa {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kKeys = 128;
+constexpr int kQ = 64;
+constexpr int kThreadsB = 320;
+constexpr int kDqWarp0 = 4;
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarpB = 9;
+constexpr unsigned long long kWaitNs = kWaitLimitNs;
+
+struct BwdTcCfg {
+  static constexpr int D = 128;
+  static constexpr int KV_CHUNK = kKeys * 128;    // 128 rows x 64 columns, 16-bit, swizzled
+  static constexpr int KV_TILE = 2 * KV_CHUNK;
+  static constexpr int Q_CHUNK = kQ * 128;        // 64 rows x 64 columns
+  static constexpr int Q_TILE = 2 * Q_CHUNK;
+  static constexpr int DS_TILE = kKeys * kQ * 2;  // [128 keys][64 queries] 16-bit, swizzled
+  static constexpr int DQ_WARP = kQ * 32 * 4;     // per drain warp: [64 queries][32 dims] fp32
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + KV_TILE;
+  static constexpr int OFF_Q = OFF_V + KV_TILE;       // 2 stages
+  static constexpr int OFF_DO = OFF_Q + 2 * Q_TILE;   // 2 stages
+  static constexpr int OFF_DS = OFF_DO + 2 * Q_TILE;  // 2 buffers
+  static constexpr int OFF_DQ = OFF_DS + 2 * DS_TILE;  // 4 warps
+  static constexpr int OFF_ROW = OFF_DQ + 4 * DQ_WARP;  // [stage][LSE*log2e 64 | Delta 64]
+  static constexpr int OFF_BAR = OFF_ROW + 2 * 2 * kQ * 4;
+  enum { B_KV = 0, B_QF = 1, B_QE = 3, B_SDP = 5, B_PDS = 7, B_DQF = 9, B_TMF = 11, B_FIN = 13, B_DRAIN = 14,
+         NBAR = 15 };
+  static constexpr int OFF_TMEM = OFF_BAR + 8 * NBAR;
+  static constexpr int OFF_ABORT = OFF_TMEM + 4;
+  static constexpr int SMEM = OFF_ABORT + 4 + 1024;
+};
+
+__device__ __forceinline__ float f32(uint32_t u) { return __uint_as_float(u); }
+
+template <typename T, bool kCap>
+__global__ void __launch_bounds__(kThreadsB, 1)
+    bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                  const BwdParams p) {
+  using C = BwdTcCfg;
+  constexpr int D = C::D;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sb + C::OFF_BAR + 8 * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
+  const uint32_t* tmem_slot = reinterpret_cast<const uint32_t*>(smem + C::OFF_TMEM);
+  float* rows = reinterpret_cast<float*>(smem + C::OFF_ROW);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nkb = (p.Sk + kKeys - 1) / kKeys;
+  const int kb = blockIdx.x % nkb;
+  const int hkv = (blockIdx.x / nkb) % p.Hkv;
+  const int b = blockIdx.x / (nkb * p.Hkv);
+  const int off = p.Sk - p.Sq;
+  const int k0 = kb * kKeys;
+  const int k1 = min(k0 + kKeys, p.Sk) - 1;
+  int i_min = 0, i_max = p.Sq - 1;
+  if (p.wr >= 0) i_min = max(i_min, k0 - off - p.wr);
+  if (p.wl >= 0) i_max = min(i_max, k1 - off + p.wl);
+  const int qb_lo = i_min / kQ;
+  const int n_qb = (i_max >= i_min) ? (i_max / kQ - qb_lo + 1) : 0;
+  const int n_iter = n_qb * p.G;
+  auto iter_q = [&](int it, int& h, int& q0) {
+    h = hkv * p.G + it / n_qb;
+    q0 = (qb_lo + it % n_qb) * kQ;
+  };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::B_KV), 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar(C::B_QF + x), 1);
+      mbar_init(bar(C::B_QE + x), 1);
+      mbar_init(bar(C::B_SDP + x), 1);
+      mbar_init(bar(C::B_PDS + x), 128);
+      mbar_init(bar(C::B_DQF + x), 1);
+      mbar_init(bar(C::B_TMF + x), 128);
+    }
+    mbar_init(bar(C::B_FIN), 1);
+    mbar_init(bar(C::B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarpB) {
+    tmem_alloc(sb + C::OFF_TMEM, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  auto fail = [&]() {
+    *abort_flag = 1;
+    report_status(p.status, kStatusTimeout);
+  };
+
+  if (warp == kLoadWarp) {
+    // -------------------------------------------------------------- loads
+    if (n_iter > 0) {
+      if (lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        tma_prefetch_desc(&tmdO);
+        mbar_expect_tx(bar(C::B_KV), 2 * C::KV_TILE);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_4d(sb + C::OFF_K + c * C::KV_CHUNK, &tmK, c * 64, hkv, k0, b, bar(C::B_KV));
+          tma_load_4d(sb + C::OFF_V + c * C::KV_CHUNK, &tmV, c * 64, hkv, k0, b, bar(C::B_KV));
+        }
+      }
+      int issued = 0;
+      for (int it = 0; it < n_iter; ++it) {
+        const int st = it & 1, u = it >> 1;
+        if (it >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar(C::B_QE + st), (u - 1) & 1, abort_flag, kWaitNs))) {
+          if (lane == 0) fail();
+          break;
+        }
+        int h, q0;
+        iter_q(it, h, q0);
+        float* r = rows + st * 2 * kQ;
+        const float* L = p.lse + ((size_t)b * p.Hq + h) * p.Sq;
+        const float* Dl = p.delta + ((size_t)b * p.Hq + h) * p.Sq;
+        for (int t = lane; t < kQ; t += 32) {
+          const int q = q0 + t;
+          float l2 = INFINITY, dl = 0.f;
+          if (q < p.Sq) {
+            const float l = L[q];
+            l2 = (l == -INFINITY) ? INFINITY : l * kLog2e;
+            dl = Dl[q];
+          }
+          r[t] = l2;
+          r[kQ + t] = dl;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_expect_tx(bar(C::B_QF + st), 2 * C::Q_TILE);
+          for (int c = 0; c < 2; ++c) {
+            tma_load_4d(sb + C::OFF_Q + st * C::Q_TILE + c * C::Q_CHUNK, &tmQ, c * 64, h, q0, b, bar(C::B_QF + st));
+            tma_load_4d(sb + C::OFF_DO + st * C::Q_TILE + c * C::Q_CHUNK, &tmdO, c * 64, h, q0, b,
+                        bar(C::B_QF + st));
+          }
+        }
+        issued = it + 1;
+      }
+      if (*abort_flag && lane == 0) {
+        volatile int never = 0;
+        mbar_wait(bar(C::B_KV), 0, &never, kWaitNs);
+        for (int it = max(0, issued - 2); it < issued; ++it)
+          mbar_wait(bar(C::B_QF + (it & 1)), (it >> 1) & 1, &never, kWaitNs);
+      }
+    }
+  } else if (warp == kMmaWarpB) {
+    // -------------------------------------------------------------- MMA issue
+    if (lane == 0 && n_iter > 0) {
+      constexpr bool kBf = Elem<T>::kBf16;
+      constexpr uint32_t idesc_s = make_idesc(kBf, 128, kQ, false, false);
+      constexpr uint32_t idesc_kv = make_idesc(kBf, 128, D, true, false);
+      constexpr uint32_t idesc_dq = make_idesc(kBf, 128, kQ, true, true);
+      const uint32_t tdV = tmem + 256, tdK = tmem + 384;
+      auto issue_sdp = [&](int it) {
+        const int x = it & 1;
+        const uint32_t tb = tmem + x * 128;
+        const uint32_t q_st = sb + C::OFF_Q + x * C::Q_TILE, do_st = sb + C::OFF_DO + x * C::Q_TILE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t okv = (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32;
+          const uint32_t oq = (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32;
+          mma_ss(tb, make_sdesc_sw128(sb + C::OFF_K + okv, 16, 1024), make_sdesc_sw128(q_st + oq, 16, 1024),
+                 idesc_s, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t okv = (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32;
+          const uint32_t oq = (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32;
+          mma_ss(tb + 64, make_sdesc_sw128(sb + C::OFF_V + okv, 16, 1024), make_sdesc_sw128(do_st + oq, 16, 1024),
+                 idesc_s, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_grads = [&](int it) {
+        const int x = it & 1;
+        const uint32_t tb = tmem + x * 128;
+        const uint32_t q_st = sb + C::OFF_Q + x * C::Q_TILE, do_st = sb + C::OFF_DO + x * C::Q_TILE;
+        const uint32_t ds = sb + C::OFF_DS + x * C::DS_TILE;
+        const bool acc = it > 0;
+#pragma unroll
+        for (int kk = 0; kk < kQ / 16; ++kk)
+          mma_ts(tdV, tb + kk * 8, make_sdesc_sw128(do_st + kk * 16 * 128, C::Q_CHUNK, 1024), idesc_kv,
+                 (acc || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < kQ / 16; ++kk)
+          mma_ts(tdK, tb + 32 + kk * 8, make_sdesc_sw128(q_st + kk * 16 * 128, C::Q_CHUNK, 1024), idesc_kv,
+                 (acc || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk)
+          mma_ss(tb + 64, make_sdesc_sw128(sb + C::OFF_K + kk * 16 * 128, C::KV_CHUNK, 1024),
+                 make_sdesc_sw128(ds + kk * 16 * 128, C::KV_CHUNK, 1024), idesc_dq, kk > 0 ? 1u : 0u);
+      };
+      bool ok = mbar_wait(bar(C::B_KV), 0, abort_flag, kWaitNs) && mbar_wait(bar(C::B_QF), 0, abort_flag, kWaitNs);
+      if (ok) {
+        tc_fence_after();
+        issue_sdp(0);
+        mma_commit(bar(C::B_SDP));
+      }
+      for (int it = 0; ok && it < n_iter; ++it) {
+        const int x = it & 1, u = it >> 1;
+        if (it + 1 < n_iter) {
+          const int x1 = (it + 1) & 1, u1 = (it + 1) >> 1;
+          ok = mbar_wait(bar(C::B_QF + x1), u1 & 1, abort_flag, kWaitNs) &&
+               (it + 1 < 2 || mbar_wait(bar(C::B_TMF + x1), (u1 - 1) & 1, abort_flag, kWaitNs));
+          if (!ok) break;
+          tc_fence_after();
+          issue_sdp(it + 1);
+          mma_commit(bar(C::B_SDP + x1));
+        }
+        ok = mbar_wait(bar(C::B_PDS + x), u & 1, abort_flag, kWaitNs);
+        if (!ok) break;
+        tc_fence_after();
+        issue_grads(it);
+        mma_commit(bar(C::B_DQF + x));
+        mma_commit(bar(C::B_QE + x));
+      }
+      if (ok) mma_commit(bar(C::B_FIN));
+      if (!ok) fail();
+      mma_commit(bar(C::B_DRAIN));
+      volatile int never = 0;
+      mbar_wait(bar(C::B_DRAIN), 0, &never, kWaitNs);
+    }
+  } else if (warp < kDqWarp0) {
+    // -------------------------------------------------------------- P^T, dS^T
+    const int r = warp * 32 + lane;
+    const int key = k0 + r;
+    const bool key_ok = key <= k1;
+    const uint32_t lanes = (uint32_t)(warp * 32) << 16;
+    bool ok = true;
+    for (int it = 0; it < n_iter; ++it) {
+      const int x = it & 1, u = it >> 1;
+      int h, q0;
+      iter_q(it, h, q0);
+      (void)h;
+      bool w = mbar_wait(bar(C::B_SDP + x), u & 1, abort_flag, kWaitNs);
+      if (it >= 2) w = w && mbar_wait(bar(C::B_DQF + x), (u - 1) & 1, abort_flag, kWaitNs);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tb = tmem + lanes + x * 128;
+      uint32_t s[kQ], dp[kQ];
+      tmem_ld32(tb + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+      tmem_ld32(tb + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+      tmem_ld32(tb + 64, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+      tmem_ld32(tb + 96, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+      tmem_wait_ld();
+      reg_fence(s);
+      reg_fence(dp);
+      const float* rw = rows + x * 2 * kQ;
+      const bool full = (k1 - k0 + 1 == kKeys) && (q0 + kQ <= p.Sq) &&
+                        (p.wl < 0 || k0 >= q0 + kQ - 1 + off - p.wl) && (p.wr < 0 || k1 <= q0 + off + p.wr);
+      uint32_t pk[kQ / 2], dk[kQ / 2];
+#pragma unroll
+      for (int c = 0; c < kQ; c += 2) {
+        float pv[2], dv[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float l2 = rw[c + e];
+          const float dl = rw[kQ + c + e];
+          float xv, fac = 1.f;
+          if (kCap) {
+            const float t = tanh_exp(f32(s[c + e]) * p.cap_in);
+            xv = p.cap_log2 * t;
+            fac = 1.f - t * t;
+          } else {
+            xv = f32(s[c + e]) * p.scale_log2;
+          }
+          float pe = fast_exp2(xv - l2);
+          if (!full) {
+            const int qp = q0 + c + e + off;
+            const bool vis = key_ok && (p.wl < 0 || key >= qp - p.wl) && (p.wr < 0 || key <= qp + p.wr);
+            pe = vis ? pe : 0.f;
+          }
+          pv[e] = pe;
+          dv[e] = pe * (f32(dp[c + e]) - dl) * fac;
+        }
+        pk[c / 2] = Elem<T>::pack(pv[0], pv[1]);
+        dk[c / 2] = Elem<T>::pack(dv[0], dv[1]);
+      }
+      tmem_st16(tb + 0, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+      tmem_st16(tb + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+      tmem_st16(tb + 32, *reinterpret_cast<uint32_t(*)[16]>(&dk[0]));
+      tmem_st16(tb + 48, *reinterpret_cast<uint32_t(*)[16]>(&dk[16]));
+      // dS^T row r -> shared memory, 128-byte swizzle (MN-major operand of dQ^T)
+      uint8_t* dsrow = smem + C::OFF_DS + x * C::DS_TILE + r * 128;
+#pragma unroll
+      for (int g = 0; g < 8; ++g)
+        *reinterpret_cast<uint4*>(dsrow + ((g ^ (r & 7)) << 4)) =
+            make_uint4(dk[4 * g], dk[4 * g + 1], dk[4 * g + 2], dk[4 * g + 3]);
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_PDS + x));
+    }
+    if (ok && n_iter > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_FIN), 0, abort_flag, kWaitNs));
+    if (!ok) {
+      fail();
+    } else {
+      tc_fence_after();
+      const size_t ks = (size_t)p.Hkv * D;
+      T* dVr = reinterpret_cast<T*>(p.dv) + ((size_t)b * p.Sk + key) * ks + (size_t)hkv * D;
+      T* dKr = reinterpret_cast<T*>(p.dk) + ((size_t)b * p.Sk + key) * ks + (size_t)hkv * D;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const float mul = which ? p.scale : 1.f;
+        T* dst = which ? dKr : dVr;
+        const uint32_t src = tmem + lanes + (which ? 384 : 256);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          if (n_iter > 0) {
+            tmem_ld32(src + c * 32, v);
+            tmem_wait_ld();
+            reg_fence(v);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
+          }
+          if (key_ok) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              uint4 o;
+              o.x = Elem<T>::pack(f32(v[8 * g + 0]) * mul, f32(v[8 * g + 1]) * mul);
+              o.y = Elem<T>::pack(f32(v[8 * g + 2]) * mul, f32(v[8 * g + 3]) * mul);
+              o.z = Elem<T>::pack(f32(v[8 * g + 4]) * mul, f32(v[8 * g + 5]) * mul);
+              o.w = Elem<T>::pack(f32(v[8 * g + 6]) * mul, f32(v[8 * g + 7]) * mul);
+              *reinterpret_cast<uint4*>(dst + c * 32 + 8 * g) = o;
+            }
+          }
+        }
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- dQ drain
+    const int wq = warp - kDqWarp0;          // TMEM lane quarter = head-dim slice
+    const uint32_t lanes = (uint32_t)(wq * 32) << 16;
+    float* tile = reinterpret_cast<float*>(smem + C::OFF_DQ + wq * C::DQ_WARP);  // [64 q][32 dims]
+    const uint32_t tile_s = sb + C::OFF_DQ + wq * C::DQ_WARP;
+    bool ok = true;
+    for (int it = 0; it < n_iter; ++it) {
+      const int x = it & 1, u = it >> 1;
+      int h, q0;
+      iter_q(it, h, q0);
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(C::B_DQF + x), u & 1, abort_flag, kWaitNs))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t v[kQ];
+      const uint32_t tb = tmem + lanes + x * 128 + 64;
+      tmem_ld32(tb, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tmem_ld32(tb + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      tmem_wait_ld();
+      reg_fence(v);
+      tc_fence_before();
+      mbar_arrive(bar(C::B_TMF + x));
+      // the previous iteration's reductions have read the tile (lane-local
+      // wait, then the warp agrees before anyone overwrites it)
+      bulk_wait_read_all();
+      __syncwarp();
+#pragma unroll
+      for (int c = 0; c < kQ; ++c) tile[c * 32 + lane] = f32(v[c]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      float* gbase = p.dq_accum + ((size_t)b * p.Sq) * p.Hq * D + (size_t)h * D + wq * 32;
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        const int row = lane + 32 * rr;
+        const int q = q0 + row;
+        if (q < p.Sq) bulk_reduce_add_f32(gbase + (size_t)q * p.Hq * D, tile_s + row * 128, 128);
+      }
+      bulk_commit();
+    }
+    bulk_wait_all();
+    if (!ok) fail();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarpB) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <typename T, bool kCap>
+cudaError_t launch_t(const BwdParams& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                     const CUtensorMap& mdo, cudaStream_t s) {
+  auto kern = bwd_tc_kernel<T, kCap>;
+  constexpr int smem = BwdTcCfg::SMEM;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int nkb = (p.Sk + kKeys - 1) / kKeys;
+  const long long items = (long long)nkb * p.Hkv * p.B;
+  if (items == 0) return cudaSuccess;
+  trace_begin(s);
+  kern<<<(unsigned)items, kThreadsB, smem, s>>>(mq, mk, mv, mdo, p);
+  trace_end(s);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool bwd_tc_supported(const BwdParams& p) {
+  return p.D == 128 && !p.deterministic && p.Sq >= 1 && p.Sk >= 1 && tma_available();
+}
+
+cudaError_t launch_bwd_main_tc(const BwdParams& p, fa_dtype dt, cudaStream_t s) {
+  CUtensorMap mq, mk, mv, mdo;
+  const bool bf = dt == FA_BF16;
+  if (!make_bshd_map(&mq, p.q, bf, p.D, p.Hq, p.Sq, p.B, kQ) ||
+      !make_bshd_map(&mdo, p.dout, bf, p.D, p.Hq, p.Sq, p.B, kQ) ||
+      !make_bshd_map(&mk, p.k, bf, p.D, p.Hkv, p.Sk, p.B, kKeys) ||
+      !make_bshd_map(&mv, p.v, bf, p.D, p.Hkv, p.Sk, p.B, kKeys))
+    return cudaErrorNotSupported;
+  const bool cap = p.softcap > 0.f;
+  if (bf) return cap ? launch_t<__nv_bfloat16, true>(p, mq, mk, mv, mdo, s) : launch_t<__nv_bfloat16, false>(p, mq, mk, mv, mdo, s);
+  return cap ? launch_t<__half, true>(p, mq, mk, mv, mdo, s) : launch_t<__half, false>(p, mq, mk, mv, mdo, s);
+}
+
+}  // namespace fa

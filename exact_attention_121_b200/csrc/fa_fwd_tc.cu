@@ -1,11 +1,441 @@
-// Forward attention on the Blackwell tensor-memory path (tcgen05): placeholder
-// until the kernel lands; fa_fwd falls back to the mma.sync kernel.
+// Forward attention on the Blackwell tensor-memory path (tcgen05 + TMA).
+//
+// The method is the one described in "FlashAttention 实战指南" (mhpq.cn), the
+// three techniques: tiles of Q, K, V are brought on chip, QK^T and its
+// softmax are formed there with a running row maximum and running sum, and the
+// n x n score matrix never reaches device memory.
+//
+// B200 design.  One CTA owns 256 query rows of one (batch, q-head) as two
+// 128-row tiles A and B, and 320 threads in four roles:
+//   warps 0-3  softmax of tile A  (thread = row = TMEM lane)
+//   warps 4-7  softmax of tile B
+//   warp  8    TMA producer: Q once, then K/V 128-key tiles through a ring of
+//              shared-memory stages (128-byte swizzle, zero fill past the ends)
+//   warp  9    MMA issuer: tcgen05.mma with fp32 accumulators in TMEM
+// Tensor memory (512 columns): S_A [0,128), S_B [128,256), O_A [256,256+D),
+// O_B [384,384+D); P (16-bit) is written over the first 64 columns of S and is
+// the A operand of O += P V straight from TMEM.  Per key tile j the MMA warp
+// issues  PV_A(j), S_A(j+1), PV_B(j), S_B(j+1),  so one tile's softmax overlaps
+// the other tile's products.  Because a tcgen05.commit tracks every earlier MMA
+// of the issuing thread, "S(j+1) is ready" also means "PV(j) is done", which is
+// when a softmax warp may rescale its O rows in TMEM.  The running maximum is
+// only moved (and O rescaled) when it grows by more than 2^8, which keeps
+// every exponent <= 2^8 and makes rescales rare.  O is divided by the sum of
+// the 16-bit probabilities the P.V product used (so the rounding of a
+// dominant probability cancels), the LSE uses the sum of the fp32 values.
+// Every wait is bounded; a timeout records FA_ERR_TIMEOUT and the CTA drains
+// its asynchronous work and exits.
+#include <math.h>
+
+#include "fa_common.cuh"
 #include "fa_kernels.h"
+#include "fa_sm100.cuh"
+#include "fa_tma.h"
 
 namespace fa {
 
-bool fwd_tc_supported(const FwdParams&) { return false; }
+namespace {
 
-cudaError_t launch_fwd_tc(const FwdParams&, fa_dtype, cudaStream_t, int*) { return cudaErrorNotSupported; }
+using namespace sm100;
+
+constexpr int kRows = 128;           // rows per Q tile, keys per K/V tile
+constexpr int kThreadsTC = 320;
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr float kRescaleLog2 = 8.0f;
+constexpr unsigned long long kTcWaitNs = kWaitLimitNs;
+
+template <int D>
+struct TcCfg {
+  static constexpr int CHUNK = kRows * 128;          // one 64-column, 128-row swizzled chunk (16 KB)
+  static constexpr int NCHUNK = D / 64;
+  static constexpr int TILE = CHUNK * NCHUNK;        // one 128-row tile
+  static constexpr int NSK = (D == 128) ? 3 : 4;     // K stages
+  static constexpr int NSV = (D == 128) ? 2 : 4;     // V stages
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = 2 * TILE;
+  static constexpr int OFF_V = OFF_K + NSK * TILE;
+  static constexpr int OFF_BAR = OFF_V + NSV * TILE;
+  // barrier indices
+  static constexpr int B_Q = 0;
+  static constexpr int B_KF = 1;             // NSK: K tile landed
+  static constexpr int B_KE = B_KF + NSK;    // NSK: K stage free (both QK^T products done)
+  static constexpr int B_VF = B_KE + NSK;    // NSV: V tile landed
+  static constexpr int B_VE = B_VF + NSV;    // NSV: V stage free (both PV products done)
+  static constexpr int B_S = B_VE + NSV;     // 2
+  static constexpr int B_P = B_S + 2;        // 2
+  static constexpr int B_O = B_P + 2;        // 2
+  static constexpr int B_DRAIN = B_O + 2;
+  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int OFF_TMEM = OFF_BAR + 8 * NBAR;
+  static constexpr int OFF_ABORT = OFF_TMEM + 4;
+  static constexpr int SMEM = OFF_ABORT + 4 + 1024;  // + alignment slack
+};
+
+__device__ __forceinline__ float f32(uint32_t u) { return __uint_as_float(u); }
+
+template <typename T, int D, bool kCap>
+__global__ void __launch_bounds__(kThreadsTC, 1)
+    fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using C = TcCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sb + C::OFF_BAR + 8 * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
+  const uint32_t* tmem_slot = reinterpret_cast<const uint32_t*>(smem + C::OFF_TMEM);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_qp = (p.Sq + 2 * kRows - 1) / (2 * kRows);
+  const int qp = (p.wr >= 0) ? (n_qp - 1 - (int)blockIdx.x) : (int)blockIdx.x;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int g = h / p.G;
+  const int q0 = qp * 2 * kRows;
+  const int off = p.Sk - p.Sq;
+  const int qlast = min(q0 + 2 * kRows, p.Sq) - 1;
+  int kmin = 0, kmax = p.Sk - 1;
+  if (p.wl >= 0) kmin = max(kmin, q0 + off - p.wl);
+  if (p.wr >= 0) kmax = min(kmax, qlast + off + p.wr);
+  const int kt_begin = kmin / kRows;
+  const int n_tiles = (kmax >= kmin) ? (kmax / kRows + 1 - kt_begin) : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::B_Q), 1);
+    for (int s = 0; s < C::NSK; ++s) {
+      mbar_init(bar(C::B_KF + s), 1);
+      mbar_init(bar(C::B_KE + s), 1);
+    }
+    for (int s = 0; s < C::NSV; ++s) {
+      mbar_init(bar(C::B_VF + s), 1);
+      mbar_init(bar(C::B_VE + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(C::B_S + t), 1);
+      mbar_init(bar(C::B_P + t), 4 * 32);
+      mbar_init(bar(C::B_O + t), 1);
+    }
+    mbar_init(bar(C::B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(sb + C::OFF_TMEM, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto fail = [&]() {
+    *abort_flag = 1;
+    report_status(p.status, kStatusTimeout);
+  };
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && n_tiles > 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      mbar_expect_tx(bar(C::B_Q), 2 * C::TILE);
+      for (int t = 0; t < 2; ++t)
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_load_4d(sb + C::OFF_Q + t * C::TILE + c * C::CHUNK, &tmQ, c * 64, h, q0 + t * kRows, b, bar(C::B_Q));
+      int issued = 0;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int sk = j % C::NSK, uk = j / C::NSK;
+        const int sv = j % C::NSV, uv = j / C::NSV;
+        const int k0 = (kt_begin + j) * kRows;
+        if (j >= C::NSK && !mbar_wait(bar(C::B_KE + sk), (uk - 1) & 1, abort_flag, kTcWaitNs)) {
+          fail();
+          break;
+        }
+        mbar_expect_tx(bar(C::B_KF + sk), C::TILE);
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_load_4d(sb + C::OFF_K + sk * C::TILE + c * C::CHUNK, &tmK, c * 64, g, k0, b, bar(C::B_KF + sk));
+        if (j >= C::NSV && !mbar_wait(bar(C::B_VE + sv), (uv - 1) & 1, abort_flag, kTcWaitNs)) {
+          fail();
+          issued = -(j + 1);  // K of tile j is in flight, V is not
+          break;
+        }
+        mbar_expect_tx(bar(C::B_VF + sv), C::TILE);
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_load_4d(sb + C::OFF_V + sv * C::TILE + c * C::CHUNK, &tmV, c * 64, g, k0, b, bar(C::B_VF + sv));
+        issued = j + 1;
+      }
+      if (*abort_flag) {
+        // let every load still in flight land before the CTA exits
+        volatile int never = 0;
+        const int nk = issued < 0 ? -issued : issued;   // tiles whose K was issued
+        const int nv = issued < 0 ? nk - 1 : issued;    // tiles whose V was issued
+        mbar_wait(bar(C::B_Q), 0, &never, kTcWaitNs);
+        for (int j = max(0, nk - C::NSK); j < nk; ++j)
+          mbar_wait(bar(C::B_KF + j % C::NSK), (j / C::NSK) & 1, &never, kTcWaitNs);
+        for (int j = max(0, nv - C::NSV); j < nv; ++j)
+          mbar_wait(bar(C::B_VF + j % C::NSV), (j / C::NSV) & 1, &never, kTcWaitNs);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0 && n_tiles > 0) {
+      constexpr bool kBf = Elem<T>::kBf16;
+      constexpr uint32_t idesc_qk = make_idesc(kBf, 128, 128, false);
+      constexpr uint32_t idesc_pv = make_idesc(kBf, 128, D, true);
+      const uint32_t tS[2] = {tmem, tmem + 128};
+      const uint32_t tO[2] = {tmem + 256, tmem + 384};
+      auto issue_qk = [&](int t, int st) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+          const uint64_t ad = make_sdesc_sw128(sb + C::OFF_Q + t * C::TILE + koff, 16, 1024);
+          const uint64_t bd = make_sdesc_sw128(sb + C::OFF_K + st * C::TILE + koff, 16, 1024);
+          mma_ss(tS[t], ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int st, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < kRows / 16; ++kk) {
+          const uint64_t bd = make_sdesc_sw128(sb + C::OFF_V + st * C::TILE + kk * 16 * 128, C::CHUNK, 1024);
+          mma_ts(tO[t], tS[t] + kk * 8, bd, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(bar(C::B_Q), 0, abort_flag, kTcWaitNs);
+      ok = ok && mbar_wait(bar(C::B_KF + 0), 0, abort_flag, kTcWaitNs);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0, 0);
+        mma_commit(bar(C::B_S + 0));
+        issue_qk(1, 0);
+        mma_commit(bar(C::B_S + 1));
+        mma_commit(bar(C::B_KE + 0));
+      }
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int sv = j % C::NSV, uv = j / C::NSV;
+        const int sk1 = (j + 1) % C::NSK, uk1 = (j + 1) / C::NSK;
+        const bool more = j + 1 < n_tiles;
+        ok = mbar_wait(bar(C::B_VF + sv), uv & 1, abort_flag, kTcWaitNs) &&
+             mbar_wait(bar(C::B_P + 0), j & 1, abort_flag, kTcWaitNs);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(0, sv, j > 0);
+        if (more) {
+          ok = mbar_wait(bar(C::B_KF + sk1), uk1 & 1, abort_flag, kTcWaitNs);
+          if (!ok) break;
+          tc_fence_after();
+          issue_qk(0, sk1);
+          mma_commit(bar(C::B_S + 0));
+        } else {
+          mma_commit(bar(C::B_O + 0));
+        }
+        ok = mbar_wait(bar(C::B_P + 1), j & 1, abort_flag, kTcWaitNs);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(1, sv, j > 0);
+        mma_commit(bar(C::B_VE + sv));
+        if (more) {
+          issue_qk(1, sk1);
+          mma_commit(bar(C::B_S + 1));
+          mma_commit(bar(C::B_KE + sk1));
+        } else {
+          mma_commit(bar(C::B_O + 1));
+        }
+      }
+      if (!ok) fail();
+      // drain: every MMA issued above has completed before TMEM is released
+      mma_commit(bar(C::B_DRAIN));
+      volatile int never = 0;
+      mbar_wait(bar(C::B_DRAIN), 0, &never, kTcWaitNs);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int t = warp >> 2;       // Q tile
+    const int wq = warp & 3;       // lane quarter
+    const int r = wq * 32 + lane;  // row in the tile = TMEM lane
+    const uint32_t lanes = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lanes + t * 128;
+    const uint32_t tO = tmem + lanes + 256 + t * 128;
+    const int qi = q0 + t * kRows + r;
+    const int qpos = qi + off;
+    const int qpos_first = q0 + off, qpos_last = qlast + off;
+    float m_run = -INFINITY, l_run = 0.f, l_q = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      // warp-uniform outcome: the TMEM accesses below are warp-collective
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(C::B_S + t), j & 1, abort_flag, kTcWaitNs))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t s[kRows];  // raw scores (fp32 bits), then log2-domain scores
+      tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+      tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+      tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+      tmem_wait_ld();
+      reg_fence(s);
+      const int k0 = (kt_begin + j) * kRows;
+      const bool full = (k0 + kRows <= p.Sk) && (p.wl < 0 || k0 >= qpos_last - p.wl) &&
+                        (p.wr < 0 || k0 + kRows - 1 <= qpos_first + p.wr);
+      // row maximum in the log2 domain (the scale is positive: max commutes)
+      float mx = -INFINITY;
+      if (kCap) {
+#pragma unroll
+        for (int i = 0; i < kRows; ++i) s[i] = __float_as_uint(p.cap_log2 * tanh_exp(f32(s[i]) * p.cap_in));
+      }
+      if (!full) {
+#pragma unroll
+        for (int i = 0; i < kRows; ++i) {
+          const int key = k0 + i;
+          const bool vis = key < p.Sk && (p.wl < 0 || key >= qpos - p.wl) && (p.wr < 0 || key <= qpos + p.wr);
+          if (!vis) s[i] = __float_as_uint(-INFINITY);
+        }
+      }
+      {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int i = 0; i < kRows; i += 4) {
+          m4[0] = fmaxf(m4[0], f32(s[i]));
+          m4[1] = fmaxf(m4[1], f32(s[i + 1]));
+          m4[2] = fmaxf(m4[2], f32(s[i + 2]));
+          m4[3] = fmaxf(m4[3], f32(s[i + 3]));
+        }
+        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      }
+      const float sl = kCap ? 1.f : p.scale_log2;  // multiplier into the log2 domain
+      mx *= sl;
+      // lazy rescale: move the running max only when it grows by > 2^8
+      const bool move = (mx > m_run + kRescaleLog2) || (m_run == -INFINITY && mx != -INFINITY);
+      const float alpha = move ? fast_exp2(m_run - mx) : 1.f;
+      if (move) m_run = mx;
+      const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+      // P = 2^(s*sl - mu), packed to 16 bits over the first 64 columns of S.
+      // Two row sums: of the exact fp32 values (for the LSE) and of the
+      // 16-bit values the P.V product actually uses (for O = sum(P V) / l),
+      // so that the rounding of a dominant probability cancels in O.
+      float rs[2] = {0.f, 0.f}, rq[2] = {0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = fast_exp2(fmaf(f32(s[c * 32 + 2 * i]), sl, -mu));
+          const float p1 = fast_exp2(fmaf(f32(s[c * 32 + 2 * i + 1]), sl, -mu));
+          rs[i & 1] += p0 + p1;
+          pk[i] = Elem<T>::pack(p0, p1);
+          const float2 pr = Elem<T>::unpack(pk[i]);
+          rq[i & 1] += pr.x + pr.y;
+        }
+        tmem_st16(tS + c * 16, pk);
+      }
+      l_run = l_run * alpha + (rs[0] + rs[1]);
+      l_q = l_q * alpha + (rq[0] + rq[1]);
+      if (__any_sync(0xffffffffu, move && j > 0 && alpha != 1.f)) {
+        // O(j-1) is complete: S(j) was committed after PV(j-1); PV(j) waits
+        // for this tile's arrive below.
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t u[32];
+          tmem_ld32(tO + c * 32, u);
+          tmem_wait_ld();
+          reg_fence(u);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(f32(u[i]) * alpha);
+          tmem_st32(tO + c * 32, u);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_P + t));
+    }
+    if (ok && n_tiles > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_O + t), 0, abort_flag, kTcWaitNs));
+    if (!ok) {
+      fail();
+    } else {
+      // ---- epilogue: O / l in 16 bits, LSE
+      tc_fence_after();
+      const float inv = l_q > 0.f ? 1.f / l_q : 0.f;
+      T* orow = reinterpret_cast<T*>(p.o) + (((size_t)b * p.Sq + qi) * p.Hq + h) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t u[32];
+        if (n_tiles > 0) {
+          tmem_ld32(tO + c * 32, u);
+          tmem_wait_ld();
+          reg_fence(u);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) u[i] = 0u;
+        }
+        if (qi < p.Sq) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint4 w;
+            w.x = Elem<T>::pack(f32(u[v4 * 8 + 0]) * inv, f32(u[v4 * 8 + 1]) * inv);
+            w.y = Elem<T>::pack(f32(u[v4 * 8 + 2]) * inv, f32(u[v4 * 8 + 3]) * inv);
+            w.z = Elem<T>::pack(f32(u[v4 * 8 + 4]) * inv, f32(u[v4 * 8 + 5]) * inv);
+            w.w = Elem<T>::pack(f32(u[v4 * 8 + 6]) * inv, f32(u[v4 * 8 + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + c * 32 + v4 * 8) = w;
+          }
+        }
+      }
+      if (qi < p.Sq)
+        p.lse[((size_t)b * p.Hq + h) * p.Sq + qi] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+template <typename T, int D, bool kCap>
+cudaError_t launch_t(const FwdParams& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                     cudaStream_t s) {
+  auto kern = fwd_tc_kernel<T, D, kCap>;
+  constexpr int smem = TcCfg<D>::SMEM;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((p.Sq + 255) / 256, p.Hq, p.B);
+  trace_begin(s);
+  kern<<<grid, kThreadsTC, smem, s>>>(mq, mk, mv, p);
+  trace_end(s);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_dt(const FwdParams& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                      cudaStream_t s) {
+  const bool cap = p.softcap > 0.f;
+  if (p.D == 64) return cap ? launch_t<T, 64, true>(p, mq, mk, mv, s) : launch_t<T, 64, false>(p, mq, mk, mv, s);
+  return cap ? launch_t<T, 128, true>(p, mq, mk, mv, s) : launch_t<T, 128, false>(p, mq, mk, mv, s);
+}
+
+}  // namespace
+
+bool fwd_tc_supported(const FwdParams& p) {
+  return (p.D == 64 || p.D == 128) && p.Sk >= 1 && p.Sq >= 1 && tma_available();
+}
+
+cudaError_t launch_fwd_tc(const FwdParams& p, fa_dtype dt, cudaStream_t s, int* launches) {
+  CUtensorMap mq, mk, mv;
+  const bool bf = dt == FA_BF16;
+  if (!make_bshd_map(&mq, p.q, bf, p.D, p.Hq, p.Sq, p.B, 128) || !make_bshd_map(&mk, p.k, bf, p.D, p.Hkv, p.Sk, p.B, 128) ||
+      !make_bshd_map(&mv, p.v, bf, p.D, p.Hkv, p.Sk, p.B, 128))
+    return cudaErrorNotSupported;
+  cudaError_t e = bf ? launch_dt<__nv_bfloat16>(p, mq, mk, mv, s) : launch_dt<__half>(p, mq, mk, mv, s);
+  if (e == cudaSuccess) ++*launches;
+  return e;
+}
 
 }  // namespace fa

@@ -46,6 +46,7 @@ struct BwdParams {
   float scale_log2;
   float softcap, cap_in, cap_log2;
   int deterministic;
+  int kernel_choice;     // 0 automatic, 1 mma.sync main kernel, 2 tcgen05 main kernel
   int* status;
 };
 
@@ -82,6 +83,8 @@ cudaError_t launch_fwd_mma(const FwdParams& p, fa_dtype dt, cudaStream_t s, int*
 bool fwd_tc_supported(const FwdParams& p);
 cudaError_t launch_fwd_tc(const FwdParams& p, fa_dtype dt, cudaStream_t s, int* launches);
 cudaError_t launch_bwd(const BwdParams& p, fa_dtype dt, cudaStream_t s, int* launches);
+bool bwd_tc_supported(const BwdParams& p);
+cudaError_t launch_bwd_main_tc(const BwdParams& p, fa_dtype dt, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams& p, fa_dtype dt, cudaStream_t s, int* launches);
 
 }  // namespace fa

@@ -1,0 +1,19 @@
+// Host helpers for TMA tensor maps over (batch, seqlen, heads, headdim)
+// tensors: the driver's cuTensorMapEncodeTiled is reached through the runtime's
+// driver entry point, so the library needs no link against libcuda.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace fa {
+
+// True when the driver exposes the tensor-map encoder.
+bool tma_available();
+
+// 4-D map (D, H, S, B) of 16-bit elements with a box of 64 head-dim elements x
+// 1 head x `box_rows` rows x 1 batch, 128-byte swizzle, zero fill outside the
+// tensor.  Returns false if the encoder is missing or rejects the map.
+bool make_bshd_map(CUtensorMap* m, const void* base, bool bf16, int D, int H, int S, int B, int box_rows);
+
+}  // namespace fa

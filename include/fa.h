@@ -203,6 +203,14 @@ fa_status fa_last_device_status(fa_stream_t stream);
 void fa_set_fwd_kernel(int which);
 
 /*
+ * Which main backward kernel fa_bwd runs: 0 = automatic, 1 = the warp-level
+ * mma.sync kernel, 2 = the tensor-memory tcgen05 kernel (head dim 128, atomic
+ * dQ mode; fa_bwd returns FA_ERR_CUDA where it does not apply).  Process wide;
+ * meant for tests and benchmarks.
+ */
+void fa_set_bwd_kernel(int which);
+
+/*
  * Diagnostic for the failure-detection path: one kernel spins (bounded, with
  * the same helper the ordered backward uses) until the int32 at device
  * address `flag` equals `expected` or `limit_ns` nanoseconds pass; on timeout

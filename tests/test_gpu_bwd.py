@@ -9,7 +9,7 @@ import torch
 
 import oracle
 from _parity import check_grad, check_lse, check_out, f64
-from exact_attention_121_b200 import api, inputs
+from exact_attention_121_b200 import _lib, api, inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -37,14 +37,19 @@ def _fwd_bwd(q, k, v, do, det, **kw):
     return out, lse, dq, dk, dv
 
 
+@pytest.mark.parametrize("which", [0, 1], ids=["auto", "mma"])
 @pytest.mark.parametrize("det", [False, True], ids=["atomic", "ordered"])
 @pytest.mark.parametrize("case", SMALL, ids=lambda c: "B%dSq%dSk%dH%d-%dD%d%s%s" % (
     c[0], c[1], c[2], c[3], c[4], c[5], c[6], "c" if c[7] else ""))
-def test_bwd_small_full_compare(case, det):
+def test_bwd_small_full_compare(case, det, which):
     B, Sq, Sk, Hq, Hkv, D, dt, causal, window, cap, scale, amp = case
     q, k, v, do = inputs.attention_inputs(B, Sq, Sk, Hq, Hkv, D, dt, seed=21, amp=amp)
     kw = dict(scale=scale, causal=causal, window=window, softcap=cap)
-    out, lse, dq, dk, dv = _fwd_bwd(q, k, v, do, det, **kw)
+    _lib.load().fa_set_bwd_kernel(which)
+    try:
+        out, lse, dq, dk, dv = _fwd_bwd(q, k, v, do, det, **kw)
+    finally:
+        _lib.load().fa_set_bwd_kernel(0)
     sc = scale or 1 / math.sqrt(D)
     dq_r, dk_r, dv_r, _ = oracle.attn_bwd(f64(do), f64(q), f64(k), f64(v), sc, causal, window[0], window[1], cap)
     check_grad(dq, dq_r, "dQ")

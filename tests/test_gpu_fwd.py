@@ -49,7 +49,7 @@ def _run(case, which, seed):
     return q, k, v, out, lse
 
 
-@pytest.mark.parametrize("which", [0, 1], ids=["auto", "mma"])
+@pytest.mark.parametrize("which", [0, 1, 2], ids=["auto", "mma", "tc"])
 @pytest.mark.parametrize("case", SMALL, ids=lambda c: "B%dSq%dSk%dH%d-%dD%d%s%s%s" % (
     c[0], c[1], c[2], c[3], c[4], c[5], c[6], "c" if c[7] else "", "w" if c[8] != (-1, -1) else ""))
 def test_fwd_small_full_compare(case, which):
@@ -130,7 +130,7 @@ def test_fwd_kernels_agree_bitwise_on_softmax_rows():
     checked through O for V = 1 (O must be exactly representable 1)."""
     q, k, _, _ = inputs.attention_inputs(2, 300, 300, 4, 4, 128, "bf16", seed=5, with_dout=False)
     v = torch.ones_like(k)
-    for which in (0, 1):
+    for which in (1, 2):
         api.fa_set_fwd_kernel(which)
         out, _ = api.fa_fwd(q.cuda(), k.cuda(), v.cuda(), causal=True)
         torch.cuda.synchronize()
