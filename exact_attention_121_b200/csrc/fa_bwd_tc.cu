@@ -1,5 +1,5 @@
 // Backward attention on the Blackwell tensor-memory path (tcgen05 + TMA),
-// head dim 128, float32 atomic-style dQ accumulation through bulk reductions.
+// head dim 64 or 128, float32 dQ accumulation through bulk reductions.
 //
 // The method: "FlashAttention 实战指南" (mhpq.cn), the three techniques — the
 // backward pass recomputes the attention probabilities from the saved row
@@ -45,12 +45,14 @@ constexpr int kLoadWarp = 8;
 constexpr int kMmaWarpB = 9;
 constexpr unsigned long long kWaitNs = kWaitLimitNs;
 
+template <int D_>
 struct BwdTcCfg {
-  static constexpr int D = 128;
+  static constexpr int D = D_;
+  static constexpr int NCH = D / 64;              // 64-column (128-byte) chunks per row
   static constexpr int KV_CHUNK = kKeys * 128;    // 128 rows x 64 columns, 16-bit, swizzled
-  static constexpr int KV_TILE = 2 * KV_CHUNK;
+  static constexpr int KV_TILE = NCH * KV_CHUNK;
   static constexpr int Q_CHUNK = kQ * 128;        // 64 rows x 64 columns
-  static constexpr int Q_TILE = 2 * Q_CHUNK;
+  static constexpr int Q_TILE = NCH * Q_CHUNK;
   static constexpr int DS_TILE = kKeys * kQ * 2;  // [128 keys][64 queries] 16-bit, swizzled
   static constexpr int DQ_WARP = kQ * 32 * 4;     // per drain warp: [64 queries][32 dims] fp32
   static constexpr int OFF_K = 0;
@@ -70,12 +72,12 @@ struct BwdTcCfg {
 
 __device__ __forceinline__ float f32(uint32_t u) { return __uint_as_float(u); }
 
-template <typename T, bool kCap>
+template <typename T, int D_, bool kCap>
 __global__ void __launch_bounds__(kThreadsB, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                   const BwdParams p) {
-  using C = BwdTcCfg;
+  using C = BwdTcCfg<D_>;
   constexpr int D = C::D;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -142,7 +144,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         tma_prefetch_desc(&tmV);
         tma_prefetch_desc(&tmdO);
         mbar_expect_tx(bar(C::B_KV), 2 * C::KV_TILE);
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < C::NCH; ++c) {
           tma_load_4d(sb + C::OFF_K + c * C::KV_CHUNK, &tmK, c * 64, hkv, k0, b, bar(C::B_KV));
           tma_load_4d(sb + C::OFF_V + c * C::KV_CHUNK, &tmV, c * 64, hkv, k0, b, bar(C::B_KV));
         }
@@ -173,7 +175,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         __syncwarp();
         if (lane == 0) {
           mbar_expect_tx(bar(C::B_QF + st), 2 * C::Q_TILE);
-          for (int c = 0; c < 2; ++c) {
+          for (int c = 0; c < C::NCH; ++c) {
             tma_load_4d(sb + C::OFF_Q + st * C::Q_TILE + c * C::Q_CHUNK, &tmQ, c * 64, h, q0, b, bar(C::B_QF + st));
             tma_load_4d(sb + C::OFF_DO + st * C::Q_TILE + c * C::Q_CHUNK, &tmdO, c * 64, h, q0, b,
                         bar(C::B_QF + st));
@@ -231,7 +233,9 @@ __global__ void __launch_bounds__(kThreadsB, 1)
                  (acc || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk)
-          mma_ss(tb + 64, make_sdesc_sw128(sb + C::OFF_K + kk * 16 * 128, C::KV_CHUNK, 1024),
+          // M = 128 head dims; with D = 64 the second 64-row half of K^T
+          // points back at the first (LBO 0) and those TMEM lanes are unused.
+          mma_ss(tb + 64, make_sdesc_sw128(sb + C::OFF_K + kk * 16 * 128, C::NCH > 1 ? C::KV_CHUNK : 0, 1024),
                  make_sdesc_sw128(ds + kk * 16 * 128, C::KV_CHUNK, 1024), idesc_dq, kk > 0 ? 1u : 0u);
       };
       bool ok = mbar_wait(bar(C::B_KV), 0, abort_flag, kWaitNs) && mbar_wait(bar(C::B_QF), 0, abort_flag, kWaitNs);
@@ -379,6 +383,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   } else {
     // -------------------------------------------------------------- dQ drain
     const int wq = warp - kDqWarp0;          // TMEM lane quarter = head-dim slice
+    const bool has_dims = wq * 32 < D;       // D = 64 uses two of the four warps
     const uint32_t lanes = (uint32_t)(wq * 32) << 16;
     float* tile = reinterpret_cast<float*>(smem + C::OFF_DQ + wq * C::DQ_WARP);  // [64 q][32 dims]
     const uint32_t tile_s = sb + C::OFF_DQ + wq * C::DQ_WARP;
@@ -392,6 +397,12 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         break;
       }
       tc_fence_after();
+      if (!has_dims) {
+        // no head-dim rows here (D = 64): keep the TMEM-free phases in step
+        tc_fence_before();
+        mbar_arrive(bar(C::B_TMF + x));
+        continue;
+      }
       uint32_t v[kQ];
       const uint32_t tb = tmem + lanes + x * 128 + 64;
       tmem_ld32(tb, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
@@ -429,11 +440,11 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   }
 }
 
-template <typename T, bool kCap>
+template <typename T, int D, bool kCap>
 cudaError_t launch_t(const BwdParams& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                      const CUtensorMap& mdo, cudaStream_t s) {
-  auto kern = bwd_tc_kernel<T, kCap>;
-  constexpr int smem = BwdTcCfg::SMEM;
+  auto kern = bwd_tc_kernel<T, D, kCap>;
+  constexpr int smem = BwdTcCfg<D>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int nkb = (p.Sk + kKeys - 1) / kKeys;
@@ -448,7 +459,7 @@ cudaError_t launch_t(const BwdParams& p, const CUtensorMap& mq, const CUtensorMa
 }  // namespace
 
 bool bwd_tc_supported(const BwdParams& p) {
-  return p.D == 128 && !p.deterministic && p.Sq >= 1 && p.Sk >= 1 && tma_available();
+  return (p.D == 64 || p.D == 128) && !p.deterministic && p.Sq >= 1 && p.Sk >= 1 && tma_available();
 }
 
 cudaError_t launch_bwd_main_tc(const BwdParams& p, fa_dtype dt, cudaStream_t s) {
@@ -460,8 +471,14 @@ cudaError_t launch_bwd_main_tc(const BwdParams& p, fa_dtype dt, cudaStream_t s) 
       !make_bshd_map(&mv, p.v, bf, p.D, p.Hkv, p.Sk, p.B, kKeys))
     return cudaErrorNotSupported;
   const bool cap = p.softcap > 0.f;
-  if (bf) return cap ? launch_t<__nv_bfloat16, true>(p, mq, mk, mv, mdo, s) : launch_t<__nv_bfloat16, false>(p, mq, mk, mv, mdo, s);
-  return cap ? launch_t<__half, true>(p, mq, mk, mv, mdo, s) : launch_t<__half, false>(p, mq, mk, mv, mdo, s);
+  if (p.D == 64) {
+    if (bf) return cap ? launch_t<__nv_bfloat16, 64, true>(p, mq, mk, mv, mdo, s)
+                       : launch_t<__nv_bfloat16, 64, false>(p, mq, mk, mv, mdo, s);
+    return cap ? launch_t<__half, 64, true>(p, mq, mk, mv, mdo, s) : launch_t<__half, 64, false>(p, mq, mk, mv, mdo, s);
+  }
+  if (bf) return cap ? launch_t<__nv_bfloat16, 128, true>(p, mq, mk, mv, mdo, s)
+                     : launch_t<__nv_bfloat16, 128, false>(p, mq, mk, mv, mdo, s);
+  return cap ? launch_t<__half, 128, true>(p, mq, mk, mv, mdo, s) : launch_t<__half, 128, false>(p, mq, mk, mv, mdo, s);
 }
 
 }  // namespace fa
