@@ -251,8 +251,9 @@ fa_status fa_fwd_kvcache(const void* q, void* k_cache, void* v_cache, const void
   fold_window(causal, window_left, window_right, &p.wl, &p.wr);
   scale = resolve_scale(scale, D);
   fill_cap(scale, softcap, &p.softcap, &p.cap_in, &p.cap_log2, &p.scale_log2);
-  // Split count: explicit, else enough (b, kv-head, split) work items for two
-  // waves over the SMs, never more splits than pages of the longest sequence.
+  // Split count: explicit, else enough (b, kv-head, split) work items for about
+  // seven waves of two CTAs per SM, never more splits than pages of the
+  // longest sequence.
   const int cap_tokens = paged ? max_pages_per_seq * page_size : num_pages_or_max_seqlen;
   const int max_units = (cap_tokens + page_size - 1) / page_size;
   if (num_splits <= 0) {
@@ -260,7 +261,7 @@ fa_status fa_fwd_kvcache(const void* q, void* k_cache, void* v_cache, const void
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int nrt = (Sq * p.G + 15) / 16;
     const long long units = (long long)B * Hkv * nrt;
-    long long n = (2LL * sms + units - 1) / units;
+    long long n = (14LL * sms + units - 1) / units;  // ~7 waves of 2 CTAs per SM
     if (n > FA_MAX_SPLITS) n = FA_MAX_SPLITS;
     if (n > max_units) n = max_units;
     num_splits = n < 1 ? 1 : (int)n;

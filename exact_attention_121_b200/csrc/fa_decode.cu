@@ -421,10 +421,15 @@ cudaError_t launch_decode_t(const DecodeParams& p, cudaStream_t s, int* launches
     ++*launches;
   }
   const bool cap = p.softcap > 0.f;
-  if (p.D == 64)
-    e = cap ? launch_split<T, 64, true>(p, s) : launch_split<T, 64, false>(p, s);
-  else
-    e = cap ? launch_split<T, 128, true>(p, s) : launch_split<T, 128, false>(p, s);
+  e = cudaErrorNotSupported;
+  if (decode_tma_supported(p)) e = launch_decode_split_tma(p, Elem<T>::kBf16 ? FA_BF16 : FA_FP16, s);
+  if (e == cudaErrorNotSupported) {
+    // pages that are not a multiple of the TMA tile: the cp.async gather kernel
+    if (p.D == 64)
+      e = cap ? launch_split<T, 64, true>(p, s) : launch_split<T, 64, false>(p, s);
+    else
+      e = cap ? launch_split<T, 128, true>(p, s) : launch_split<T, 128, false>(p, s);
+  }
   if (e != cudaSuccess) return e;
   ++*launches;
   if (p.num_splits > 1) {

@@ -86,5 +86,7 @@ cudaError_t launch_bwd(const BwdParams& p, fa_dtype dt, cudaStream_t s, int* lau
 bool bwd_tc_supported(const BwdParams& p);
 cudaError_t launch_bwd_main_tc(const BwdParams& p, fa_dtype dt, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams& p, fa_dtype dt, cudaStream_t s, int* launches);
+bool decode_tma_supported(const DecodeParams& p);
+cudaError_t launch_decode_split_tma(const DecodeParams& p, fa_dtype dt, cudaStream_t s);
 
 }  // namespace fa
