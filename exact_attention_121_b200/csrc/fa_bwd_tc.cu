@@ -11,19 +11,23 @@
 //   S^T  = K Q_i^T        (M=128 keys, N=64 queries, K=D)      -> TMEM
 //   dP^T = V dO_i^T                                            -> TMEM
 //   P^T  = exp(S^T - LSE), dS^T = P^T (dP^T - Delta) [* (1 - tanh^2)]
-//          (warps 0-3, thread = key = TMEM lane; P^T and dS^T go back to
+//          (warps 0-7, thread = key = TMEM lane; P^T and dS^T go back to
 //           TMEM in 16 bits, dS^T also to shared memory)
 //   dV  += P^T dO_i       (A = P^T from TMEM)                  -> TMEM
 //   dK  += dS^T Q_i       (A = dS^T from TMEM)                 -> TMEM
 //   dQ^T = K^T dS^T       (M=128 head dims, N=64 queries)      -> TMEM
-//   dQ  += dQ^T^T         (warps 4-7, thread = head-dim index: TMEM ->
+//   dQ  += dQ^T^T         (warps 8-11, thread = head-dim index: TMEM ->
 //                          shared memory -> bulk fp32 add into the dQ
 //                          accumulator in global memory)
 // S^T/dP^T live in two TMEM buffers, so the elementwise work of iteration i
 // overlaps the products of iteration i+1.  TMEM (512 columns): buffer x at
-// [128x, 128x+128) holds S^T | dP^T, then P^T | dS^T | dQ^T; dV [256,384),
-// dK [384,512).  Warp 8 loads (TMA for K, V, Q_i, dO_i; plain loads for
-// LSE/Delta), warp 9 issues the MMAs.  Every wait is bounded.
+// [128x, 128x+128) holds S^T [0,64) | dP^T [64,128); the warps that handle
+// query half h write P^T (16-bit pairs) to [32h, 32h+16) and dS^T to
+// [64+32h, 64+32h+16), and dQ^T goes over [64,128) once dK has read dS^T;
+// dV [256,384), dK [384,512).  Warps 0-7 do the elementwise step (two warps
+// per TMEM lane quarter, one per query half), warps 8-11 drain dQ, warp 12
+// loads (TMA for K, V, Q_i, dO_i; plain loads for LSE/Delta), warp 13 issues
+// the MMAs.  Every wait is bounded.
 #include <math.h>
 
 #include "fa_common.cuh"
@@ -39,10 +43,10 @@ using namespace sm100;
 
 constexpr int kKeys = 128;
 constexpr int kQ = 64;
-constexpr int kThreadsB = 320;
-constexpr int kDqWarp0 = 4;
-constexpr int kLoadWarp = 8;
-constexpr int kMmaWarpB = 9;
+constexpr int kThreadsB = 448;
+constexpr int kDqWarp0 = 8;   // warps 0-7: P^T/dS^T (two per TMEM lane quarter), 8-11: dQ drain
+constexpr int kLoadWarp = 12;
+constexpr int kMmaWarpB = 13;
 constexpr unsigned long long kWaitNs = kWaitLimitNs;
 
 template <int D_>
@@ -54,17 +58,18 @@ struct BwdTcCfg {
   static constexpr int Q_CHUNK = kQ * 128;        // 64 rows x 64 columns
   static constexpr int Q_TILE = NCH * Q_CHUNK;
   static constexpr int DS_TILE = kKeys * kQ * 2;  // [128 keys][64 queries] 16-bit, swizzled
-  static constexpr int DQ_WARP = kQ * 32 * 4;     // per drain warp: [64 queries][32 dims] fp32
+  static constexpr int DQ_TILE = kQ * D * 4;      // [64 queries][D] fp32, dense (TMA reduce box)
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + KV_TILE;
-  static constexpr int OFF_Q = OFF_V + KV_TILE;       // 2 stages
-  static constexpr int OFF_DO = OFF_Q + 2 * Q_TILE;   // 2 stages
-  static constexpr int OFF_DS = OFF_DO + 2 * Q_TILE;  // 2 buffers
-  static constexpr int OFF_DQ = OFF_DS + 2 * DS_TILE;  // 4 warps
-  static constexpr int OFF_ROW = OFF_DQ + 4 * DQ_WARP;  // [stage][LSE*log2e 64 | Delta 64]
-  static constexpr int OFF_BAR = OFF_ROW + 2 * 2 * kQ * 4;
-  enum { B_KV = 0, B_QF = 1, B_QE = 3, B_SDP = 5, B_PDS = 7, B_DQF = 9, B_TMF = 11, B_FIN = 13, B_DRAIN = 14,
-         NBAR = 15 };
+  static constexpr int NQS = 3;                        // Q/dO/LSE/Delta stages
+  static constexpr int OFF_Q = OFF_V + KV_TILE;        // NQS stages
+  static constexpr int OFF_DO = OFF_Q + NQS * Q_TILE;  // NQS stages
+  static constexpr int OFF_DS = OFF_DO + NQS * Q_TILE;  // 2 buffers
+  static constexpr int OFF_DQ = OFF_DS + 2 * DS_TILE;   // 1 buffer
+  static constexpr int OFF_ROW = OFF_DQ + DQ_TILE;      // [stage][LSE*log2e 64 | Delta 64]
+  static constexpr int OFF_BAR = OFF_ROW + NQS * 2 * kQ * 4;
+  enum { B_KV = 0, B_QF = 1, B_QE = 4, B_SDP = 7, B_PDS = 9, B_DQF = 11, B_TMF = 13, B_FIN = 15, B_DRAIN = 16,
+         B_DQT_FULL = 17, B_DQT_FREE = 18, NBAR = 19 };
   static constexpr int OFF_TMEM = OFF_BAR + 8 * NBAR;
   static constexpr int OFF_ABORT = OFF_TMEM + 4;
   static constexpr int SMEM = OFF_ABORT + 4 + 1024;
@@ -76,7 +81,7 @@ template <typename T, int D_, bool kCap>
 __global__ void __launch_bounds__(kThreadsB, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
   using C = BwdTcCfg<D_>;
   constexpr int D = C::D;
   extern __shared__ uint8_t smem_raw[];
@@ -109,11 +114,15 @@ __global__ void __launch_bounds__(kThreadsB, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::B_KV), 1);
-    for (int x = 0; x < 2; ++x) {
+    for (int x = 0; x < C::NQS; ++x) {
       mbar_init(bar(C::B_QF + x), 1);
       mbar_init(bar(C::B_QE + x), 1);
+    }
+    mbar_init(bar(C::B_DQT_FULL), 128);
+    mbar_init(bar(C::B_DQT_FREE), 1);
+    for (int x = 0; x < 2; ++x) {
       mbar_init(bar(C::B_SDP + x), 1);
-      mbar_init(bar(C::B_PDS + x), 128);
+      mbar_init(bar(C::B_PDS + x), 256);
       mbar_init(bar(C::B_DQF + x), 1);
       mbar_init(bar(C::B_TMF + x), 128);
     }
@@ -151,8 +160,9 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       }
       int issued = 0;
       for (int it = 0; it < n_iter; ++it) {
-        const int st = it & 1, u = it >> 1;
-        if (it >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar(C::B_QE + st), (u - 1) & 1, abort_flag, kWaitNs))) {
+        const int st = it % C::NQS, u = it / C::NQS;
+        if (it >= C::NQS &&
+            !__all_sync(0xffffffffu, mbar_wait(bar(C::B_QE + st), (u - 1) & 1, abort_flag, kWaitNs))) {
           if (lane == 0) fail();
           break;
         }
@@ -186,8 +196,8 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       if (*abort_flag && lane == 0) {
         volatile int never = 0;
         mbar_wait(bar(C::B_KV), 0, &never, kWaitNs);
-        for (int it = max(0, issued - 2); it < issued; ++it)
-          mbar_wait(bar(C::B_QF + (it & 1)), (it >> 1) & 1, &never, kWaitNs);
+        for (int it = max(0, issued - C::NQS); it < issued; ++it)
+          mbar_wait(bar(C::B_QF + it % C::NQS), (it / C::NQS) & 1, &never, kWaitNs);
       }
     }
   } else if (warp == kMmaWarpB) {
@@ -199,9 +209,9 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       constexpr uint32_t idesc_dq = make_idesc(kBf, 128, kQ, true, true);
       const uint32_t tdV = tmem + 256, tdK = tmem + 384;
       auto issue_sdp = [&](int it) {
-        const int x = it & 1;
+        const int x = it & 1, st = it % C::NQS;
         const uint32_t tb = tmem + x * 128;
-        const uint32_t q_st = sb + C::OFF_Q + x * C::Q_TILE, do_st = sb + C::OFF_DO + x * C::Q_TILE;
+        const uint32_t q_st = sb + C::OFF_Q + st * C::Q_TILE, do_st = sb + C::OFF_DO + st * C::Q_TILE;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t okv = (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32;
@@ -218,18 +228,21 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         }
       };
       auto issue_grads = [&](int it) {
-        const int x = it & 1;
+        const int x = it & 1, st = it % C::NQS;
         const uint32_t tb = tmem + x * 128;
-        const uint32_t q_st = sb + C::OFF_Q + x * C::Q_TILE, do_st = sb + C::OFF_DO + x * C::Q_TILE;
+        const uint32_t q_st = sb + C::OFF_Q + st * C::Q_TILE, do_st = sb + C::OFF_DO + st * C::Q_TILE;
         const uint32_t ds = sb + C::OFF_DS + x * C::DS_TILE;
         const bool acc = it > 0;
 #pragma unroll
         for (int kk = 0; kk < kQ / 16; ++kk)
-          mma_ts(tdV, tb + kk * 8, make_sdesc_sw128(do_st + kk * 16 * 128, C::Q_CHUNK, 1024), idesc_kv,
+          // 16-query k-step kk of P^T sits at column 32*(kk/2) + 8*(kk%2)
+          mma_ts(tdV, tb + (kk >> 1) * 32 + (kk & 1) * 8, make_sdesc_sw128(do_st + kk * 16 * 128, C::Q_CHUNK, 1024),
+                 idesc_kv,
                  (acc || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < kQ / 16; ++kk)
-          mma_ts(tdK, tb + 32 + kk * 8, make_sdesc_sw128(q_st + kk * 16 * 128, C::Q_CHUNK, 1024), idesc_kv,
+          mma_ts(tdK, tb + 64 + (kk >> 1) * 32 + (kk & 1) * 8,
+                 make_sdesc_sw128(q_st + kk * 16 * 128, C::Q_CHUNK, 1024), idesc_kv,
                  (acc || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk)
@@ -248,7 +261,8 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         const int x = it & 1, u = it >> 1;
         if (it + 1 < n_iter) {
           const int x1 = (it + 1) & 1, u1 = (it + 1) >> 1;
-          ok = mbar_wait(bar(C::B_QF + x1), u1 & 1, abort_flag, kWaitNs) &&
+          const int s1 = (it + 1) % C::NQS, v1 = (it + 1) / C::NQS;
+          ok = mbar_wait(bar(C::B_QF + s1), v1 & 1, abort_flag, kWaitNs) &&
                (it + 1 < 2 || mbar_wait(bar(C::B_TMF + x1), (u1 - 1) & 1, abort_flag, kWaitNs));
           if (!ok) break;
           tc_fence_after();
@@ -260,7 +274,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         tc_fence_after();
         issue_grads(it);
         mma_commit(bar(C::B_DQF + x));
-        mma_commit(bar(C::B_QE + x));
+        mma_commit(bar(C::B_QE + it % C::NQS));
       }
       if (ok) mma_commit(bar(C::B_FIN));
       if (!ok) fail();
@@ -270,10 +284,12 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     }
   } else if (warp < kDqWarp0) {
     // -------------------------------------------------------------- P^T, dS^T
-    const int r = warp * 32 + lane;
+    // warp = (hh, wq): TMEM lane quarter wq (32 keys) and query half hh.
+    const int wq = warp & 3, hh = warp >> 2;
+    const int r = wq * 32 + lane;
     const int key = k0 + r;
     const bool key_ok = key <= k1;
-    const uint32_t lanes = (uint32_t)(warp * 32) << 16;
+    const uint32_t lanes = (uint32_t)(wq * 32) << 16;
     bool ok = true;
     for (int it = 0; it < n_iter; ++it) {
       const int x = it & 1, u = it >> 1;
@@ -288,20 +304,21 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       }
       tc_fence_after();
       const uint32_t tb = tmem + lanes + x * 128;
-      uint32_t s[kQ], dp[kQ];
-      tmem_ld32(tb + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-      tmem_ld32(tb + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-      tmem_ld32(tb + 64, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-      tmem_ld32(tb + 96, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+      const float* rw = rows + (it % C::NQS) * 2 * kQ + 32 * hh;
+      const bool full = (k1 - k0 + 1 == kKeys) && (q0 + kQ <= p.Sq) &&
+                        (p.wl < 0 || k0 >= q0 + kQ - 1 + off - p.wl) && (p.wr < 0 || k1 <= q0 + off + p.wr);
+      // This warp's 32 queries: S^T columns [32hh, 32hh+32), dP^T columns
+      // [64+32hh, ...).  P^T (16-bit pairs) goes to [32hh, 32hh+16) and dS^T
+      // to [64+32hh, ...): inside the columns only this warp reads.
+      uint32_t s[32], dp[32];
+      tmem_ld32(tb + 32 * hh, s);
+      tmem_ld32(tb + 64 + 32 * hh, dp);
       tmem_wait_ld();
       reg_fence(s);
       reg_fence(dp);
-      const float* rw = rows + x * 2 * kQ;
-      const bool full = (k1 - k0 + 1 == kKeys) && (q0 + kQ <= p.Sq) &&
-                        (p.wl < 0 || k0 >= q0 + kQ - 1 + off - p.wl) && (p.wr < 0 || k1 <= q0 + off + p.wr);
-      uint32_t pk[kQ / 2], dk[kQ / 2];
+      uint32_t pk[16], dk[16];
 #pragma unroll
-      for (int c = 0; c < kQ; c += 2) {
+      for (int c = 0; c < 32; c += 2) {
         float pv[2], dv[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
@@ -317,7 +334,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
           }
           float pe = fast_exp2(xv - l2);
           if (!full) {
-            const int qp = q0 + c + e + off;
+            const int qp = q0 + 32 * hh + c + e + off;
             const bool vis = key_ok && (p.wl < 0 || key >= qp - p.wl) && (p.wr < 0 || key <= qp + p.wr);
             pe = vis ? pe : 0.f;
           }
@@ -327,16 +344,17 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         pk[c / 2] = Elem<T>::pack(pv[0], pv[1]);
         dk[c / 2] = Elem<T>::pack(dv[0], dv[1]);
       }
-      tmem_st16(tb + 0, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-      tmem_st16(tb + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
-      tmem_st16(tb + 32, *reinterpret_cast<uint32_t(*)[16]>(&dk[0]));
-      tmem_st16(tb + 48, *reinterpret_cast<uint32_t(*)[16]>(&dk[16]));
-      // dS^T row r -> shared memory, 128-byte swizzle (MN-major operand of dQ^T)
+      tmem_st16(tb + 32 * hh, pk);
+      tmem_st16(tb + 64 + 32 * hh, dk);
+      // dS^T row r, queries of this half -> shared memory, 128-byte swizzle
+      // (MN-major operand of dQ^T)
       uint8_t* dsrow = smem + C::OFF_DS + x * C::DS_TILE + r * 128;
 #pragma unroll
-      for (int g = 0; g < 8; ++g)
-        *reinterpret_cast<uint4*>(dsrow + ((g ^ (r & 7)) << 4)) =
+      for (int g = 0; g < 4; ++g) {
+        const int gg = 4 * hh + g;
+        *reinterpret_cast<uint4*>(dsrow + ((gg ^ (r & 7)) << 4)) =
             make_uint4(dk[4 * g], dk[4 * g + 1], dk[4 * g + 2], dk[4 * g + 3]);
+      }
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
@@ -346,17 +364,18 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     if (!ok) {
       fail();
     } else {
+      // ---- dV and dK rows of this warp's keys, head-dim half hh
       tc_fence_after();
       const size_t ks = (size_t)p.Hkv * D;
-      T* dVr = reinterpret_cast<T*>(p.dv) + ((size_t)b * p.Sk + key) * ks + (size_t)hkv * D;
-      T* dKr = reinterpret_cast<T*>(p.dk) + ((size_t)b * p.Sk + key) * ks + (size_t)hkv * D;
+      T* dVr = reinterpret_cast<T*>(p.dv) + ((size_t)b * p.Sk + key) * ks + (size_t)hkv * D + hh * (D / 2);
+      T* dKr = reinterpret_cast<T*>(p.dk) + ((size_t)b * p.Sk + key) * ks + (size_t)hkv * D + hh * (D / 2);
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const float mul = which ? p.scale : 1.f;
         T* dst = which ? dKr : dVr;
-        const uint32_t src = tmem + lanes + (which ? 384 : 256);
+        const uint32_t src = tmem + lanes + (which ? 384 : 256) + hh * (D / 2);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           uint32_t v[32];
           if (n_iter > 0) {
             tmem_ld32(src + c * 32, v);
@@ -385,50 +404,58 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     const int wq = warp - kDqWarp0;          // TMEM lane quarter = head-dim slice
     const bool has_dims = wq * 32 < D;       // D = 64 uses two of the four warps
     const uint32_t lanes = (uint32_t)(wq * 32) << 16;
-    float* tile = reinterpret_cast<float*>(smem + C::OFF_DQ + wq * C::DQ_WARP);  // [64 q][32 dims]
-    const uint32_t tile_s = sb + C::OFF_DQ + wq * C::DQ_WARP;
+    // The dQ tile of an iteration is [64 queries][D] fp32 in shared memory
+    // (one buffer); every drain thread writes its head-dim column, then
+    // one thread adds the whole tile into the global accumulator with a single
+    // tiled TMA reduction.  Rows past Sq fall outside the tensor and are
+    // skipped by the TMA unit.
+    const bool issuer = (warp == kDqWarp0) && lane == 0;
     bool ok = true;
     for (int it = 0; it < n_iter; ++it) {
       const int x = it & 1, u = it >> 1;
       int h, q0;
       iter_q(it, h, q0);
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(C::B_DQF + x), u & 1, abort_flag, kWaitNs))) {
+      bool w = mbar_wait(bar(C::B_DQF + x), u & 1, abort_flag, kWaitNs);
+      // the tile is free once the reduction of iteration it-1 has read it
+      if (it >= 1) w = w && mbar_wait(bar(C::B_DQT_FREE), (it - 1) & 1, abort_flag, kWaitNs);
+      if (!__all_sync(0xffffffffu, w)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      if (!has_dims) {
-        // no head-dim rows here (D = 64): keep the TMEM-free phases in step
+      float* tile = reinterpret_cast<float*>(smem + C::OFF_DQ);
+      if (has_dims) {
+        uint32_t v[kQ];
+        const uint32_t tb = tmem + lanes + x * 128 + 64;
+        tmem_ld32(tb, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(tb + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tmem_wait_ld();
+        reg_fence(v);
         tc_fence_before();
         mbar_arrive(bar(C::B_TMF + x));
-        continue;
-      }
-      uint32_t v[kQ];
-      const uint32_t tb = tmem + lanes + x * 128 + 64;
-      tmem_ld32(tb, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tmem_ld32(tb + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-      tmem_wait_ld();
-      reg_fence(v);
-      tc_fence_before();
-      mbar_arrive(bar(C::B_TMF + x));
-      // the previous iteration's reductions have read the tile (lane-local
-      // wait, then the warp agrees before anyone overwrites it)
-      bulk_wait_read_all();
-      __syncwarp();
 #pragma unroll
-      for (int c = 0; c < kQ; ++c) tile[c * 32 + lane] = f32(v[c]);
-      fence_proxy_async_smem();
-      __syncwarp();
-      float* gbase = p.dq_accum + ((size_t)b * p.Sq) * p.Hq * D + (size_t)h * D + wq * 32;
-#pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const int row = lane + 32 * rr;
-        const int q = q0 + row;
-        if (q < p.Sq) bulk_reduce_add_f32(gbase + (size_t)q * p.Hq * D, tile_s + row * 128, 128);
+        for (int c = 0; c < kQ; ++c) tile[c * D + wq * 32 + lane] = f32(v[c]);
+        fence_proxy_async_smem();
+      } else {
+        // no head-dim rows here (D = 64): keep the barrier phases in step
+        tc_fence_before();
+        mbar_arrive(bar(C::B_TMF + x));
       }
-      bulk_commit();
+      mbar_arrive(bar(C::B_DQT_FULL));
+      if (issuer) {
+        if (!mbar_wait(bar(C::B_DQT_FULL), it & 1, abort_flag, kWaitNs)) {
+          ok = false;
+        } else {
+          tma_reduce_add_4d(&tmDQ, 0, h, q0, b, sb + C::OFF_DQ);
+          bulk_commit();
+          // the tile may be rewritten once the reduction has read it
+          bulk_wait_read_all();
+          mbar_arrive(bar(C::B_DQT_FREE));
+        }
+      }
+      if (!__all_sync(0xffffffffu, ok)) break;
     }
-    bulk_wait_all();
+    if (issuer) bulk_wait_all();
     if (!ok) fail();
   }
 
@@ -442,7 +469,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
 
 template <typename T, int D, bool kCap>
 cudaError_t launch_t(const BwdParams& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                     const CUtensorMap& mdo, cudaStream_t s) {
+                     const CUtensorMap& mdo, const CUtensorMap& mdq, cudaStream_t s) {
   auto kern = bwd_tc_kernel<T, D, kCap>;
   constexpr int smem = BwdTcCfg<D>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -451,7 +478,7 @@ cudaError_t launch_t(const BwdParams& p, const CUtensorMap& mq, const CUtensorMa
   const long long items = (long long)nkb * p.Hkv * p.B;
   if (items == 0) return cudaSuccess;
   trace_begin(s);
-  kern<<<(unsigned)items, kThreadsB, smem, s>>>(mq, mk, mv, mdo, p);
+  kern<<<(unsigned)items, kThreadsB, smem, s>>>(mq, mk, mv, mdo, mdq, p);
   trace_end(s);
   return cudaGetLastError();
 }
@@ -463,22 +490,23 @@ bool bwd_tc_supported(const BwdParams& p) {
 }
 
 cudaError_t launch_bwd_main_tc(const BwdParams& p, fa_dtype dt, cudaStream_t s) {
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdq;
   const bool bf = dt == FA_BF16;
   if (!make_bshd_map(&mq, p.q, bf, p.D, p.Hq, p.Sq, p.B, kQ) ||
       !make_bshd_map(&mdo, p.dout, bf, p.D, p.Hq, p.Sq, p.B, kQ) ||
       !make_bshd_map(&mk, p.k, bf, p.D, p.Hkv, p.Sk, p.B, kKeys) ||
-      !make_bshd_map(&mv, p.v, bf, p.D, p.Hkv, p.Sk, p.B, kKeys))
+      !make_bshd_map(&mv, p.v, bf, p.D, p.Hkv, p.Sk, p.B, kKeys) ||
+      !make_bshd_map_f32(&mdq, p.dq_accum, p.D, p.Hq, p.Sq, p.B, kQ))
     return cudaErrorNotSupported;
   const bool cap = p.softcap > 0.f;
   if (p.D == 64) {
-    if (bf) return cap ? launch_t<__nv_bfloat16, 64, true>(p, mq, mk, mv, mdo, s)
-                       : launch_t<__nv_bfloat16, 64, false>(p, mq, mk, mv, mdo, s);
-    return cap ? launch_t<__half, 64, true>(p, mq, mk, mv, mdo, s) : launch_t<__half, 64, false>(p, mq, mk, mv, mdo, s);
+    if (bf) return cap ? launch_t<__nv_bfloat16, 64, true>(p, mq, mk, mv, mdo, mdq, s)
+                       : launch_t<__nv_bfloat16, 64, false>(p, mq, mk, mv, mdo, mdq, s);
+    return cap ? launch_t<__half, 64, true>(p, mq, mk, mv, mdo, mdq, s) : launch_t<__half, 64, false>(p, mq, mk, mv, mdo, mdq, s);
   }
-  if (bf) return cap ? launch_t<__nv_bfloat16, 128, true>(p, mq, mk, mv, mdo, s)
-                     : launch_t<__nv_bfloat16, 128, false>(p, mq, mk, mv, mdo, s);
-  return cap ? launch_t<__half, 128, true>(p, mq, mk, mv, mdo, s) : launch_t<__half, 128, false>(p, mq, mk, mv, mdo, s);
+  if (bf) return cap ? launch_t<__nv_bfloat16, 128, true>(p, mq, mk, mv, mdo, mdq, s)
+                     : launch_t<__nv_bfloat16, 128, false>(p, mq, mk, mv, mdo, mdq, s);
+  return cap ? launch_t<__half, 128, true>(p, mq, mk, mv, mdo, mdq, s) : launch_t<__half, 128, false>(p, mq, mk, mv, mdo, mdq, s);
 }
 
 }  // namespace fa

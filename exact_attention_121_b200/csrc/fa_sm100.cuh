@@ -71,7 +71,22 @@ __device__ __forceinline__ void bulk_reduce_add_f32(float* dst, uint32_t src, ui
                "r"(bytes)
                : "memory");
 }
+// Tiled TMA reduction shared -> global (fp32 add), 4-D box at (c0..c3); box
+// elements outside the tensor are skipped.
+__device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                                  uint32_t src) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2, %3, %4}], [%5];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(src)
+      : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most one committed bulk group of this thread is still reading
+// its shared-memory source.
+__device__ __forceinline__ void bulk_wait_read_1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
 // Wait until every committed bulk group of this thread has finished reading
 // its shared-memory source.
 __device__ __forceinline__ void bulk_wait_read_all() {

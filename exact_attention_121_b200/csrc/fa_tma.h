@@ -16,4 +16,9 @@ bool tma_available();
 // tensor.  Returns false if the encoder is missing or rejects the map.
 bool make_bshd_map(CUtensorMap* m, const void* base, bool bf16, int D, int H, int S, int B, int box_rows);
 
+// 4-D map (D, H, S, B) of fp32 elements with a box of all D elements x 1 head
+// x `box_rows` rows x 1 batch, no swizzle (dense row-major box in shared
+// memory); used as the target of tiled reductions.
+bool make_bshd_map_f32(CUtensorMap* m, const void* base, int D, int H, int S, int B, int box_rows);
+
 }  // namespace fa
