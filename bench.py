@@ -36,6 +36,17 @@ import torch  # noqa: E402
 METRIC = "attention TFLOPs/s fwd+bwd (seqlen sweep 512-16k d64/d128, GQA+local, paged decode)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# Launch whose per-launch roofline is reported for each kernel class.
+ROOFLINE_UNIT = {"fwd": "H16D128S4096n", "bwd": "H16D128S4096n", "decode": "decode"}
+# DRAM bytes (read + write) per launch from one ncu capture of that launch
+# (profiles/*_H16D128S4096n.md, profiles/decode_tma_kernel_paged_B8.md).  An
+# entry must be removed whenever its kernel changes.
+TRAFFIC_PER_LAUNCH = {
+    ("fwd", "H16D128S4096n"): 201.680384e6 + 48.214272e6,
+    ("bwd", "H16D128S4096n"): 405.318656e6 + 222.136832e6,
+    ("decode", "decode"): 521.960192e6 + 8.847872e6,
+}
+
 
 # ---------------------------------------------------------------------------
 # algorithmic work
@@ -283,19 +294,22 @@ class Tracer:
         self.lib.fa_set_trace_events(a.cuda_event, b.cuda_event)
         work = {"fwd": getattr(unit, "flops_fwd", 0), "bwd": getattr(unit, "flops_bwd", 0),
                 "decode": getattr(unit, "bytes", 0)}[cls]
-        self.pending.append((cls, a, b, work))
+        self.pending.append((cls, unit.name(), a, b, work))
 
     def disarm(self):
         if self.enabled:
             self.lib.fa_set_trace_events(None, None)
 
     def collect(self):
-        for cls, a, b, work in self.pending:
+        """Totals per kernel class; per (class, unit) totals in self.per_unit."""
+        self.per_unit = getattr(self, "per_unit", {})
+        for cls, name, a, b, work in self.pending:
             ms = a.elapsed_time(b)
-            t = self.totals.setdefault(cls, [0.0, 0, 0])
-            t[0] += ms
-            t[1] += 1
-            t[2] += work
+            for d, key in ((self.totals, cls), (self.per_unit, (cls, name))):
+                t = d.setdefault(key, [0.0, 0, 0])
+                t[0] += ms
+                t[1] += 1
+                t[2] += work
         self.pending = []
         return self.totals
 
@@ -475,20 +489,30 @@ def main():
         ms_e2e = float(t.item())
     e2e_value = world * flops_step * args.e2e_steps / (ms_e2e / 1e3) / 1e12
 
-    # roofline of the dominant kernel class (largest traced time)
+    # Roofline of the dominant kernel class (largest traced time), per launch
+    # of the representative sweep point when it ran (so that `achieved` and
+    # the ncu `traffic` describe the same launch), else over all its launches.
     dom = max(totals.items(), key=lambda kv: kv[1][0])
-    cls, (kms, cnt, work) = dom
+    cls, (kms_all, cnt_all, work_all) = dom
+    rep = ROOFLINE_UNIT[cls]
+    kms, cnt, work = tracer.per_unit.get((cls, rep), (kms_all, cnt_all, work_all))
+    if (cls, rep) not in tracer.per_unit:
+        rep = "all launches"
+    scale = 1e9 if cls == "decode" else 1e12
+    achieved = (work / cnt) / (kms / cnt / 1e3) / scale
+    achieved_all = work_all / (kms_all / 1e3) / scale
     if cls == "decode":
-        achieved = work / (kms / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None}
+        pk = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk, "unit": "GB/s", "frac": achieved / pk}
     else:
-        achieved = work / (kms / 1e3) / 1e12
         pk = peaks["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
-                "frac": achieved / pk, "traffic": None}
-    roof["kernel"] = {"fwd": "forward attention kernel", "bwd": "main backward kernel (dK/dV/dQ)",
-                      "decode": "split-KV decode kernel"}[cls]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s", "frac": achieved / pk}
+    roof["traffic"] = TRAFFIC_PER_LAUNCH.get((cls, rep))
+    roof["launch"] = rep
+    roof["algorithmic_per_launch"] = work / cnt
+    roof["achieved_all_launches"] = achieved_all
+    roof["kernel"] = {"fwd": "fwd_tc_kernel (tcgen05 forward)", "bwd": "bwd_tc_kernel (tcgen05 backward)",
+                      "decode": "decode_tma_kernel (split-KV decode)"}[cls]
     roof["peak_source"] = f"{peak_src} ({'bf16_tflops_sustained' if cls != 'decode' else 'hbm_gbs'})"
     kernels = {c: {"ms_total": v[0], "launches": v[1],
                    ("gbs" if c == "decode" else "tflops"): v[2] / (v[0] / 1e3) / (1e9 if c == "decode" else 1e12)}
