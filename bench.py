@@ -389,6 +389,22 @@ def cpu_oracle_sample(budget_s=12.0):
                        f"{el:.1f} s", elapsed_s=el, flops=n * flops)
 
 
+def max_over_ranks(ms, pg, dev):
+    """The slowest rank's time: every rank contributes its own device-timed
+    milliseconds (one all-reduce, taken in the same order on every rank)."""
+    if pg is None:
+        return float(ms)
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=dev)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world, flops_step, steps, ms):
+    """Aggregate throughput of `world` replicas, each of which ran `steps`
+    steps of `flops_step` flops, over the slowest rank's `ms`."""
+    return world * flops_step * steps / (ms / 1e3) / 1e12
+
+
 def reference_arm(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -456,12 +472,8 @@ def main():
     ms, launches = time_steps(units, args.steps, args.warmup, tracer, barrier=barrier)
     clk = clocks.stop()
     totals = tracer.collect()
-    ms_max = ms
-    if pg:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms_max = float(t.item())
-    value = world * flops_step * args.steps / (ms_max / 1e3) / 1e12
+    ms_max = max_over_ranks(ms, pg, dev)
+    value = whole_job_tflops(world, flops_step, args.steps, ms_max)
 
     # per-unit detail (untimed for the headline; separate short pass)
     detail = {}
@@ -483,11 +495,8 @@ def main():
     h2d = sum(u.e2e_bytes()[0] for u in units)
     d2h = sum(u.e2e_bytes()[1] for u in units)
     ms_e2e, _ = time_steps(units, args.e2e_steps, 1, Tracer(lib), e2e=True, barrier=barrier)
-    if pg:
-        t = torch.tensor([ms_e2e], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms_e2e = float(t.item())
-    e2e_value = world * flops_step * args.e2e_steps / (ms_e2e / 1e3) / 1e12
+    ms_e2e = max_over_ranks(ms_e2e, pg, dev)
+    e2e_value = whole_job_tflops(world, flops_step, args.e2e_steps, ms_e2e)
 
     # Roofline of the dominant kernel class (largest traced time), per launch
     # of the representative sweep point when it ran (so that `achieved` and
