@@ -42,8 +42,6 @@ ROOFLINE_UNIT = {"fwd": "H16D128S4096n", "bwd": "H16D128S4096n", "decode": "deco
 # (profiles/*_H16D128S4096n.md, profiles/decode_tma_kernel_paged_B8.md).  An
 # entry must be removed whenever its kernel changes.
 TRAFFIC_PER_LAUNCH = {
-    ("fwd", "H16D128S4096n"): 201.680384e6 + 48.214272e6,
-    ("bwd", "H16D128S4096n"): 405.318656e6 + 222.136832e6,
     ("decode", "decode"): 521.960192e6 + 8.847872e6,
 }
 

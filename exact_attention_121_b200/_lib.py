@@ -34,6 +34,7 @@ SIGNATURES = {
     "fa_set_fwd_kernel": (None, [_I]),
     "fa_set_bwd_kernel": (None, [_I]),
     "fa_selftest_bounded_wait": (_I, [_P, _I, ctypes.c_longlong, _P]),
+    "fa_selftest_exp2_poly": (_I, [_P, _P, _I, _P]),
     "fa_last_launch_count": (_I, []),
     "fa_set_trace_events": (None, [_P, _P]),
 }

@@ -80,7 +80,29 @@ __global__ void selftest_wait_kernel(const int* flag, int expected, unsigned lon
   if (threadIdx.x == 0 && !fa::wait_eq_bounded(flag, expected, limit_ns)) fa::report_status(status, FA_ERR_TIMEOUT);
 }
 
+__global__ void selftest_exp2_kernel(const float* x, float* y, int n) {
+  const long long i = 2 * (blockIdx.x * (long long)blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    fa::exp2_poly2(x[i], x[i + 1], y[i], y[i + 1]);
+  } else if (i < n) {
+    float unused;
+    fa::exp2_poly2(x[i], 0.f, y[i], unused);
+  }
+}
+
 }  // namespace
+
+extern "C" fa_status fa_selftest_exp2_poly(const float* x, float* y, int n, fa_stream_t stream) {
+  g_last_launches = 0;
+  if (n < 0 || (n > 0 && (!x || !y))) return FA_ERR_INVALID_ARG;
+  if (n == 0) return FA_OK;
+  const int threads = 256;
+  const long long pairs = (n + 1) / 2;
+  selftest_exp2_kernel<<<(unsigned)((pairs + threads - 1) / threads), threads, 0, stream>>>(x, y, n);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  g_last_launches = 1;
+  return FA_OK;
+}
 
 namespace fa {
 void trace_begin(cudaStream_t s) {

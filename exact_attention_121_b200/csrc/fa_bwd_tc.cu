@@ -176,10 +176,10 @@ __global__ void __launch_bounds__(kThreadsB, 1)
           float l2 = INFINITY, dl = 0.f;
           if (q < p.Sq) {
             const float l = L[q];
-            l2 = (l == -INFINITY) ? INFINITY : l * kLog2e;
+            l2 = (l == -INFINITY) ? INFINITY : l * kLog2e;  // stored negated below
             dl = Dl[q];
           }
-          r[t] = l2;
+          r[t] = -l2;  // x - LSE*log2e becomes one fma: s * scale_log2 + (-LSE*log2e)
           r[kQ + t] = dl;
         }
         __syncwarp();
@@ -308,52 +308,72 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       const bool full = (k1 - k0 + 1 == kKeys) && (q0 + kQ <= p.Sq) &&
                         (p.wl < 0 || k0 >= q0 + kQ - 1 + off - p.wl) && (p.wr < 0 || k1 <= q0 + off + p.wr);
       // This warp's 32 queries: S^T columns [32hh, 32hh+32), dP^T columns
-      // [64+32hh, ...).  P^T (16-bit pairs) goes to [32hh, 32hh+16) and dS^T
-      // to [64+32hh, ...): inside the columns only this warp reads.
-      uint32_t s[32], dp[32];
-      tmem_ld32(tb + 32 * hh, s);
-      tmem_ld32(tb + 64 + 32 * hh, dp);
-      tmem_wait_ld();
-      reg_fence(s);
-      reg_fence(dp);
-      uint32_t pk[16], dk[16];
-#pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        float pv[2], dv[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float l2 = rw[c + e];
-          const float dl = rw[kQ + c + e];
-          float xv, fac = 1.f;
-          if (kCap) {
-            const float t = tanh_exp(f32(s[c + e]) * p.cap_in);
-            xv = p.cap_log2 * t;
-            fac = 1.f - t * t;
-          } else {
-            xv = f32(s[c + e]) * p.scale_log2;
-          }
-          float pe = fast_exp2(xv - l2);
-          if (!full) {
-            const int qp = q0 + 32 * hh + c + e + off;
-            const bool vis = key_ok && (p.wl < 0 || key >= qp - p.wl) && (p.wr < 0 || key <= qp + p.wr);
-            pe = vis ? pe : 0.f;
-          }
-          pv[e] = pe;
-          dv[e] = pe * (f32(dp[c + e]) - dl) * fac;
-        }
-        pk[c / 2] = Elem<T>::pack(pv[0], pv[1]);
-        dk[c / 2] = Elem<T>::pack(dv[0], dv[1]);
-      }
-      tmem_st16(tb + 32 * hh, pk);
-      tmem_st16(tb + 64 + 32 * hh, dk);
-      // dS^T row r, queries of this half -> shared memory, 128-byte swizzle
-      // (MN-major operand of dQ^T)
+      // [64+32hh, ...), taken in two sub-blocks of 16 queries (sb) to keep
+      // few registers live.  P^T (16-bit pairs) of sub-block sb goes to
+      // [32hh+8sb, +8) and dS^T to [64+32hh+8sb, +8): inside columns this
+      // warp has already read.
+      const unsigned long long sl2 = f2_pack(p.scale_log2, p.scale_log2);
       uint8_t* dsrow = smem + C::OFF_DS + x * C::DS_TILE + r * 128;
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const int gg = 4 * hh + g;
-        *reinterpret_cast<uint4*>(dsrow + ((gg ^ (r & 7)) << 4)) =
-            make_uint4(dk[4 * g], dk[4 * g + 1], dk[4 * g + 2], dk[4 * g + 3]);
+      for (int sbk = 0; sbk < 2; ++sbk) {
+        const int q16 = 32 * hh + 16 * sbk;  // first query of the sub-block
+        uint32_t s[16], dp[16];
+        tmem_ld16(tb + q16, s);
+        tmem_ld16(tb + 64 + q16, dp);
+        const float4* nl4 = reinterpret_cast<const float4*>(rw + 16 * sbk);       // -LSE*log2e
+        const float4* dl4 = reinterpret_cast<const float4*>(rw + kQ + 16 * sbk);  // Delta
+        float nl[16], dlv[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float4 a4 = nl4[j], b4 = dl4[j];
+          nl[4 * j] = a4.x; nl[4 * j + 1] = a4.y; nl[4 * j + 2] = a4.z; nl[4 * j + 3] = a4.w;
+          dlv[4 * j] = b4.x; dlv[4 * j + 1] = b4.y; dlv[4 * j + 2] = b4.z; dlv[4 * j + 3] = b4.w;
+        }
+        tmem_wait_ld();
+        reg_fence(s);
+        reg_fence(dp);
+        uint32_t pk[8], dk[8];
+#pragma unroll
+        for (int c = 0; c < 16; c += 2) {
+          float pv[2], dv[2];
+          if (kCap) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const float t = tanh_exp(f32(s[c + e]) * p.cap_in);
+              pv[e] = fast_exp2(fmaf(p.cap_log2, t, nl[c + e]));
+              dv[e] = (f32(dp[c + e]) - dlv[c + e]) * (1.f - t * t);
+            }
+          } else {
+            // packed f32x2: one instruction per query pair
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(f32(s[c]), f32(s[c + 1])), sl2, f2_pack(nl[c], nl[c + 1])), x0, x1);
+            pv[0] = fast_exp2(x0);
+            pv[1] = fast_exp2(x1);
+            f2_unpack(f2_sub(f2_pack(f32(dp[c]), f32(dp[c + 1])), f2_pack(dlv[c], dlv[c + 1])), dv[0], dv[1]);
+          }
+          if (!full) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int qp = q0 + q16 + c + e + off;
+              const bool vis = key_ok && (p.wl < 0 || key >= qp - p.wl) && (p.wr < 0 || key <= qp + p.wr);
+              pv[e] = vis ? pv[e] : 0.f;
+            }
+          }
+          // dS = P (dP - Delta) [* (1 - tanh^2)]
+          f2_unpack(f2_mul(f2_pack(pv[0], pv[1]), f2_pack(dv[0], dv[1])), dv[0], dv[1]);
+          pk[c / 2] = Elem<T>::pack(pv[0], pv[1]);
+          dk[c / 2] = Elem<T>::pack(dv[0], dv[1]);
+        }
+        tmem_st8(tb + 32 * hh + 8 * sbk, pk);
+        tmem_st8(tb + 64 + 32 * hh + 8 * sbk, dk);
+        // dS^T row r, these 16 queries -> shared memory, 128-byte swizzle
+        // (MN-major operand of dQ^T)
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          const int gg = 4 * hh + 2 * sbk + g;
+          *reinterpret_cast<uint4*>(dsrow + ((gg ^ (r & 7)) << 4)) =
+              make_uint4(dk[4 * g], dk[4 * g + 1], dk[4 * g + 2], dk[4 * g + 3]);
+        }
       }
       tmem_wait_st();
       fence_proxy_async_smem();

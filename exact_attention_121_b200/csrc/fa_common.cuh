@@ -140,6 +140,73 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// 2^x for a pair of arguments on the FMA pipe (packed f32x2 arithmetic):
+// x = n + f with n = round(x) (adding and subtracting 1.5 * 2^23 rounds to the
+// nearest integer), 2^f ~ p(f) on |f| <= 1/2 by a degree-4 polynomial fitted
+// for minimum relative error (exp2_poly_fit.py: max relative error 2.9e-6 in
+// float32), and 2^n applied by adding n to the exponent field.  Arguments are
+// clamped to >= -125 so the result stays a normal float; callers use it only
+// where no argument is -inf (a masked score must give exactly 0).
+constexpr float kExp2C1 = 0.693124175f;
+constexpr float kExp2C2 = 0.240240991f;
+constexpr float kExp2C3 = 0.0559063703f;
+constexpr float kExp2C4 = 0.00958281849f;
+
+__device__ __forceinline__ unsigned long long f2_pack(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(unsigned long long v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ unsigned long long f2_sub(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+  const float kRound = 12582912.0f;  // 1.5 * 2^23
+  const unsigned long long x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const unsigned long long rnd = f2_pack(kRound, kRound);
+  const unsigned long long t = f2_add(x, rnd);      // low mantissa bits hold round(x)
+  const unsigned long long f = f2_sub(x, f2_sub(t, rnd));
+  unsigned long long p = f2_fma(f2_pack(kExp2C4, kExp2C4), f, f2_pack(kExp2C3, kExp2C3));
+  p = f2_fma(p, f, f2_pack(kExp2C2, kExp2C2));
+  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
+  p = f2_fma(p, f, f2_pack(1.0f, 1.0f));
+  float t0, t1, p0, p1;
+  f2_unpack(t, t0, t1);
+  f2_unpack(p, p0, p1);
+  // bits(t) = 0x4B400000 + n and 0x4B400000 << 23 == 0 (mod 2^32): bits(t) << 23 == n << 23
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+// max(a, b, c) in one instruction (three-operand form, sm_100 and later).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // tanh(x) from the identity tanh(x) = 1 - 2 / (e^{2x} + 1); absolute error
 // ~1e-7, far tighter than the hardware tanh approximation.
 __device__ __forceinline__ float tanh_exp(float x) {

@@ -13,12 +13,16 @@
 //              shared-memory stages (128-byte swizzle, zero fill past the ends)
 //   warp  9    MMA issuer: tcgen05.mma with fp32 accumulators in TMEM
 // Tensor memory (512 columns): S_A [0,128), S_B [128,256), O_A [256,256+D),
-// O_B [384,384+D); P (16-bit) is written over the first 64 columns of S and is
-// the A operand of O += P V straight from TMEM.  Per key tile j the MMA warp
-// issues  PV_A(j), S_A(j+1), PV_B(j), S_B(j+1),  so one tile's softmax overlaps
-// the other tile's products.  Because a tcgen05.commit tracks every earlier MMA
-// of the issuing thread, "S(j+1) is ready" also means "PV(j) is done", which is
-// when a softmax warp may rescale its O rows in TMEM.  The running maximum is
+// O_B [384,384+D); P (16-bit) is the A operand of O += P V straight from TMEM.
+// Head dim 128: P is written over the first 64 columns of S, and per key tile
+// j the MMA warp issues  PV_A(j), S_A(j+1), PV_B(j), S_B(j+1),  so one tile's
+// softmax overlaps the other tile's products.  Because a tcgen05.commit tracks
+// every earlier MMA of the issuing thread, "S(j+1) is ready" also means "PV(j)
+// is done", which is when a softmax warp may rescale its O rows in TMEM.
+// Head dim 64: P_t has its own 64 columns after O_t, so S_t(j+1) is issued as
+// soon as the softmax warps have read S_t(j) into registers, and the next
+// tile's scores are ready when the softmax finishes; the softmax waits for
+// PV_t(j-1) only before it writes P_t(j) or rescales O_t.  The running maximum is
 // only moved (and O rescaled) when it grows by more than 2^8, which keeps
 // every exponent <= 2^8 and makes rescales rare.  O is divided by the sum of
 // the 16-bit probabilities the P.V product used (so the rounding of a
@@ -43,6 +47,17 @@ constexpr int kThreadsTC = 320;
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kRescaleLog2 = 8.0f;
+
+// Share of the softmax exponentials computed on the FMA pipe instead of the
+// MUFU unit: FA_POLY_PAIRS of every 16 element pairs (unmasked tiles only).
+// Measured on B200 at S=4096, B=4, non-causal, TFLOP/s (D64 / D128):
+// 0 -> 609 / 1004, 2 -> 512 / 817, 4 -> 467 / 770: the extra FMA/ALU
+// instructions cost more than the MUFU time they free, so the default is 0.
+#ifndef FA_POLY_PAIRS
+#define FA_POLY_PAIRS 0
+#endif
+__host__ __device__ constexpr bool poly_pair(int i) { return ((i * FA_POLY_PAIRS) % 16) < FA_POLY_PAIRS; }
+
 constexpr unsigned long long kTcWaitNs = kWaitLimitNs;
 
 template <int D>
@@ -65,7 +80,9 @@ struct TcCfg {
   static constexpr int B_S = B_VE + NSV;     // 2
   static constexpr int B_P = B_S + 2;        // 2
   static constexpr int B_O = B_P + 2;        // 2
-  static constexpr int B_DRAIN = B_O + 2;
+  static constexpr int B_SF = B_O + 2;       // 2: S read out of TMEM (separate-P layout)
+  static constexpr int B_PV = B_SF + 2;      // 2: PV product done (separate-P layout)
+  static constexpr int B_DRAIN = B_PV + 2;
   static constexpr int NBAR = B_DRAIN + 1;
   static constexpr int OFF_TMEM = OFF_BAR + 8 * NBAR;
   static constexpr int OFF_ABORT = OFF_TMEM + 4;
@@ -79,6 +96,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = TcCfg<D>;
+  // Head dim 64 leaves TMEM room for P beside O (P_t at [256+128t+64, +64)),
+  // so S_t can be refilled while P_t still feeds the PV product.
+  constexpr bool kSepP = (D == 64);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -116,6 +136,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       mbar_init(bar(C::B_S + t), 1);
       mbar_init(bar(C::B_P + t), 4 * 32);
       mbar_init(bar(C::B_O + t), 1);
+      mbar_init(bar(C::B_SF + t), 4 * 32);
+      mbar_init(bar(C::B_PV + t), 1);
     }
     mbar_init(bar(C::B_DRAIN), 1);
     *abort_flag = 0;
@@ -187,6 +209,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       constexpr uint32_t idesc_pv = make_idesc(kBf, 128, D, true);
       const uint32_t tS[2] = {tmem, tmem + 128};
       const uint32_t tO[2] = {tmem + 256, tmem + 384};
+      const uint32_t tP[2] = {kSepP ? tmem + 256 + D : tS[0], kSepP ? tmem + 384 + D : tS[1]};
       auto issue_qk = [&](int t, int st) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -200,7 +223,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 #pragma unroll
         for (int kk = 0; kk < kRows / 16; ++kk) {
           const uint64_t bd = make_sdesc_sw128(sb + C::OFF_V + st * C::TILE + kk * 16 * 128, C::CHUNK, 1024);
-          mma_ts(tO[t], tS[t] + kk * 8, bd, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+          mma_ts(tO[t], tP[t] + kk * 8, bd, idesc_pv, (acc || kk > 0) ? 1u : 0u);
         }
       };
       bool ok = mbar_wait(bar(C::B_Q), 0, abort_flag, kTcWaitNs);
@@ -213,7 +236,44 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         mma_commit(bar(C::B_S + 1));
         mma_commit(bar(C::B_KE + 0));
       }
-      for (int j = 0; ok && j < n_tiles; ++j) {
+      // Separate-P order: QK_t(j+1) as soon as the softmax has read S_t(j),
+      // PV_t(j) once it has written P_t(j).
+      for (int j = 0; kSepP && ok && j < n_tiles; ++j) {
+        const int sv = j % C::NSV, uv = j / C::NSV;
+        const int sk1 = (j + 1) % C::NSK, uk1 = (j + 1) / C::NSK;
+        const bool more = j + 1 < n_tiles;
+        if (more) {
+          ok = mbar_wait(bar(C::B_KF + sk1), uk1 & 1, abort_flag, kTcWaitNs) &&
+               mbar_wait(bar(C::B_SF + 0), j & 1, abort_flag, kTcWaitNs);
+          if (!ok) break;
+          tc_fence_after();
+          issue_qk(0, sk1);
+          mma_commit(bar(C::B_S + 0));
+        }
+        ok = mbar_wait(bar(C::B_VF + sv), uv & 1, abort_flag, kTcWaitNs) &&
+             mbar_wait(bar(C::B_P + 0), j & 1, abort_flag, kTcWaitNs);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(0, sv, j > 0);
+        mma_commit(bar(C::B_PV + 0));
+        if (!more) mma_commit(bar(C::B_O + 0));
+        if (more) {
+          ok = mbar_wait(bar(C::B_SF + 1), j & 1, abort_flag, kTcWaitNs);
+          if (!ok) break;
+          tc_fence_after();
+          issue_qk(1, sk1);
+          mma_commit(bar(C::B_S + 1));
+          mma_commit(bar(C::B_KE + sk1));
+        }
+        ok = mbar_wait(bar(C::B_P + 1), j & 1, abort_flag, kTcWaitNs);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(1, sv, j > 0);
+        mma_commit(bar(C::B_PV + 1));
+        mma_commit(bar(C::B_VE + sv));
+        if (!more) mma_commit(bar(C::B_O + 1));
+      }
+      for (int j = 0; !kSepP && ok && j < n_tiles; ++j) {
         const int sv = j % C::NSV, uv = j / C::NSV;
         const int sk1 = (j + 1) % C::NSK, uk1 = (j + 1) / C::NSK;
         const bool more = j + 1 < n_tiles;
@@ -258,6 +318,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     const uint32_t lanes = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lanes + t * 128;
     const uint32_t tO = tmem + lanes + 256 + t * 128;
+    const uint32_t tP = kSepP ? tO + D : tS;
     const int qi = q0 + t * kRows + r;
     const int qpos = qi + off;
     const int qpos_first = q0 + off, qpos_last = qlast + off;
@@ -277,6 +338,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
       tmem_wait_ld();
       reg_fence(s);
+      if (kSepP) {
+        // S_t may be overwritten by the next QK^T from here on
+        tc_fence_before();
+        mbar_arrive(bar(C::B_SF + t));
+      }
       const int k0 = (kt_begin + j) * kRows;
       const bool full = (k0 + kRows <= p.Sk) && (p.wl < 0 || k0 >= qpos_last - p.wl) &&
                         (p.wr < 0 || k0 + kRows - 1 <= qpos_first + p.wr);
@@ -297,11 +363,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       {
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int i = 0; i < kRows; i += 4) {
-          m4[0] = fmaxf(m4[0], f32(s[i]));
-          m4[1] = fmaxf(m4[1], f32(s[i + 1]));
-          m4[2] = fmaxf(m4[2], f32(s[i + 2]));
-          m4[3] = fmaxf(m4[3], f32(s[i + 3]));
+        for (int i = 0; i < kRows; i += 8) {
+          m4[0] = fmax3(m4[0], f32(s[i]), f32(s[i + 1]));
+          m4[1] = fmax3(m4[1], f32(s[i + 2]), f32(s[i + 3]));
+          m4[2] = fmax3(m4[2], f32(s[i + 4]), f32(s[i + 5]));
+          m4[3] = fmax3(m4[3], f32(s[i + 6]), f32(s[i + 7]));
         }
         mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       }
@@ -312,30 +378,56 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       const float alpha = move ? fast_exp2(m_run - mx) : 1.f;
       if (move) m_run = mx;
       const float mu = (m_run == -INFINITY) ? 0.f : m_run;
-      // P = 2^(s*sl - mu), packed to 16 bits over the first 64 columns of S.
+      // P = 2^(s*sl - mu), packed to 16 bits into P_t (over the first 64
+      // columns of S_t at head dim 128).
       // Two row sums: of the exact fp32 values (for the LSE) and of the
       // 16-bit values the P.V product actually uses (for O = sum(P V) / l),
       // so that the rounding of a dominant probability cancels in O.
-      float rs[2] = {0.f, 0.f}, rq[2] = {0.f, 0.f};
+      // packed f32x2 arithmetic: one instruction per element pair for the
+      // scale-and-shift and for each of the two row sums
+      const unsigned long long sl2 = f2_pack(sl, sl), nmu2 = f2_pack(-mu, -mu);
+      unsigned long long rs2 = f2_pack(0.f, 0.f), rq2 = f2_pack(0.f, 0.f);
+      uint32_t pkall[4][16];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
+        uint32_t (&pk)[16] = pkall[c];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = fast_exp2(fmaf(f32(s[c * 32 + 2 * i]), sl, -mu));
-          const float p1 = fast_exp2(fmaf(f32(s[c * 32 + 2 * i + 1]), sl, -mu));
-          rs[i & 1] += p0 + p1;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(f32(s[c * 32 + 2 * i]), f32(s[c * 32 + 2 * i + 1])), sl2, nmu2), x0, x1);
+          float p0, p1;
+          if (full && poly_pair(i)) {
+            exp2_poly2(x0, x1, p0, p1);
+          } else {
+            p0 = fast_exp2(x0);
+            p1 = fast_exp2(x1);
+          }
+          rs2 = f2_add(rs2, f2_pack(p0, p1));
           pk[i] = Elem<T>::pack(p0, p1);
           const float2 pr = Elem<T>::unpack(pk[i]);
-          rq[i & 1] += pr.x + pr.y;
+          rq2 = f2_add(rq2, f2_pack(pr.x, pr.y));
         }
-        tmem_st16(tS + c * 16, pk);
+        if (!kSepP) tmem_st16(tP + c * 16, pk);
       }
-      l_run = l_run * alpha + (rs[0] + rs[1]);
-      l_q = l_q * alpha + (rq[0] + rq[1]);
+      if (kSepP) {
+        // P_t and O_t are free once PV_t(j-1) has completed
+        if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(bar(C::B_PV + t), (j - 1) & 1, abort_flag, kTcWaitNs))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_st16(tP + c * 16, pkall[c]);
+      }
+      float rsa, rsb, rqa, rqb;
+      f2_unpack(rs2, rsa, rsb);
+      f2_unpack(rq2, rqa, rqb);
+      l_run = l_run * alpha + (rsa + rsb);
+      l_q = l_q * alpha + (rqa + rqb);
       if (__any_sync(0xffffffffu, move && j > 0 && alpha != 1.f)) {
-        // O(j-1) is complete: S(j) was committed after PV(j-1); PV(j) waits
-        // for this tile's arrive below.
+        // O(j-1) is complete (head dim 128: S(j) was committed after
+        // PV(j-1); head dim 64: waited for above); PV(j) waits for this
+        // tile's arrive below.
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t u[32];

@@ -228,6 +228,17 @@ fa_status fa_selftest_bounded_wait(const int* flag, int expected, long long limi
  */
 void fa_set_trace_events(void* start_event, void* stop_event);
 
+/*
+ * Diagnostic: y[i] = 2^x[i] for n device floats, computed with the FMA-pipe
+ * polynomial that the forward kernel can use for a share of its softmax
+ * exponentials (compile-time FA_POLY_PAIRS; off by default because it
+ * measured slower).  Arguments below -125 are clamped to -125.  x and y are
+ * device pointers the caller owns; returns FA_ERR_INVALID_ARG for n < 0 or a
+ * null pointer with n > 0.  For tests that hold it to its error bound
+ * against float64.
+ */
+fa_status fa_selftest_exp2_poly(const float* x, float* y, int n, fa_stream_t stream);
+
 /* Number of kernels the last fa_* call launched (for launch accounting). */
 int fa_last_launch_count(void);
 
