@@ -95,9 +95,12 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int nkb = (p.Sk + kKeys - 1) / kKeys;
-  const int kb = blockIdx.x % nkb;
-  const int hkv = (blockIdx.x / nkb) % p.Hkv;
-  const int b = blockIdx.x / (nkb * p.Hkv);
+  // a right bound (causal) gives early key blocks the most query blocks, a
+  // left bound alone the late ones: those go first
+  int kb, hb;
+  group_order((int)blockIdx.x, nkb, p.Hkv * p.B, p.wr < 0 && p.wl >= 0, kb, hb);
+  const int hkv = hb % p.Hkv;
+  const int b = hb / p.Hkv;
   const int off = p.Sk - p.Sq;
   const int k0 = kb * kKeys;
   const int k1 = min(k0 + kKeys, p.Sk) - 1;
@@ -497,6 +500,7 @@ cudaError_t launch_t(const BwdParams& p, const CUtensorMap& mq, const CUtensorMa
   const int nkb = (p.Sk + kKeys - 1) / kKeys;
   const long long items = (long long)nkb * p.Hkv * p.B;
   if (items == 0) return cudaSuccess;
+  if (items > 0x7fffffffLL) return cudaErrorInvalidValue;  // block index is an int
   trace_begin(s);
   kern<<<(unsigned)items, kThreadsB, smem, s>>>(mq, mk, mv, mdo, mdq, p);
   trace_end(s);

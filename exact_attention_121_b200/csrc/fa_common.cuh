@@ -200,6 +200,23 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float&
   y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
+// Order of CTAs over (work item, head) pairs for a 1-D grid of
+// n_items * n_heads blocks.  Heads go in groups of kHeadGroup; inside a group
+// every head's item of one rank comes before the next rank.  A wave of CTAs
+// then covers few heads (their K/V stays in L2), and with `reverse` the
+// highest item index comes first, so that the items that see the most keys
+// (causal masks make them uneven) start first and the last wave is light.
+constexpr int kHeadGroup = 8;
+__device__ __forceinline__ void group_order(int L, int n_items, int n_heads, bool reverse, int& item, int& head) {
+  const int per_group = kHeadGroup * n_items;
+  const int grp = L / per_group;
+  const int r = L - grp * per_group;
+  const int gsz = min(kHeadGroup, n_heads - grp * kHeadGroup);
+  const int rank = r / gsz;
+  head = grp * kHeadGroup + (r - rank * gsz);
+  item = reverse ? n_items - 1 - rank : rank;
+}
+
 // max(a, b, c) in one instruction (three-operand form, sm_100 and later).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;

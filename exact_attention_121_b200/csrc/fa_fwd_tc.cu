@@ -109,9 +109,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_qp = (p.Sq + 2 * kRows - 1) / (2 * kRows);
-  const int qp = (p.wr >= 0) ? (n_qp - 1 - (int)blockIdx.x) : (int)blockIdx.x;
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
+  // with a right bound (causal) later query pairs see more keys: first
+  int qp, hb;
+  group_order((int)blockIdx.x, n_qp, p.Hq * p.B, p.wr >= 0, qp, hb);
+  const int h = hb % p.Hq;
+  const int b = hb / p.Hq;
   const int g = h / p.G;
   const int q0 = qp * 2 * kRows;
   const int off = p.Sk - p.Sq;
@@ -498,7 +500,9 @@ cudaError_t launch_t(const FwdParams& p, const CUtensorMap& mq, const CUtensorMa
   constexpr int smem = TcCfg<D>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((p.Sq + 255) / 256, p.Hq, p.B);
+  const long long ctas = (long long)((p.Sq + 255) / 256) * p.Hq * p.B;
+  if (ctas > 0x7fffffffLL) return cudaErrorInvalidValue;  // block index is an int
+  dim3 grid((unsigned)ctas);
   trace_begin(s);
   kern<<<grid, kThreadsTC, smem, s>>>(mq, mk, mv, p);
   trace_end(s);
