@@ -5,7 +5,8 @@ A step is one pass of the whole hot path over one batch of synthetic inputs:
   * the seqlen sweep at hidden 2048 (H=32,D=64 and H=16,D=128; S = 512..16k,
     B = 16384/S; causal and non-causal; bf16): forward + backward of each point;
   * the GQA + local-attention workload (B=2, S=4096, Hq=32, Hkv=8, D=128,
-    window (1024,0), softcap 30): forward + backward;
+    window (1024,0), softcap 30): forward + backward, once with atomic and
+    once with deterministic (ordered) dQ accumulation;
   * the paged KV-cache decode (B=8, Hq=32, Hkv=8, D=128, lengths U[1,32768],
     page 256): append + split-KV attention + combine.
 ``value`` is algorithmic attention TFLOP/s of the whole step (4*D flops per
@@ -158,7 +159,7 @@ class AttnUnit:
 
     def name(self):
         c = self.cfg
-        return "H%dD%dS%d%s" % (c["Hq"], c["D"], c["Sq"], "c" if c["causal"] else "n")
+        return "H%dD%dS%d%s%s" % (c["Hq"], c["D"], c["Sq"], "c" if c["causal"] else "n", "-det" if self.det else "")
 
     def run(self, tracer):
         api = self.api
@@ -327,6 +328,7 @@ def build_units(dev, workload, point=None):
             units.append(AttnUnit(cfg, dev))
     if workload in ("full", "gqa"):
         units.append(AttnUnit(inputs.gqa_local_config(), dev))
+        units.append(AttnUnit(inputs.gqa_local_config(), dev, deterministic=True))
     if workload in ("full", "decode"):
         units.append(DecodeUnit(inputs.paged_decode_config(), dev))
     if workload == "small":

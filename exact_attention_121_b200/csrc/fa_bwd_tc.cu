@@ -72,7 +72,8 @@ struct BwdTcCfg {
          B_DQT_FULL = 17, B_DQT_FREE = 18, NBAR = 19 };
   static constexpr int OFF_TMEM = OFF_BAR + 8 * NBAR;
   static constexpr int OFF_ABORT = OFF_TMEM + 4;
-  static constexpr int SMEM = OFF_ABORT + 4 + 1024;
+  static constexpr int OFF_ITEM = OFF_ABORT + 4;  // claimed work item (deterministic mode)
+  static constexpr int SMEM = OFF_ITEM + 4 + 1024;
 };
 
 __device__ __forceinline__ float f32(uint32_t u) { return __uint_as_float(u); }
@@ -94,27 +95,6 @@ __global__ void __launch_bounds__(kThreadsB, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int nkb = (p.Sk + kKeys - 1) / kKeys;
-  // a right bound (causal) gives early key blocks the most query blocks, a
-  // left bound alone the late ones: those go first
-  int kb, hb;
-  group_order((int)blockIdx.x, nkb, p.Hkv * p.B, p.wr < 0 && p.wl >= 0, kb, hb);
-  const int hkv = hb % p.Hkv;
-  const int b = hb / p.Hkv;
-  const int off = p.Sk - p.Sq;
-  const int k0 = kb * kKeys;
-  const int k1 = min(k0 + kKeys, p.Sk) - 1;
-  int i_min = 0, i_max = p.Sq - 1;
-  if (p.wr >= 0) i_min = max(i_min, k0 - off - p.wr);
-  if (p.wl >= 0) i_max = min(i_max, k1 - off + p.wl);
-  const int qb_lo = i_min / kQ;
-  const int n_qb = (i_max >= i_min) ? (i_max / kQ - qb_lo + 1) : 0;
-  const int n_iter = n_qb * p.G;
-  auto iter_q = [&](int it, int& h, int& q0) {
-    h = hkv * p.G + it / n_qb;
-    q0 = (qb_lo + it % n_qb) * kQ;
-  };
-
   if (threadIdx.x == 0) {
     mbar_init(bar(C::B_KV), 1);
     for (int x = 0; x < C::NQS; ++x) {
@@ -132,6 +112,10 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     mbar_init(bar(C::B_FIN), 1);
     mbar_init(bar(C::B_DRAIN), 1);
     *abort_flag = 0;
+    // Deterministic mode: items are claimed in order from a global counter,
+    // key block major, so every key block a CTA waits for below belongs to
+    // a CTA that is already running or done.
+    if (p.deterministic) *reinterpret_cast<volatile int*>(smem + C::OFF_ITEM) = atomicAdd(p.work_counter, 1);
     fence_mbar_init();
   }
   if (warp == kMmaWarpB) {
@@ -145,6 +129,33 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   auto fail = [&]() {
     *abort_flag = 1;
     report_status(p.status, kStatusTimeout);
+  };
+
+  const int nkb = (p.Sk + kKeys - 1) / kKeys;
+  int kb, hb;
+  if (p.deterministic) {
+    const int item = *reinterpret_cast<volatile int*>(smem + C::OFF_ITEM);
+    kb = item / (p.Hkv * p.B);
+    hb = item - kb * (p.Hkv * p.B);
+  } else {
+    // a right bound (causal) gives early key blocks the most query blocks, a
+    // left bound alone the late ones: those go first
+    group_order((int)blockIdx.x, nkb, p.Hkv * p.B, p.wr < 0 && p.wl >= 0, kb, hb);
+  }
+  const int hkv = hb % p.Hkv;
+  const int b = hb / p.Hkv;
+  const int off = p.Sk - p.Sq;
+  const int k0 = kb * kKeys;
+  const int k1 = min(k0 + kKeys, p.Sk) - 1;
+  int i_min = 0, i_max = p.Sq - 1;
+  if (p.wr >= 0) i_min = max(i_min, k0 - off - p.wr);
+  if (p.wl >= 0) i_max = min(i_max, k1 - off + p.wl);
+  const int qb_lo = i_min / kQ;
+  const int n_qb = (i_max >= i_min) ? (i_max / kQ - qb_lo + 1) : 0;
+  const int n_iter = n_qb * p.G;
+  auto iter_q = [&](int it, int& h, int& q0) {
+    h = hkv * p.G + it / n_qb;
+    q0 = (qb_lo + it % n_qb) * kQ;
   };
 
   if (warp == kLoadWarp) {
@@ -469,10 +480,31 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         if (!mbar_wait(bar(C::B_DQT_FULL), it & 1, abort_flag, kWaitNs)) {
           ok = false;
         } else {
-          tma_reduce_add_4d(&tmDQ, 0, h, q0, b, sb + C::OFF_DQ);
-          bulk_commit();
-          // the tile may be rewritten once the reduction has read it
-          bulk_wait_read_all();
+          int* sem = nullptr;
+          if (p.deterministic) {
+            // add after the key blocks before this one that see query block
+            // q0/64, in ascending order: wait for their count
+            sem = p.sem + ((size_t)b * p.Hq + h) * ((p.Sq + kQ - 1) / kQ) + q0 / kQ;
+            const int kb_lo = (p.wl >= 0) ? max(0, q0 + off - p.wl) / kKeys : 0;
+            if (!wait_eq_bounded(sem, kb - kb_lo, kWaitNs)) {
+              ok = false;
+              sem = nullptr;
+            }
+            fence_proxy_async_global();
+          }
+          if (ok) {
+            tma_reduce_add_4d(&tmDQ, 0, h, q0, b, sb + C::OFF_DQ);
+            bulk_commit();
+            if (sem) {
+              // the additions are complete in global memory before the count moves
+              bulk_wait_all();
+              fence_proxy_async_global();
+              red_release_add(sem, 1);
+            } else {
+              // the tile may be rewritten once the reduction has read it
+              bulk_wait_read_all();
+            }
+          }
           mbar_arrive(bar(C::B_DQT_FREE));
         }
       }
@@ -510,7 +542,7 @@ cudaError_t launch_t(const BwdParams& p, const CUtensorMap& mq, const CUtensorMa
 }  // namespace
 
 bool bwd_tc_supported(const BwdParams& p) {
-  return (p.D == 64 || p.D == 128) && !p.deterministic && p.Sq >= 1 && p.Sk >= 1 && tma_available();
+  return (p.D == 64 || p.D == 128) && p.Sq >= 1 && p.Sk >= 1 && tma_available();
 }
 
 cudaError_t launch_bwd_main_tc(const BwdParams& p, fa_dtype dt, cudaStream_t s) {

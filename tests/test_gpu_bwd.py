@@ -94,7 +94,8 @@ def test_gqa_local_full_size_slices(det):
             check_grad(dv[b:b + 1, :, g:g + 1], dv_r, f"dV b{b} g{g}")
 
 
-def test_deterministic_is_bit_identical():
+@pytest.mark.parametrize("which", [0, 1], ids=["auto", "mma"])
+def test_deterministic_is_bit_identical(which):
     cfg = inputs.gqa_local_config()
     q, k, v, do = inputs.attention_inputs(cfg["B"], cfg["Sq"], cfg["Sk"], cfg["Hq"], cfg["Hkv"], cfg["D"],
                                           cfg["dtype"], seed=cfg["seed"], amp=cfg["amp"])
@@ -102,9 +103,13 @@ def test_deterministic_is_bit_identical():
     qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
     out, lse = api.fa_fwd(qd, kd, vd, **kw)
     runs = []
-    for _ in range(3):
-        runs.append([t.clone() for t in api.fa_bwd(dod, qd, kd, vd, out, lse, deterministic=True, **kw)])
-    torch.cuda.synchronize()
+    _lib.load().fa_set_bwd_kernel(which)
+    try:
+        for _ in range(3):
+            runs.append([t.clone() for t in api.fa_bwd(dod, qd, kd, vd, out, lse, deterministic=True, **kw)])
+        torch.cuda.synchronize()
+    finally:
+        _lib.load().fa_set_bwd_kernel(0)
     for r in runs[1:]:
         for a, b in zip(runs[0], r):
             assert torch.equal(a.view(torch.int16), b.view(torch.int16))
