@@ -23,8 +23,10 @@
 // overlaps the products of iteration i+1.  TMEM (512 columns): buffer x at
 // [128x, 128x+128) holds S^T [0,64) | dP^T [64,128); the warps that handle
 // query half h write P^T (16-bit pairs) to [32h, 32h+16) and dS^T to
-// [64+32h, 64+32h+16), and dQ^T goes over [64,128) once dK has read dS^T;
-// dV [256,384), dK [384,512).  Warps 0-7 do the elementwise step (two warps
+// [64+32h, 64+32h+16).  Head dim 128: dQ^T goes over [64,128) once dK has
+// read dS^T; dV [256,384), dK [384,512).  Head dim 64: dV [256,320), dK
+// [320,384), and one N = 128 product per pair of blocks writes dQ^T of both
+// to [384,512).  Warps 0-7 do the elementwise step (two warps
 // per TMEM lane quarter, one per query half), warps 8-11 drain dQ, warp 12
 // loads (TMA for K, V, Q_i, dO_i; plain loads for LSE/Delta), warp 13 issues
 // the MMAs.  Every wait is bounded.
@@ -59,14 +61,20 @@ struct BwdTcCfg {
   static constexpr int Q_TILE = NCH * Q_CHUNK;
   static constexpr int DS_TILE = kKeys * kQ * 2;  // [128 keys][64 queries] 16-bit, swizzled
   static constexpr int DQ_TILE = kQ * D * 4;      // [64 queries][D] fp32, dense (TMA reduce box)
+  // Head dim 64: dQ^T of two consecutive blocks comes from one N = 128
+  // product, so dS keeps four buffers (a pair is two adjacent ones) and the
+  // drain stages two dQ tiles.
+  static constexpr bool PAIR = (D == 64);
+  static constexpr int NDS = PAIR ? 4 : 2;
+  static constexpr int NDQ = PAIR ? 2 : 1;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + KV_TILE;
   static constexpr int NQS = 3;                        // Q/dO/LSE/Delta stages
   static constexpr int OFF_Q = OFF_V + KV_TILE;        // NQS stages
   static constexpr int OFF_DO = OFF_Q + NQS * Q_TILE;  // NQS stages
-  static constexpr int OFF_DS = OFF_DO + NQS * Q_TILE;  // 2 buffers
-  static constexpr int OFF_DQ = OFF_DS + 2 * DS_TILE;   // 1 buffer
-  static constexpr int OFF_ROW = OFF_DQ + DQ_TILE;      // [stage][LSE*log2e 64 | Delta 64]
+  static constexpr int OFF_DS = OFF_DO + NQS * Q_TILE;  // NDS buffers
+  static constexpr int OFF_DQ = OFF_DS + NDS * DS_TILE; // NDQ tiles
+  static constexpr int OFF_ROW = OFF_DQ + NDQ * DQ_TILE;  // [stage][LSE*log2e 64 | Delta 64]
   static constexpr int OFF_BAR = OFF_ROW + NQS * 2 * kQ * 4;
   enum { B_KV = 0, B_QF = 1, B_QE = 4, B_SDP = 7, B_PDS = 9, B_DQF = 11, B_TMF = 13, B_FIN = 15, B_DRAIN = 16,
          B_DQT_FULL = 17, B_DQT_FREE = 18, NBAR = 19 };
@@ -85,6 +93,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
                   const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
   using C = BwdTcCfg<D_>;
   constexpr int D = C::D;
+  constexpr bool kPair = C::PAIR;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -221,7 +230,9 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       constexpr uint32_t idesc_s = make_idesc(kBf, 128, kQ, false, false);
       constexpr uint32_t idesc_kv = make_idesc(kBf, 128, D, true, false);
       constexpr uint32_t idesc_dq = make_idesc(kBf, 128, kQ, true, true);
-      const uint32_t tdV = tmem + 256, tdK = tmem + 384;
+      constexpr uint32_t idesc_dq2 = make_idesc(kBf, 128, 2 * kQ, true, true);
+      // head dim 64: dV [256,320), dK [320,384), dQ^T of a block pair [384,512)
+      const uint32_t tdV = tmem + 256, tdK = tmem + (kPair ? 320 : 384);
       auto issue_sdp = [&](int it) {
         const int x = it & 1, st = it % C::NQS;
         const uint32_t tb = tmem + x * 128;
@@ -245,7 +256,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         const int x = it & 1, st = it % C::NQS;
         const uint32_t tb = tmem + x * 128;
         const uint32_t q_st = sb + C::OFF_Q + st * C::Q_TILE, do_st = sb + C::OFF_DO + st * C::Q_TILE;
-        const uint32_t ds = sb + C::OFF_DS + x * C::DS_TILE;
+        const uint32_t ds = sb + C::OFF_DS + (it % C::NDS) * C::DS_TILE;
         const bool acc = it > 0;
 #pragma unroll
         for (int kk = 0; kk < kQ / 16; ++kk)
@@ -258,12 +269,24 @@ __global__ void __launch_bounds__(kThreadsB, 1)
           mma_ts(tdK, tb + 64 + (kk >> 1) * 32 + (kk & 1) * 8,
                  make_sdesc_sw128(q_st + kk * 16 * 128, C::Q_CHUNK, 1024), idesc_kv,
                  (acc || kk > 0) ? 1u : 0u);
+        if (kPair) return;
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk)
-          // M = 128 head dims; with D = 64 the second 64-row half of K^T
-          // points back at the first (LBO 0) and those TMEM lanes are unused.
           mma_ss(tb + 64, make_sdesc_sw128(sb + C::OFF_K + kk * 16 * 128, C::NCH > 1 ? C::KV_CHUNK : 0, 1024),
                  make_sdesc_sw128(ds + kk * 16 * 128, C::KV_CHUNK, 1024), idesc_dq, kk > 0 ? 1u : 0u);
+      };
+      // Head dim 64: dQ^T of blocks (it0, it0 + n - 1), n = 2 (or 1 for a
+      // last unpaired block) into [384, 384 + 64n): M = 128 head dims, where
+      // the second 64-row half of K^T points back at the first (LBO 0) and
+      // those TMEM lanes are unused; N = 64n queries from n adjacent dS
+      // buffers (LBO = one buffer).
+      auto issue_dq_pair = [&](int it0, int n) {
+        const uint32_t ds = sb + C::OFF_DS + (it0 % C::NDS) * C::DS_TILE;
+        const uint32_t idesc = n == 2 ? idesc_dq2 : idesc_dq;
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk)
+          mma_ss(tmem + 384, make_sdesc_sw128(sb + C::OFF_K + kk * 16 * 128, 0, 1024),
+                 make_sdesc_sw128(ds + kk * 16 * 128, C::DS_TILE, 1024), idesc, kk > 0 ? 1u : 0u);
       };
       bool ok = mbar_wait(bar(C::B_KV), 0, abort_flag, kWaitNs) && mbar_wait(bar(C::B_QF), 0, abort_flag, kWaitNs);
       if (ok) {
@@ -276,8 +299,9 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         if (it + 1 < n_iter) {
           const int x1 = (it + 1) & 1, u1 = (it + 1) >> 1;
           const int s1 = (it + 1) % C::NQS, v1 = (it + 1) / C::NQS;
+          // dQ^T(it-1) sits in buffer x1 at head dim 128: drained first
           ok = mbar_wait(bar(C::B_QF + s1), v1 & 1, abort_flag, kWaitNs) &&
-               (it + 1 < 2 || mbar_wait(bar(C::B_TMF + x1), (u1 - 1) & 1, abort_flag, kWaitNs));
+               (kPair || it + 1 < 2 || mbar_wait(bar(C::B_TMF + x1), (u1 - 1) & 1, abort_flag, kWaitNs));
           if (!ok) break;
           tc_fence_after();
           issue_sdp(it + 1);
@@ -287,7 +311,20 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         if (!ok) break;
         tc_fence_after();
         issue_grads(it);
-        mma_commit(bar(C::B_DQF + x));
+        if (!kPair) {
+          mma_commit(bar(C::B_DQF + x));
+        } else if ((it & 1) || it == n_iter - 1) {
+          // pair m = it / 2 complete (or the last block alone): its dQ^T
+          // region is free once the drain has read pair m - 1
+          const int m = it >> 1;
+          if (m >= 1 && !mbar_wait(bar(C::B_TMF), (m - 1) & 1, abort_flag, kWaitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_dq_pair(2 * m, (it & 1) ? 2 : 1);
+          mma_commit(bar(C::B_DQF));
+        }
         mma_commit(bar(C::B_QE + it % C::NQS));
       }
       if (ok) mma_commit(bar(C::B_FIN));
@@ -310,8 +347,10 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       int h, q0;
       iter_q(it, h, q0);
       (void)h;
-      bool w = mbar_wait(bar(C::B_SDP + x), u & 1, abort_flag, kWaitNs);
-      if (it >= 2) w = w && mbar_wait(bar(C::B_DQF + x), (u - 1) & 1, abort_flag, kWaitNs);
+      // S^T/dP^T(it) ready also means (commit order) that the products of
+      // it-2 that read this TMEM buffer and the dQ^T that read this dS
+      // buffer are done
+      const bool w = mbar_wait(bar(C::B_SDP + x), u & 1, abort_flag, kWaitNs);
       if (!__all_sync(0xffffffffu, w)) {
         ok = false;
         break;
@@ -327,7 +366,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       // [32hh+8sb, +8) and dS^T to [64+32hh+8sb, +8): inside columns this
       // warp has already read.
       const unsigned long long sl2 = f2_pack(p.scale_log2, p.scale_log2);
-      uint8_t* dsrow = smem + C::OFF_DS + x * C::DS_TILE + r * 128;
+      uint8_t* dsrow = smem + C::OFF_DS + (it % C::NDS) * C::DS_TILE + r * 128;
 #pragma unroll
       for (int sbk = 0; sbk < 2; ++sbk) {
         const int q16 = 32 * hh + 16 * sbk;  // first query of the sub-block
@@ -407,7 +446,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       for (int which = 0; which < 2; ++which) {
         const float mul = which ? p.scale : 1.f;
         T* dst = which ? dKr : dVr;
-        const uint32_t src = tmem + lanes + (which ? 384 : 256) + hh * (D / 2);
+        const uint32_t src = tmem + lanes + (which ? (kPair ? 320 : 384) : 256) + hh * (D / 2);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
           uint32_t v[32];
@@ -438,48 +477,60 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     const int wq = warp - kDqWarp0;          // TMEM lane quarter = head-dim slice
     const bool has_dims = wq * 32 < D;       // D = 64 uses two of the four warps
     const uint32_t lanes = (uint32_t)(wq * 32) << 16;
-    // The dQ tile of an iteration is [64 queries][D] fp32 in shared memory
-    // (one buffer); every drain thread writes its head-dim column, then
-    // one thread adds the whole tile into the global accumulator with a single
-    // tiled TMA reduction.  Rows past Sq fall outside the tensor and are
-    // skipped by the TMA unit.
+    // A drain group is one block (head dim 128, dQ^T in TMEM buffer it & 1)
+    // or a pair of blocks (head dim 64, dQ^T of both in [384, 512)).  The
+    // dQ tile of a block is [64 queries][D] fp32 in shared memory; every
+    // drain thread writes its head-dim column, then one thread adds each
+    // tile into the global accumulator with a single tiled TMA reduction.
+    // Rows past Sq fall outside the tensor and are skipped by the TMA unit.
     const bool issuer = (warp == kDqWarp0) && lane == 0;
+    const int n_groups = kPair ? (n_iter + 1) / 2 : n_iter;
     bool ok = true;
-    for (int it = 0; it < n_iter; ++it) {
-      const int x = it & 1, u = it >> 1;
-      int h, q0;
-      iter_q(it, h, q0);
-      bool w = mbar_wait(bar(C::B_DQF + x), u & 1, abort_flag, kWaitNs);
-      // the tile is free once the reduction of iteration it-1 has read it
-      if (it >= 1) w = w && mbar_wait(bar(C::B_DQT_FREE), (it - 1) & 1, abort_flag, kWaitNs);
+    for (int gi = 0; gi < n_groups; ++gi) {
+      const int it0 = kPair ? 2 * gi : gi;
+      const int cnt = kPair ? min(2, n_iter - it0) : 1;
+      const int bx = kPair ? 0 : (gi & 1);
+      const int ph = kPair ? (gi & 1) : ((gi >> 1) & 1);
+      bool w = mbar_wait(bar(C::B_DQF + bx), ph, abort_flag, kWaitNs);
+      // the tiles are free once the reductions of the previous group have read them
+      if (gi >= 1) w = w && mbar_wait(bar(C::B_DQT_FREE), (gi - 1) & 1, abort_flag, kWaitNs);
       if (!__all_sync(0xffffffffu, w)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float* tile = reinterpret_cast<float*>(smem + C::OFF_DQ);
       if (has_dims) {
-        uint32_t v[kQ];
-        const uint32_t tb = tmem + lanes + x * 128 + 64;
-        tmem_ld32(tb, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        tmem_ld32(tb + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-        tmem_wait_ld();
-        reg_fence(v);
-        tc_fence_before();
-        mbar_arrive(bar(C::B_TMF + x));
 #pragma unroll
-        for (int c = 0; c < kQ; ++c) tile[c * D + wq * 32 + lane] = f32(v[c]);
+        for (int i = 0; i < C::NDQ; ++i) {
+          if (i < cnt) {
+            uint32_t v[kQ];
+            const uint32_t tb = tmem + lanes + (kPair ? 384 + 64 * i : bx * 128 + 64);
+            tmem_ld32(tb, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+            tmem_ld32(tb + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+            tmem_wait_ld();
+            reg_fence(v);
+            if (i == cnt - 1) {
+              // dQ^T of the group is in registers: the region may be rewritten
+              tc_fence_before();
+              mbar_arrive(bar(C::B_TMF + bx));
+            }
+            float* tile = reinterpret_cast<float*>(smem + C::OFF_DQ + i * C::DQ_TILE);
+#pragma unroll
+            for (int c = 0; c < kQ; ++c) tile[c * D + wq * 32 + lane] = f32(v[c]);
+          }
+        }
         fence_proxy_async_smem();
       } else {
         // no head-dim rows here (D = 64): keep the barrier phases in step
         tc_fence_before();
-        mbar_arrive(bar(C::B_TMF + x));
+        mbar_arrive(bar(C::B_TMF + bx));
       }
       mbar_arrive(bar(C::B_DQT_FULL));
       if (issuer) {
-        if (!mbar_wait(bar(C::B_DQT_FULL), it & 1, abort_flag, kWaitNs)) {
-          ok = false;
-        } else {
+        if (!mbar_wait(bar(C::B_DQT_FULL), gi & 1, abort_flag, kWaitNs)) ok = false;
+        for (int i = 0; ok && i < cnt; ++i) {
+          int h, q0;
+          iter_q(it0 + i, h, q0);
           int* sem = nullptr;
           if (p.deterministic) {
             // add after the key blocks before this one that see query block
@@ -488,25 +539,22 @@ __global__ void __launch_bounds__(kThreadsB, 1)
             const int kb_lo = (p.wl >= 0) ? max(0, q0 + off - p.wl) / kKeys : 0;
             if (!wait_eq_bounded(sem, kb - kb_lo, kWaitNs)) {
               ok = false;
-              sem = nullptr;
+              break;
             }
             fence_proxy_async_global();
           }
-          if (ok) {
-            tma_reduce_add_4d(&tmDQ, 0, h, q0, b, sb + C::OFF_DQ);
-            bulk_commit();
-            if (sem) {
-              // the additions are complete in global memory before the count moves
-              bulk_wait_all();
-              fence_proxy_async_global();
-              red_release_add(sem, 1);
-            } else {
-              // the tile may be rewritten once the reduction has read it
-              bulk_wait_read_all();
-            }
+          tma_reduce_add_4d(&tmDQ, 0, h, q0, b, sb + C::OFF_DQ + i * C::DQ_TILE);
+          bulk_commit();
+          if (sem) {
+            // the additions are complete in global memory before the count moves
+            bulk_wait_all();
+            fence_proxy_async_global();
+            red_release_add(sem, 1);
           }
-          mbar_arrive(bar(C::B_DQT_FREE));
         }
+        // the tiles may be rewritten once the reductions have read them
+        bulk_wait_read_all();
+        mbar_arrive(bar(C::B_DQT_FREE));
       }
       if (!__all_sync(0xffffffffu, ok)) break;
     }
