@@ -30,33 +30,58 @@ constexpr int kKB = 64;   // keys per CTA
 constexpr int kQB = 64;   // query rows per iteration
 constexpr int kBwdThreads = 128;
 
-template <typename T>
+// Delta_i = sum_d dO_id O_id for every (b, i, h) row, the fp32 dQ
+// accumulator zeroed, and (deterministic mode) the ordering counters reset.
+// A row is D/8 lanes with 16-byte loads; a warp takes 32/(D/8) rows per step
+// and keeps kPreSteps steps of loads in flight (the kernel is HBM-bound).
+constexpr int kPreSteps = 4;
+template <typename T, int D>
 __global__ void bwd_preprocess_kernel(const BwdParams p, int n_sem) {
-  const int D = p.D;
+  constexpr int kLanesPerRow = D / 8;
+  constexpr int kRowsPerStep = 32 / kLanesPerRow;
   const long long rows = (long long)p.B * p.Sq * p.Hq;  // (b, i, h) order
   const int lane = threadIdx.x & 31;
+  const int sub = lane / kLanesPerRow, l = lane % kLanesPerRow;
   const long long warp0 = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
   const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
-  for (long long r = warp0; r < rows; r += nwarps) {
-    const T* dO = reinterpret_cast<const T*>(p.dout) + r * D;
-    const T* O = reinterpret_cast<const T*>(p.o) + r * D;
-    float acc = 0.f;
-    for (int d = lane * 4; d < D; d += 128) {
-      const uint2 a = *reinterpret_cast<const uint2*>(dO + d);
-      const uint2 c = *reinterpret_cast<const uint2*>(O + d);
-      const float2 a0 = Elem<T>::unpack(a.x), a1 = Elem<T>::unpack(a.y);
-      const float2 c0 = Elem<T>::unpack(c.x), c1 = Elem<T>::unpack(c.y);
-      acc += a0.x * c0.x + a0.y * c0.y + a1.x * c1.x + a1.y * c1.y;
-      *reinterpret_cast<float4*>(p.dq_accum + r * D + d) = make_float4(0.f, 0.f, 0.f, 0.f);
+  constexpr int kRowsPerWarp = kRowsPerStep * kPreSteps;
+  for (long long base = warp0 * kRowsPerWarp; base < rows; base += nwarps * kRowsPerWarp) {
+    uint4 a[kPreSteps], c[kPreSteps];
+#pragma unroll
+    for (int u = 0; u < kPreSteps; ++u) {
+      const long long r = base + u * kRowsPerStep + sub;
+      if (r < rows) {
+        a[u] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.dout) + r * D + l * 8));
+        c[u] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.o) + r * D + l * 8));
+      } else {
+        a[u] = c[u] = make_uint4(0, 0, 0, 0);
+      }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) {
-      const int h = (int)(r % p.Hq);
-      const long long bi = r / p.Hq;
-      const int i = (int)(bi % p.Sq);
-      const int b = (int)(bi / p.Sq);
-      p.delta[((size_t)b * p.Hq + h) * p.Sq + i] = acc;
+    for (int u = 0; u < kPreSteps; ++u) {
+      const long long r = base + u * kRowsPerStep + sub;
+      const uint32_t av[4] = {a[u].x, a[u].y, a[u].z, a[u].w}, cv[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
+      float acc = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 x = Elem<T>::unpack(av[j]), y = Elem<T>::unpack(cv[j]);
+        acc = fmaf(x.x, y.x, acc);
+        acc = fmaf(x.y, y.y, acc);
+      }
+#pragma unroll
+      for (int o = kLanesPerRow / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (r < rows) {
+        float4* z = reinterpret_cast<float4*>(p.dq_accum + r * D + l * 8);
+        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (l == 0) {
+          const int h = (int)(r % p.Hq);
+          const long long bi = r / p.Hq;
+          const int i = (int)(bi % p.Sq);
+          const int b = (int)(bi / p.Sq);
+          p.delta[((size_t)b * p.Hq + h) * p.Sq + i] = acc;
+        }
+      }
     }
   }
   if (p.deterministic) {
@@ -389,7 +414,10 @@ template <typename T>
 cudaError_t launch_bwd_t(const BwdParams& p, cudaStream_t s, int* launches) {
   const int nqb = (p.Sq + kQB - 1) / kQB;
   const int n_sem = p.B * p.Hq * nqb;
-  bwd_preprocess_kernel<T><<<148 * 8, 256, 0, s>>>(p, n_sem);
+  if (p.D == 64)
+    bwd_preprocess_kernel<T, 64><<<148 * 8, 256, 0, s>>>(p, n_sem);
+  else
+    bwd_preprocess_kernel<T, 128><<<148 * 8, 256, 0, s>>>(p, n_sem);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   ++*launches;
