@@ -181,13 +181,13 @@ class AttnUnit:
         self.pin_in = [pinned.get(t, i) for i, t in enumerate(self.host_in)]
         self.pin_out = [pinned.get_like(t) for t in (self.out, self.dq, self.dk, self.dv)]
 
-    def run_e2e(self, tracer):
+    def copy_in(self):
         for dst, src in zip((self.q, self.k, self.v, self.do), self.pin_in):
             dst.copy_(src, non_blocking=True)
-        n = self.run(tracer)
+
+    def copy_out(self):
         for dst, src in zip(self.pin_out, (self.out, self.dq, self.dk, self.dv)):
             dst.copy_(src, non_blocking=True)
-        return n
 
     def e2e_bytes(self):
         return (sum(t.numel() * t.element_size() for t in (self.q, self.k, self.v, self.do)),
@@ -239,12 +239,12 @@ class DecodeUnit:
         self.pin_in = [pinned.get(t, i) for i, t in enumerate(self.host_in)]
         self.pin_out = [pinned.get_like(self.out)]
 
-    def run_e2e(self, tracer):
+    def copy_in(self):
         for dst, src in zip((self.q, self.kn, self.vn), self.pin_in):
             dst.copy_(src, non_blocking=True)
-        n = self.run(tracer)
+
+    def copy_out(self):
         self.pin_out[0].copy_(self.out, non_blocking=True)
-        return n
 
     def e2e_bytes(self):
         return (sum(t.numel() * t.element_size() for t in (self.q, self.kn, self.vn)),
@@ -252,7 +252,9 @@ class DecodeUnit:
 
 
 class Pinned:
-    """Pinned host staging buffers, shared between units of equal byte size."""
+    """Pinned host staging buffers: one per input tensor (each unit's own
+    values), outputs shared between units of equal byte size (the copies out
+    run in order on one stream)."""
 
     def __init__(self):
         self.pool = {}
@@ -264,9 +266,7 @@ class Pinned:
         return self.pool[key]
 
     def get(self, t, slot):
-        nb = t.numel() * t.element_size()
-        buf = self._buf(nb, "in%d" % slot)
-        view = buf.view(t.dtype).view(t.shape)
+        view = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
         view.copy_(t)
         return view
 
@@ -338,20 +338,61 @@ def build_units(dev, workload, point=None):
 
 
 def time_steps(units, steps, warmup, tracer, e2e=False, barrier=None):
+    """Device time of `steps` steps.  With e2e, every unit's inputs come from
+    pinned host memory on a copy-in stream and its outputs go back on a
+    copy-out stream, overlapped with the other units' kernels: unit u's
+    kernels wait for its inputs, its copy-out waits for its kernels, its next
+    copy-in waits for its kernels and its next kernels wait for its copy-out."""
     stream = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     launches = 0
+
+    def one_step(tr, ev):
+        n = 0
+        for i, u in enumerate(units):
+            if not e2e:
+                n += u.run(tr)
+                continue
+            with torch.cuda.stream(s_in):
+                if ev["done"][i] is not None:
+                    s_in.wait_event(ev["done"][i])
+                u.copy_in()
+                e_in = torch.cuda.Event()
+                e_in.record(s_in)
+            stream.wait_event(e_in)
+            if ev["out"][i] is not None:
+                stream.wait_event(ev["out"][i])
+            n += u.run(tr)
+            e_done = torch.cuda.Event()
+            e_done.record(stream)
+            ev["done"][i] = e_done
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(e_done)
+                u.copy_out()
+                e_out = torch.cuda.Event()
+                e_out.record(s_out)
+            ev["out"][i] = e_out
+        return n
+
+    ev = {"done": [None] * len(units), "out": [None] * len(units)}
     for _ in range(warmup):
-        for u in units:
-            (u.run_e2e if e2e else u.run)(Tracer(tracer.lib))
+        one_step(Tracer(tracer.lib), ev)
     torch.cuda.synchronize()
     if barrier:
         barrier()
     torch.cuda.synchronize()
+    ev = {"done": [None] * len(units), "out": [None] * len(units)}
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
+    s_in.wait_event(start)
+    s_out.wait_event(start)
     for _ in range(steps):
-        for u in units:
-            launches += (u.run_e2e if e2e else u.run)(tracer)
+        launches += one_step(tracer, ev)
+    # the step ends when the last result is back in host memory
+    for side in (s_in, s_out):
+        e_end = torch.cuda.Event()
+        e_end.record(side)
+        stream.wait_event(e_end)
     stop.record(stream)
     torch.cuda.synchronize()
     if barrier:
