@@ -26,7 +26,7 @@ there, so each function states the reading it implements):
   running sum updated block by block), recomputation in the backward.
   -> :func:`attn_fwd_online` (used only to pin :func:`attn_fwd`).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 
 * softcap: ``s = softcap * tanh(u / softcap)`` applied after the scale and
   before the mask; ``softcap <= 0`` switches it off.
@@ -41,6 +41,10 @@ Readings where the pages are silent (each is listed in the design doc):
   ``cache_seqlens[b] + Snew`` keys and does not update ``cache_seqlens``.
 * split s of a sequence with P pages covers pages
   ``ceil(s*P/n) .. ceil((s+1)*P/n) - 1``.
+* varlen: sequences packed along the token axis with ``cu_seqlens`` offsets
+  (sequence b is tokens ``cu[b] .. cu[b+1]-1``); each sequence is attended on
+  its own, with the masks and the bottom-right alignment of its own lengths;
+  the LSE layout is (Hq, total_q).
 
 Layouts follow the pages' (batch, seqlen, nheads, headdim) convention.
 """
@@ -429,3 +433,47 @@ def combine_splits(o_parts, lse_parts):
     wn = np.where(finite[None], w / np.where(finite, tot, 1.0)[None], 0.0)  # (n, Hq, Sq)
     o = np.einsum("nhi,nihd->ihd", wn, o_parts)
     return o, lse
+
+
+# ---------------------------------------------------------------------------
+# variable-length (packed) batches
+# ---------------------------------------------------------------------------
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale=None, causal=False, window_left=-1,
+                    window_right=-1, softcap=0.0):
+    """Packed batch: q (total_q, Hq, D), k/v (total_k, Hkv, D).  Every
+    sequence b is the dense problem on its own token slices.  Returns O
+    (total_q, Hq, D) and LSE (Hq, total_q)."""
+    cq, ck = np.asarray(cu_seqlens_q), np.asarray(cu_seqlens_k)
+    Hq = q.shape[1]
+    out = np.zeros(q.shape, dtype=np.float64)
+    lse = np.full((Hq, q.shape[0]), NEG_INF)
+    for b in range(len(cq) - 1):
+        q0, q1, k0, k1 = int(cq[b]), int(cq[b + 1]), int(ck[b]), int(ck[b + 1])
+        if q1 == q0:
+            continue
+        o_b, l_b = attn_fwd(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1], scale, causal, window_left,
+                            window_right, softcap)
+        out[q0:q1] = o_b[0]
+        lse[:, q0:q1] = l_b[0]
+    return out, lse
+
+
+def attn_bwd_varlen(dout, q, k, v, cu_seqlens_q, cu_seqlens_k, scale=None, causal=False, window_left=-1,
+                    window_right=-1, softcap=0.0):
+    """Gradients of sum(dout * O) for a packed batch; each sequence is the
+    dense backward on its own slices.  Returns dq, dk, dv in the packed
+    layouts."""
+    cq, ck = np.asarray(cu_seqlens_q), np.asarray(cu_seqlens_k)
+    dq = np.zeros(q.shape, dtype=np.float64)
+    dk = np.zeros(k.shape, dtype=np.float64)
+    dv = np.zeros(v.shape, dtype=np.float64)
+    for b in range(len(cq) - 1):
+        q0, q1, k0, k1 = int(cq[b]), int(cq[b + 1]), int(ck[b]), int(ck[b + 1])
+        if q1 == q0 or k1 == k0:
+            continue
+        g = attn_bwd(dout[None, q0:q1], q[None, q0:q1], k[None, k0:k1], v[None, k0:k1], scale, causal,
+                     window_left, window_right, softcap)
+        dq[q0:q1], dk[k0:k1], dv[k0:k1] = g[0][0], g[1][0], g[2][0]
+    return dq, dk, dv
+

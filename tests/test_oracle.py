@@ -419,3 +419,92 @@ def test_rows_equal_full_forward():
             orow, lrow = oracle.attn_fwd_rows(q, k, v, b, h, rows, **kw)
             np.testing.assert_allclose(orow, o[b, rows, h], atol=1e-14)
             np.testing.assert_allclose(lrow, lse[b, h, rows], atol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# variable-length (packed) batches
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal,wl,wr,cap", [(False, -1, -1, 0.0), (True, -1, -1, 0.0), (False, 3, 2, 4.0)])
+def test_varlen_equal_lengths_equal_dense_batch(causal, wl, wr, cap):
+    rng = np.random.default_rng(40)
+    B, Sq, Sk, Hq, Hkv, D = 3, 7, 9, 4, 2, 8
+    q, k, v, do = _rand((B, Sq, Hq, D), rng), _rand((B, Sk, Hkv, D), rng), _rand((B, Sk, Hkv, D), rng), \
+        _rand((B, Sq, Hq, D), rng)
+    cq, ck = np.arange(B + 1) * Sq, np.arange(B + 1) * Sk
+    o_d, l_d = attn64.attn_fwd(q, k, v, 0.4, causal, wl, wr, cap)
+    o_v, l_v = attn64.attn_fwd_varlen(q.reshape(B * Sq, Hq, D), k.reshape(B * Sk, Hkv, D), v.reshape(B * Sk, Hkv, D),
+                                      cq, ck, 0.4, causal, wl, wr, cap)
+    np.testing.assert_allclose(o_v, o_d.reshape(B * Sq, Hq, D), atol=1e-13)
+    # LSE (B, Hq, Sq) -> (Hq, B*Sq)
+    np.testing.assert_allclose(l_v, l_d.transpose(1, 0, 2).reshape(Hq, B * Sq), atol=1e-13)
+    g_d = attn64.attn_bwd(do, q, k, v, 0.4, causal, wl, wr, cap)
+    g_v = attn64.attn_bwd_varlen(do.reshape(B * Sq, Hq, D), q.reshape(B * Sq, Hq, D), k.reshape(B * Sk, Hkv, D),
+                                 v.reshape(B * Sk, Hkv, D), cq, ck, 0.4, causal, wl, wr, cap)
+    for a, b in zip(g_v, g_d[:3]):
+        np.testing.assert_allclose(a, b.reshape(a.shape), atol=1e-12)
+
+
+def test_varlen_sequences_do_not_see_each_other():
+    # changing one sequence's tokens leaves the other sequences' outputs and
+    # gradients unchanged (no attention across the packing boundary)
+    rng = np.random.default_rng(41)
+    cq, ck = np.array([0, 5, 5, 12]), np.array([0, 3, 9, 17])
+    q, k, v, do = _rand((12, 2, 4), rng), _rand((17, 1, 4), rng), _rand((17, 1, 4), rng), _rand((12, 2, 4), rng)
+    o1, l1 = attn64.attn_fwd_varlen(q, k, v, cq, ck, None, True)
+    g1 = attn64.attn_bwd_varlen(do, q, k, v, cq, ck, None, True)
+    k2, v2, q2 = k.copy(), v.copy(), q.copy()
+    k2[9:], v2[9:], q2[5:] = 5.0, -3.0, 2.0  # sequence 2 changed
+    o2, l2 = attn64.attn_fwd_varlen(q2, k2, v2, cq, ck, None, True)
+    g2 = attn64.attn_bwd_varlen(do, q2, k2, v2, cq, ck, None, True)
+    np.testing.assert_array_equal(o1[:5], o2[:5])
+    np.testing.assert_array_equal(l1[:, :5], l2[:, :5])
+    np.testing.assert_array_equal(g1[1][:9], g2[1][:9])
+    np.testing.assert_array_equal(g1[2][:9], g2[2][:9])
+    # sequence 1 has no queries: it contributes nothing, its keys get no gradient
+    assert np.all(g1[1][3:9] == 0) and np.all(g1[2][3:9] == 0)
+    # a packed sequence equals the same problem run alone
+    o_s, l_s = attn64.attn_fwd(q[None, 5:12], k[None, 9:17], v[None, 9:17], None, True)
+    np.testing.assert_allclose(o1[5:12], o_s[0], atol=1e-13)
+    np.testing.assert_allclose(l1[:, 5:12], l_s[0], atol=1e-13)
+
+
+def test_varlen_permuting_sequences_permutes_results():
+    rng = np.random.default_rng(42)
+    lq, lk = [4, 1, 6], [6, 3, 6]
+    seqs = [(_rand((a, 2, 4), rng), _rand((b, 2, 4), rng), _rand((b, 2, 4), rng)) for a, b in zip(lq, lk)]
+
+    def pack(order):
+        qs = np.concatenate([seqs[i][0] for i in order])
+        ks = np.concatenate([seqs[i][1] for i in order])
+        vs = np.concatenate([seqs[i][2] for i in order])
+        cq = np.concatenate([[0], np.cumsum([lq[i] for i in order])])
+        ck = np.concatenate([[0], np.cumsum([lk[i] for i in order])])
+        return attn64.attn_fwd_varlen(qs, ks, vs, cq, ck, None, True, 2, 0)
+
+    o_a, l_a = pack([0, 1, 2])
+    o_b, l_b = pack([2, 0, 1])
+    np.testing.assert_allclose(o_b[:6], o_a[5:11], atol=1e-13)   # sequence 2
+    np.testing.assert_allclose(o_b[6:10], o_a[:4], atol=1e-13)   # sequence 0
+    np.testing.assert_allclose(l_b[:, 10:], l_a[:, 4:5], atol=1e-13)  # sequence 1
+
+
+def test_varlen_backward_finite_differences():
+    rng = np.random.default_rng(43)
+    cq, ck = np.array([0, 3, 5]), np.array([0, 4, 6])
+    q, k, v, do = _rand((5, 2, 3), rng), _rand((6, 1, 3), rng), _rand((6, 1, 3), rng), _rand((5, 2, 3), rng)
+    dq, dk, dv = attn64.attn_bwd_varlen(do, q, k, v, cq, ck, 0.7, True, -1, -1, 3.0)
+
+    def loss(q_, k_, v_):
+        return float(np.sum(do * attn64.attn_fwd_varlen(q_, k_, v_, cq, ck, 0.7, True, -1, -1, 3.0)[0]))
+
+    h = 1e-6
+    for arr, grad, which in ((q, dq, 0), (k, dk, 1), (v, dv, 2)):
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            args_p = [q.copy(), k.copy(), v.copy()]
+            args_m = [q.copy(), k.copy(), v.copy()]
+            args_p[which][idx] += h
+            args_m[which][idx] -= h
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-8)
