@@ -194,6 +194,47 @@ class AttnUnit:
                 sum(t.numel() * t.element_size() for t in (self.out, self.dq, self.dk, self.dv)))
 
 
+class VarlenUnit(AttnUnit):
+    """Packed variable-length batch: forward + backward through the varlen calls."""
+
+    def __init__(self, cfg, dev):
+        from exact_attention_121_b200 import api, inputs
+        self.api = api
+        self.cfg = cfg
+        self.det = False
+        lens = cfg["lens"]
+        q, k, v, do, cu_q, cu_k = inputs.varlen_inputs(lens, lens, cfg["Hq"], cfg["Hkv"], cfg["D"], cfg["dtype"],
+                                                       seed=cfg["seed"], amp=cfg["amp"])
+        self.host_in = (q, k, v, do)
+        self.q, self.k, self.v, self.do = (t.to(dev) for t in (q, k, v, do))
+        self.cu_q, self.cu_k = cu_q.to(dev), cu_k.to(dev)
+        self.max_len = max(lens)
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty(cfg["Hq"], q.shape[0], device=dev)
+        self.dq, self.dk, self.dv = torch.empty_like(self.q), torch.empty_like(self.k), torch.empty_like(self.v)
+        n = api.fa_bwd_varlen_workspace_size(len(lens), self.max_len, q.shape[0], cfg["Hq"], cfg["D"], False)
+        self.ws = torch.empty(n, dtype=torch.uint8, device=dev)
+        pairs = sum(visible_pairs(L, L, cfg["causal"], cfg["window"][0], cfg["window"][1]) for L in lens)
+        self.flops_fwd = 4 * cfg["D"] * pairs * cfg["Hq"]
+        self.flops_bwd = 10 * cfg["D"] * pairs * cfg["Hq"]
+        self.kw = dict(scale=cfg["scale"], causal=cfg["causal"], window=cfg["window"], softcap=cfg["softcap"])
+
+    def name(self):
+        return "varlen%dxD%d" % (len(self.cfg["lens"]), self.cfg["D"])
+
+    def run(self, tracer):
+        api = self.api
+        tracer.arm("fwd", self)
+        api.fa_fwd_varlen(self.q, self.k, self.v, self.cu_q, self.cu_k, self.max_len, self.max_len, out=self.out,
+                          lse=self.lse, **self.kw)
+        n = api.fa_last_launch_count()
+        tracer.arm("bwd", self)
+        api.fa_bwd_varlen(self.do, self.q, self.k, self.v, self.out, self.lse, self.cu_q, self.cu_k, self.max_len,
+                          self.max_len, self.dq, self.dk, self.dv, workspace=self.ws, **self.kw)
+        tracer.disarm()
+        return n + api.fa_last_launch_count()
+
+
 class DecodeUnit:
     kind = "decode"
 
@@ -334,6 +375,8 @@ def build_units(dev, workload, point=None):
         units.append(DecodeUnit(inputs.paged_decode_config(), dev))
     if workload == "small":
         units.append(AttnUnit(inputs.fwd_bwd_512_config(), dev))
+    if workload == "varlen":
+        units.append(VarlenUnit(inputs.varlen_config(), dev))
     return units
 
 
@@ -475,7 +518,7 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="full", choices=["full", "sweep", "gqa", "decode", "small", "point"])
+    ap.add_argument("--workload", default="full", choices=["full", "sweep", "gqa", "decode", "small", "point", "varlen"])
     ap.add_argument("--point", default="H16D128S4096n", help="sweep point for --workload point")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -109,6 +109,79 @@ def fa_bwd(dout, q, k, v, out, lse, dq=None, dk=None, dv=None, scale=None, causa
     return dq, dk, dv
 
 
+def _cu(t, name, device):
+    if t.dtype != torch.int32 or t.dim() != 1:
+        raise ValueError(f"{name} must be a 1-D int32 tensor")
+    _check_tensor(t, name, torch.int32, device)
+
+
+def fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, out=None, lse=None,
+                  scale=None, causal=False, window=(-1, -1), softcap=0.0, stream=None):
+    """Forward attention on a packed batch: q (total_q, Hq, D), k/v (total_k,
+    Hkv, D), cu_seqlens_* (B+1) int32 device offsets.  Returns (out, lse), lse
+    fp32 (Hq, total_q)."""
+    lib = _lib.load()
+    total_q, Hq, D = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    B = cu_seqlens_q.numel() - 1
+    dt = q.dtype
+    if dt not in _DT:
+        raise ValueError(f"unsupported dtype {dt}")
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _check_tensor(t, n, dt, q.device)
+    _cu(cu_seqlens_q, "cu_seqlens_q", q.device)
+    _cu(cu_seqlens_k, "cu_seqlens_k", q.device)
+    if cu_seqlens_k.numel() != B + 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k differ in length")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    _check_tensor(lse, "lse", torch.float32, q.device)
+    wl, wr = _window(window)
+    code = lib.fa_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens_q),
+                             _ptr(cu_seqlens_k), B, int(max_seqlen_q), int(max_seqlen_k), total_q, total_k, Hq,
+                             Hkv, D, _DT[dt], float(scale or 0.0), int(bool(causal)), wl, wr,
+                             float(softcap or 0.0), _stream(stream))
+    _lib.check(code, "fa_fwd_varlen")
+    return out, lse
+
+
+def fa_bwd_varlen_workspace_size(B, max_seqlen_q, total_q, Hq, D, deterministic=False):
+    return int(_lib.load().fa_bwd_varlen_workspace_size(B, max_seqlen_q, total_q, Hq, D, int(bool(deterministic))))
+
+
+def fa_bwd_varlen(dout, q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, dq=None,
+                  dk=None, dv=None, scale=None, causal=False, window=(-1, -1), softcap=0.0, deterministic=False,
+                  workspace=None, stream=None):
+    """Backward of :func:`fa_fwd_varlen`; returns (dq, dk, dv)."""
+    lib = _lib.load()
+    total_q, Hq, D = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    B = cu_seqlens_q.numel() - 1
+    dt = q.dtype
+    for t, n in ((dout, "dout"), (q, "q"), (k, "k"), (v, "v"), (out, "out"), (dq, "dq"), (dk, "dk"),
+                 (dv, "dv")):
+        _check_tensor(t, n, dt, q.device)
+    _check_tensor(lse, "lse", torch.float32, q.device)
+    _cu(cu_seqlens_q, "cu_seqlens_q", q.device)
+    _cu(cu_seqlens_k, "cu_seqlens_k", q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = fa_bwd_varlen_workspace_size(B, max_seqlen_q, total_q, Hq, D, deterministic)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    wl, wr = _window(window)
+    code = lib.fa_bwd_varlen(_ptr(dout), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dq), _ptr(dk),
+                             _ptr(dv), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), B, int(max_seqlen_q),
+                             int(max_seqlen_k), total_q, total_k, Hq, Hkv, D, _DT[dt], float(scale or 0.0),
+                             int(bool(causal)), wl, wr, float(softcap or 0.0), int(bool(deterministic)),
+                             _ptr(workspace), workspace.numel(), _stream(stream))
+    _lib.check(code, "fa_bwd_varlen")
+    return dq, dk, dv
+
+
 def fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits):
     return int(_lib.load().fa_kvcache_workspace_size(B, Sq, Hq, D, int(num_splits)))
 

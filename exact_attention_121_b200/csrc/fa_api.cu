@@ -233,6 +233,105 @@ fa_status fa_bwd(const void* dout, const void* q, const void* k, const void* v, 
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- packed batches
+
+static fa_status check_varlen(const int* cu_q, const int* cu_k, int B, int max_q, int max_k, int total_q,
+                              int total_k) {
+  if (max_q < 0 || max_k < 0 || total_q < 0 || total_k < 0) return FA_ERR_INVALID_ARG;
+  if (B > 0 && (!cu_q || !cu_k)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_k) & 3u)) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* out, float* lse, const int* cu_seqlens_q,
+                        const int* cu_seqlens_k, int B, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                        int Hq, int Hkv, int D, fa_dtype dt, float scale, int causal, int window_left,
+                        int window_right, float softcap, fa_stream_t stream) {
+  g_last_launches = 0;
+  fa_status st = check_common(B, max_seqlen_q, Hq, Hkv, D, dt, scale, softcap);
+  if (st != FA_OK) return st;
+  st = check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q, total_k);
+  if (st != FA_OK) return st;
+  if (B == 0 || total_q == 0 || max_seqlen_q == 0) return FA_OK;
+  if (!q || !out || !lse) return FA_ERR_INVALID_ARG;
+  if (total_k > 0 && (!k || !v)) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return FA_ERR_INVALID_ARG;
+  fa::FwdParams p{};
+  p.q = q; p.k = k; p.v = v; p.o = out; p.lse = lse;
+  p.B = B; p.Sq = max_seqlen_q; p.Sk = max_seqlen_k; p.Hq = Hq; p.Hkv = Hkv; p.D = D; p.G = Hq / Hkv;
+  p.cu_q = cu_seqlens_q; p.cu_k = cu_seqlens_k; p.total_q = total_q; p.total_k = total_k;
+  fold_window(causal, window_left, window_right, &p.wl, &p.wr);
+  scale = resolve_scale(scale, D);
+  fill_cap(scale, softcap, &p.softcap, &p.cap_in, &p.cap_log2, &p.scale_log2);
+  p.status = status_ptr();
+  if (!p.status) return FA_ERR_CUDA;
+  // packed batches run on the tcgen05 kernel only
+  if (g_fwd_kernel_choice == 1 || !fa::fwd_tc_supported(p)) return FA_ERR_UNSUPPORTED;
+  int launches = 0;
+  const cudaError_t e = fa::launch_fwd_tc(p, dt, stream, &launches);
+  g_last_launches = launches;
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_bwd_varlen_workspace_size(int B, int max_seqlen_q, int total_q, int Hq, int D, int deterministic) {
+  if (B < 0 || max_seqlen_q < 0 || total_q < 0 || Hq <= 0 || (D != 64 && D != 128)) return 0;
+  size_t n = round256((size_t)total_q * Hq * D * sizeof(float));  // dQ accumulator (total_q, Hq, D)
+  n += round256((size_t)Hq * total_q * sizeof(float));              // Delta (Hq, total_q)
+  if (deterministic) n += round256(((size_t)B * Hq * fa::bwd_num_qblocks(max_seqlen_q) + 1) * sizeof(int));
+  return n;
+}
+
+fa_status fa_bwd_varlen(const void* dout, const void* q, const void* k, const void* v, const void* out,
+                        const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens_q,
+                        const int* cu_seqlens_k, int B, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                        int Hq, int Hkv, int D, fa_dtype dt, float scale, int causal, int window_left,
+                        int window_right, float softcap, int deterministic, void* workspace, size_t ws_bytes,
+                        fa_stream_t stream) {
+  g_last_launches = 0;
+  fa_status st = check_common(B, max_seqlen_q, Hq, Hkv, D, dt, scale, softcap);
+  if (st != FA_OK) return st;
+  st = check_varlen(cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q, total_k);
+  if (st != FA_OK) return st;
+  if (B == 0 || (total_q == 0 && total_k == 0)) return FA_OK;
+  const void* ptrs[] = {dout, q, k, v, out, lse, dq, dk, dv, workspace};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return FA_ERR_INVALID_ARG;
+  if (total_q > 0 && (!dout || !q || !out || !lse || !dq)) return FA_ERR_INVALID_ARG;
+  if (total_k > 0 && (!k || !v || !dk || !dv)) return FA_ERR_INVALID_ARG;
+  const size_t need = fa_bwd_varlen_workspace_size(B, max_seqlen_q, total_q, Hq, D, deterministic);
+  if (ws_bytes < need || (need > 0 && !workspace)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
+  fa::BwdParams p{};
+  p.dout = dout; p.q = q; p.k = k; p.v = v; p.o = out; p.lse = lse; p.dq = dq; p.dk = dk; p.dv = dv;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.dq_accum = reinterpret_cast<float*>(ws);
+  ws += round256((size_t)total_q * Hq * D * sizeof(float));
+  p.delta = reinterpret_cast<float*>(ws);
+  ws += round256((size_t)Hq * total_q * sizeof(float));
+  if (deterministic) {
+    p.sem = reinterpret_cast<int*>(ws);
+    p.work_counter = p.sem + (size_t)B * Hq * fa::bwd_num_qblocks(max_seqlen_q);
+  }
+  p.B = B; p.Sq = max_seqlen_q; p.Sk = max_seqlen_k; p.Hq = Hq; p.Hkv = Hkv; p.D = D; p.G = Hq / Hkv;
+  p.cu_q = cu_seqlens_q; p.cu_k = cu_seqlens_k; p.total_q = total_q; p.total_k = total_k;
+  fold_window(causal, window_left, window_right, &p.wl, &p.wr);
+  scale = resolve_scale(scale, D);
+  p.scale = scale;
+  fill_cap(scale, softcap, &p.softcap, &p.cap_in, &p.cap_log2, &p.scale_log2);
+  p.deterministic = deterministic ? 1 : 0;
+  // packed batches run on the tcgen05 kernel only
+  if (g_bwd_kernel_choice == 1) return FA_ERR_UNSUPPORTED;
+  p.kernel_choice = 2;
+  p.status = status_ptr();
+  if (!p.status) return FA_ERR_CUDA;
+  int launches = 0;
+  const cudaError_t e = fa::launch_bwd(p, dt, stream, &launches);
+  g_last_launches = launches;
+  if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 size_t fa_kvcache_workspace_size(int B, int Sq, int Hq, int D, int num_splits) {
   if (B < 0 || Sq < 0 || Hq <= 0 || (D != 64 && D != 128)) return 0;
   if (num_splits <= 0 || num_splits > FA_MAX_SPLITS) num_splits = FA_MAX_SPLITS;

@@ -39,7 +39,8 @@ template <typename T, int D>
 __global__ void bwd_preprocess_kernel(const BwdParams p, int n_sem) {
   constexpr int kLanesPerRow = D / 8;
   constexpr int kRowsPerStep = 32 / kLanesPerRow;
-  const long long rows = (long long)p.B * p.Sq * p.Hq;  // (b, i, h) order
+  // (token, h) order; a packed batch has total_q tokens
+  const long long rows = (p.cu_q ? (long long)p.total_q : (long long)p.B * p.Sq) * p.Hq;
   const int lane = threadIdx.x & 31;
   const int sub = lane / kLanesPerRow, l = lane % kLanesPerRow;
   const long long warp0 = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
@@ -76,10 +77,14 @@ __global__ void bwd_preprocess_kernel(const BwdParams p, int n_sem) {
         z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (l == 0) {
           const int h = (int)(r % p.Hq);
-          const long long bi = r / p.Hq;
-          const int i = (int)(bi % p.Sq);
-          const int b = (int)(bi / p.Sq);
-          p.delta[((size_t)b * p.Hq + h) * p.Sq + i] = acc;
+          const long long tok = r / p.Hq;
+          if (p.cu_q) {
+            p.delta[(size_t)h * p.total_q + tok] = acc;  // (Hq, total_q)
+          } else {
+            const int i = (int)(tok % p.Sq);
+            const int b = (int)(tok / p.Sq);
+            p.delta[((size_t)b * p.Hq + h) * p.Sq + i] = acc;
+          }
         }
       }
     }
@@ -377,7 +382,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_main_kernel(const BwdParam
 
 template <typename T>
 __global__ void bwd_convert_kernel(const BwdParams p) {
-  const long long n4 = (long long)p.B * p.Sq * p.Hq * p.D / 4;
+  const long long n4 = (p.cu_q ? (long long)p.total_q : (long long)p.B * p.Sq) * p.Hq * p.D / 4;
   T* dq = reinterpret_cast<T*>(p.dq);
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
     const float4 a = reinterpret_cast<const float4*>(p.dq_accum)[i];

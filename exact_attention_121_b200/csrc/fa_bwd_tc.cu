@@ -153,14 +153,17 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   }
   const int hkv = hb % p.Hkv;
   const int b = hb / p.Hkv;
-  const int off = p.Sk - p.Sq;
+  // this sequence's lengths and rows (packed batches: its own lengths)
+  const SeqView seq = seq_view(p, b);
+  const int Sq = seq.sq, Sk = seq.sk;
+  const int off = Sk - Sq;
   const int k0 = kb * kKeys;
-  const int k1 = min(k0 + kKeys, p.Sk) - 1;
-  int i_min = 0, i_max = p.Sq - 1;
+  const int k1 = min(k0 + kKeys, Sk) - 1;  // < k0: no keys of this sequence here
+  int i_min = 0, i_max = Sq - 1;
   if (p.wr >= 0) i_min = max(i_min, k0 - off - p.wr);
   if (p.wl >= 0) i_max = min(i_max, k1 - off + p.wl);
   const int qb_lo = i_min / kQ;
-  const int n_qb = (i_max >= i_min) ? (i_max / kQ - qb_lo + 1) : 0;
+  const int n_qb = (k1 >= k0 && i_max >= i_min) ? (i_max / kQ - qb_lo + 1) : 0;
   const int n_iter = n_qb * p.G;
   auto iter_q = [&](int it, int& h, int& q0) {
     h = hkv * p.G + it / n_qb;
@@ -177,8 +180,8 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         tma_prefetch_desc(&tmdO);
         mbar_expect_tx(bar(C::B_KV), 2 * C::KV_TILE);
         for (int c = 0; c < C::NCH; ++c) {
-          tma_load_4d(sb + C::OFF_K + c * C::KV_CHUNK, &tmK, c * 64, hkv, k0, b, bar(C::B_KV));
-          tma_load_4d(sb + C::OFF_V + c * C::KV_CHUNK, &tmV, c * 64, hkv, k0, b, bar(C::B_KV));
+          tma_load_4d(sb + C::OFF_K + c * C::KV_CHUNK, &tmK, c * 64, hkv, seq.ktma + k0, seq.tb, bar(C::B_KV));
+          tma_load_4d(sb + C::OFF_V + c * C::KV_CHUNK, &tmV, c * 64, hkv, seq.ktma + k0, seq.tb, bar(C::B_KV));
         }
       }
       int issued = 0;
@@ -192,12 +195,12 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         int h, q0;
         iter_q(it, h, q0);
         float* r = rows + st * 2 * kQ;
-        const float* L = p.lse + ((size_t)b * p.Hq + h) * p.Sq;
-        const float* Dl = p.delta + ((size_t)b * p.Hq + h) * p.Sq;
+        const float* L = p.lse + stat_base(p, seq, b, h);
+        const float* Dl = p.delta + stat_base(p, seq, b, h);
         for (int t = lane; t < kQ; t += 32) {
           const int q = q0 + t;
           float l2 = INFINITY, dl = 0.f;
-          if (q < p.Sq) {
+          if (q < Sq) {  // rows past the sequence: P = 0, Delta = 0
             const float l = L[q];
             l2 = (l == -INFINITY) ? INFINITY : l * kLog2e;  // stored negated below
             dl = Dl[q];
@@ -209,8 +212,9 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         if (lane == 0) {
           mbar_expect_tx(bar(C::B_QF + st), 2 * C::Q_TILE);
           for (int c = 0; c < C::NCH; ++c) {
-            tma_load_4d(sb + C::OFF_Q + st * C::Q_TILE + c * C::Q_CHUNK, &tmQ, c * 64, h, q0, b, bar(C::B_QF + st));
-            tma_load_4d(sb + C::OFF_DO + st * C::Q_TILE + c * C::Q_CHUNK, &tmdO, c * 64, h, q0, b,
+            tma_load_4d(sb + C::OFF_Q + st * C::Q_TILE + c * C::Q_CHUNK, &tmQ, c * 64, h, seq.qtma + q0, seq.tb,
+                        bar(C::B_QF + st));
+            tma_load_4d(sb + C::OFF_DO + st * C::Q_TILE + c * C::Q_CHUNK, &tmdO, c * 64, h, seq.qtma + q0, seq.tb,
                         bar(C::B_QF + st));
           }
         }
@@ -233,10 +237,11 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       constexpr uint32_t idesc_dq2 = make_idesc(kBf, 128, 2 * kQ, true, true);
       // head dim 64: dV [256,320), dK [320,384), dQ^T of a block pair [384,512)
       const uint32_t tdV = tmem + 256, tdK = tmem + (kPair ? 320 : 384);
-      auto issue_sdp = [&](int it) {
+      // S^T(it) into [0,64) of buffer it&1, dP^T(it) into [64,128)
+      auto issue_s = [&](int it) {
         const int x = it & 1, st = it % C::NQS;
         const uint32_t tb = tmem + x * 128;
-        const uint32_t q_st = sb + C::OFF_Q + st * C::Q_TILE, do_st = sb + C::OFF_DO + st * C::Q_TILE;
+        const uint32_t q_st = sb + C::OFF_Q + st * C::Q_TILE;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t okv = (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32;
@@ -244,6 +249,11 @@ __global__ void __launch_bounds__(kThreadsB, 1)
           mma_ss(tb, make_sdesc_sw128(sb + C::OFF_K + okv, 16, 1024), make_sdesc_sw128(q_st + oq, 16, 1024),
                  idesc_s, kk > 0 ? 1u : 0u);
         }
+      };
+      auto issue_dp = [&](int it) {
+        const int x = it & 1, st = it % C::NQS;
+        const uint32_t tb = tmem + x * 128;
+        const uint32_t do_st = sb + C::OFF_DO + st * C::Q_TILE;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t okv = (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32;
@@ -291,7 +301,8 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       bool ok = mbar_wait(bar(C::B_KV), 0, abort_flag, kWaitNs) && mbar_wait(bar(C::B_QF), 0, abort_flag, kWaitNs);
       if (ok) {
         tc_fence_after();
-        issue_sdp(0);
+        issue_s(0);
+        issue_dp(0);
         mma_commit(bar(C::B_SDP));
       }
       for (int it = 0; ok && it < n_iter; ++it) {
@@ -299,12 +310,18 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         if (it + 1 < n_iter) {
           const int x1 = (it + 1) & 1, u1 = (it + 1) >> 1;
           const int s1 = (it + 1) % C::NQS, v1 = (it + 1) / C::NQS;
-          // dQ^T(it-1) sits in buffer x1 at head dim 128: drained first
-          ok = mbar_wait(bar(C::B_QF + s1), v1 & 1, abort_flag, kWaitNs) &&
-               (kPair || it + 1 < 2 || mbar_wait(bar(C::B_TMF + x1), (u1 - 1) & 1, abort_flag, kWaitNs));
+          ok = mbar_wait(bar(C::B_QF + s1), v1 & 1, abort_flag, kWaitNs);
           if (!ok) break;
           tc_fence_after();
-          issue_sdp(it + 1);
+          issue_s(it + 1);
+          // head dim 128: dQ^T(it-1) sits over the dP^T columns of buffer x1
+          // (not the S^T ones): only dP^T(it+1) waits for its drain
+          if (!kPair && it + 1 >= 2) {
+            ok = mbar_wait(bar(C::B_TMF + x1), (u1 - 1) & 1, abort_flag, kWaitNs);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          issue_dp(it + 1);
           mma_commit(bar(C::B_SDP + x1));
         }
         ok = mbar_wait(bar(C::B_PDS + x), u & 1, abort_flag, kWaitNs);
@@ -358,7 +375,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       tc_fence_after();
       const uint32_t tb = tmem + lanes + x * 128;
       const float* rw = rows + (it % C::NQS) * 2 * kQ + 32 * hh;
-      const bool full = (k1 - k0 + 1 == kKeys) && (q0 + kQ <= p.Sq) &&
+      const bool full = (k1 - k0 + 1 == kKeys) && (q0 + kQ <= Sq) &&
                         (p.wl < 0 || k0 >= q0 + kQ - 1 + off - p.wl) && (p.wr < 0 || k1 <= q0 + off + p.wr);
       // This warp's 32 queries: S^T columns [32hh, 32hh+32), dP^T columns
       // [64+32hh, ...), taken in two sub-blocks of 16 queries (sb) to keep
@@ -440,8 +457,8 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       // ---- dV and dK rows of this warp's keys, head-dim half hh
       tc_fence_after();
       const size_t ks = (size_t)p.Hkv * D;
-      T* dVr = reinterpret_cast<T*>(p.dv) + ((size_t)b * p.Sk + key) * ks + (size_t)hkv * D + hh * (D / 2);
-      T* dKr = reinterpret_cast<T*>(p.dk) + ((size_t)b * p.Sk + key) * ks + (size_t)hkv * D + hh * (D / 2);
+      T* dVr = reinterpret_cast<T*>(p.dv) + (size_t)(seq.ktok + key) * ks + (size_t)hkv * D + hh * (D / 2);
+      T* dKr = reinterpret_cast<T*>(p.dk) + (size_t)(seq.ktok + key) * ks + (size_t)hkv * D + hh * (D / 2);
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const float mul = which ? p.scale : 1.f;
@@ -543,7 +560,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
             }
             fence_proxy_async_global();
           }
-          tma_reduce_add_4d(&tmDQ, 0, h, q0, b, sb + C::OFF_DQ + i * C::DQ_TILE);
+          tma_reduce_add_4d(&tmDQ, 0, h, seq.qtma + q0, seq.tb, sb + C::OFF_DQ + i * C::DQ_TILE);
           bulk_commit();
           if (sem) {
             // the additions are complete in global memory before the count moves
@@ -596,11 +613,13 @@ bool bwd_tc_supported(const BwdParams& p) {
 cudaError_t launch_bwd_main_tc(const BwdParams& p, fa_dtype dt, cudaStream_t s) {
   CUtensorMap mq, mk, mv, mdo, mdq;
   const bool bf = dt == FA_BF16;
-  if (!make_bshd_map(&mq, p.q, bf, p.D, p.Hq, p.Sq, p.B, kQ) ||
-      !make_bshd_map(&mdo, p.dout, bf, p.D, p.Hq, p.Sq, p.B, kQ) ||
-      !make_bshd_map(&mk, p.k, bf, p.D, p.Hkv, p.Sk, p.B, kKeys) ||
-      !make_bshd_map(&mv, p.v, bf, p.D, p.Hkv, p.Sk, p.B, kKeys) ||
-      !make_bshd_map_f32(&mdq, p.dq_accum, p.D, p.Hq, p.Sq, p.B, kQ))
+  // a packed batch is one batch of total_q / total_k token rows
+  const int mq_s = p.cu_q ? p.total_q : p.Sq, mk_s = p.cu_q ? p.total_k : p.Sk, mb = p.cu_q ? 1 : p.B;
+  if (!make_bshd_map(&mq, p.q, bf, p.D, p.Hq, mq_s, mb, kQ) ||
+      !make_bshd_map(&mdo, p.dout, bf, p.D, p.Hq, mq_s, mb, kQ) ||
+      !make_bshd_map(&mk, p.k, bf, p.D, p.Hkv, mk_s, mb, kKeys) ||
+      !make_bshd_map(&mv, p.v, bf, p.D, p.Hkv, mk_s, mb, kKeys) ||
+      !make_bshd_map_f32(&mdq, p.dq_accum, p.D, p.Hq, mq_s, mb, kQ))
     return cudaErrorNotSupported;
   const bool cap = p.softcap > 0.f;
   if (p.D == 64) {

@@ -217,6 +217,51 @@ __device__ __forceinline__ void group_order(int L, int n_items, int n_heads, boo
   item = reverse ? n_items - 1 - rank : rank;
 }
 
+// Where sequence b of a batch lives.  Dense batches: every sequence has Sq
+// query and Sk key rows, token row t of sequence b is b*S + t and the TMA
+// batch coordinate is b.  Packed (variable-length) batches: lengths and first
+// rows come from the cu_seqlens offsets, and the TMA maps cover all tokens as
+// a single batch.
+struct SeqView {
+  int sq, sk;              // query / key rows of the sequence
+  long long qtok, ktok;    // token index of its first query / key row
+  int qtma, ktma, tb;      // TMA row offset of the sequence, TMA batch coordinate
+};
+template <class P>
+__device__ __forceinline__ SeqView seq_view(const P& p, int b) {
+  SeqView v;
+  if (p.cu_q) {
+    // offsets outside [0, total] or lengths above the stated maxima are the
+    // caller's error: clamp them so every access stays inside the tensors,
+    // and record FA_ERR_INVALID_ARG in the status word
+    const int a0 = p.cu_q[b], a1 = p.cu_q[b + 1], c0 = p.cu_k[b], c1 = p.cu_k[b + 1];
+    const int q0 = min(max(a0, 0), p.total_q), k0 = min(max(c0, 0), p.total_k);
+    v.sq = min(min(max(a1, q0), p.total_q) - q0, p.Sq);
+    v.sk = min(min(max(c1, k0), p.total_k) - k0, p.Sk);
+    if (q0 != a0 || k0 != c0 || v.sq != a1 - a0 || v.sk != c1 - c0) report_status(p.status, kStatusBadArg);
+    v.qtok = q0;
+    v.ktok = k0;
+    v.qtma = q0;
+    v.ktma = k0;
+    v.tb = 0;
+  } else {
+    v.sq = p.Sq;
+    v.sk = p.Sk;
+    v.qtok = (long long)b * p.Sq;
+    v.ktok = (long long)b * p.Sk;
+    v.qtma = 0;
+    v.ktma = 0;
+    v.tb = b;
+  }
+  return v;
+}
+// Offset of the row statistics (LSE, Delta) of (b, h): dense layout
+// (B, Hq, Sq), packed layout (Hq, total_q).
+template <class P>
+__device__ __forceinline__ long long stat_base(const P& p, const SeqView& v, int b, int h) {
+  return p.cu_q ? (long long)h * p.total_q + v.qtok : ((long long)b * p.Hq + h) * p.Sq;
+}
+
 // max(a, b, c) in one instruction (three-operand form, sm_100 and later).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;

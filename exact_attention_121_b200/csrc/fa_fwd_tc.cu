@@ -116,9 +116,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   const int b = hb / p.Hq;
   const int g = h / p.G;
   const int q0 = qp * 2 * kRows;
-  const int off = p.Sk - p.Sq;
-  const int qlast = min(q0 + 2 * kRows, p.Sq) - 1;
-  int kmin = 0, kmax = p.Sk - 1;
+  // this sequence's lengths and rows (packed batches: its own lengths)
+  const SeqView seq = seq_view(p, b);
+  const int Sq = seq.sq, Sk = seq.sk;
+  if (q0 >= Sq) return;  // a shorter sequence of a packed batch: no rows here
+  const int off = Sk - Sq;
+  const int qlast = min(q0 + 2 * kRows, Sq) - 1;
+  int kmin = 0, kmax = Sk - 1;
   if (p.wl >= 0) kmin = max(kmin, q0 + off - p.wl);
   if (p.wr >= 0) kmax = min(kmax, qlast + off + p.wr);
   const int kt_begin = kmin / kRows;
@@ -168,7 +172,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       mbar_expect_tx(bar(C::B_Q), 2 * C::TILE);
       for (int t = 0; t < 2; ++t)
         for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_4d(sb + C::OFF_Q + t * C::TILE + c * C::CHUNK, &tmQ, c * 64, h, q0 + t * kRows, b, bar(C::B_Q));
+          tma_load_4d(sb + C::OFF_Q + t * C::TILE + c * C::CHUNK, &tmQ, c * 64, h, seq.qtma + q0 + t * kRows, seq.tb,
+                      bar(C::B_Q));
       int issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
         const int sk = j % C::NSK, uk = j / C::NSK;
@@ -180,7 +185,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
         mbar_expect_tx(bar(C::B_KF + sk), C::TILE);
         for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_4d(sb + C::OFF_K + sk * C::TILE + c * C::CHUNK, &tmK, c * 64, g, k0, b, bar(C::B_KF + sk));
+          tma_load_4d(sb + C::OFF_K + sk * C::TILE + c * C::CHUNK, &tmK, c * 64, g, seq.ktma + k0, seq.tb,
+                      bar(C::B_KF + sk));
         if (j >= C::NSV && !mbar_wait(bar(C::B_VE + sv), (uv - 1) & 1, abort_flag, kTcWaitNs)) {
           fail();
           issued = -(j + 1);  // K of tile j is in flight, V is not
@@ -188,7 +194,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
         mbar_expect_tx(bar(C::B_VF + sv), C::TILE);
         for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_4d(sb + C::OFF_V + sv * C::TILE + c * C::CHUNK, &tmV, c * 64, g, k0, b, bar(C::B_VF + sv));
+          tma_load_4d(sb + C::OFF_V + sv * C::TILE + c * C::CHUNK, &tmV, c * 64, g, seq.ktma + k0, seq.tb,
+                      bar(C::B_VF + sv));
         issued = j + 1;
       }
       if (*abort_flag) {
@@ -346,7 +353,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         mbar_arrive(bar(C::B_SF + t));
       }
       const int k0 = (kt_begin + j) * kRows;
-      const bool full = (k0 + kRows <= p.Sk) && (p.wl < 0 || k0 >= qpos_last - p.wl) &&
+      const bool full = (k0 + kRows <= Sk) && (p.wl < 0 || k0 >= qpos_last - p.wl) &&
                         (p.wr < 0 || k0 + kRows - 1 <= qpos_first + p.wr);
       // row maximum in the log2 domain (the scale is positive: max commutes)
       float mx = -INFINITY;
@@ -358,7 +365,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 #pragma unroll
         for (int i = 0; i < kRows; ++i) {
           const int key = k0 + i;
-          const bool vis = key < p.Sk && (p.wl < 0 || key >= qpos - p.wl) && (p.wr < 0 || key <= qpos + p.wr);
+          const bool vis = key < Sk && (p.wl < 0 || key >= qpos - p.wl) && (p.wr < 0 || key <= qpos + p.wr);
           if (!vis) s[i] = __float_as_uint(-INFINITY);
         }
       }
@@ -452,7 +459,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       // ---- epilogue: O / l in 16 bits, LSE
       tc_fence_after();
       const float inv = l_q > 0.f ? 1.f / l_q : 0.f;
-      T* orow = reinterpret_cast<T*>(p.o) + (((size_t)b * p.Sq + qi) * p.Hq + h) * D;
+      T* orow = reinterpret_cast<T*>(p.o) + ((size_t)(seq.qtok + qi) * p.Hq + h) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t u[32];
@@ -464,7 +471,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) u[i] = 0u;
         }
-        if (qi < p.Sq) {
+        if (qi < Sq) {
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4) {
             uint4 w;
@@ -476,8 +483,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           }
         }
       }
-      if (qi < p.Sq)
-        p.lse[((size_t)b * p.Hq + h) * p.Sq + qi] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+      if (qi < Sq)
+        p.lse[stat_base(p, seq, b, h) + qi] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
     }
   }
 
@@ -526,8 +533,10 @@ bool fwd_tc_supported(const FwdParams& p) {
 cudaError_t launch_fwd_tc(const FwdParams& p, fa_dtype dt, cudaStream_t s, int* launches) {
   CUtensorMap mq, mk, mv;
   const bool bf = dt == FA_BF16;
-  if (!make_bshd_map(&mq, p.q, bf, p.D, p.Hq, p.Sq, p.B, 128) || !make_bshd_map(&mk, p.k, bf, p.D, p.Hkv, p.Sk, p.B, 128) ||
-      !make_bshd_map(&mv, p.v, bf, p.D, p.Hkv, p.Sk, p.B, 128))
+  // a packed batch is one batch of total_q / total_k token rows
+  const int mq_s = p.cu_q ? p.total_q : p.Sq, mk_s = p.cu_q ? p.total_k : p.Sk, mb = p.cu_q ? 1 : p.B;
+  if (!make_bshd_map(&mq, p.q, bf, p.D, p.Hq, mq_s, mb, 128) || !make_bshd_map(&mk, p.k, bf, p.D, p.Hkv, mk_s, mb, 128) ||
+      !make_bshd_map(&mv, p.v, bf, p.D, p.Hkv, mk_s, mb, 128))
     return cudaErrorNotSupported;
   cudaError_t e = bf ? launch_dt<__nv_bfloat16>(p, mq, mk, mv, s) : launch_dt<__half>(p, mq, mk, mv, s);
   if (e == cudaSuccess) ++*launches;

@@ -24,6 +24,11 @@ struct FwdParams {
   float cap_in;          // scale / softcap: raw dot product -> tanh argument
   float cap_log2;        // softcap * log2(e)
   int* status;           // device status word
+  // packed variable-length batch: (B+1) token offsets, else null; Sq/Sk are
+  // then the longest sequence and total_q the packed query tokens
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;
 };
 
 struct BwdParams {
@@ -48,6 +53,11 @@ struct BwdParams {
   int deterministic;
   int kernel_choice;     // 0 automatic, 1 mma.sync main kernel, 2 tcgen05 main kernel
   int* status;
+  // packed variable-length batch (see FwdParams); dq_accum is then
+  // (total_q, Hq, D) and delta (Hq, total_q)
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;
 };
 
 struct DecodeParams {

@@ -124,3 +124,32 @@ def paged_decode_config():
     return dict(B=8, Hq=32, Hkv=8, D=128, dtype="bf16", page_size=256, pages_per_seq=129,
                 max_len=32768, Sq=1, Snew=1, causal=True, seed=5,
                 scale=1.0 / math.sqrt(128))
+
+
+def varlen_lengths(B, min_len, max_len, seed):
+    """B sequence lengths drawn U{min_len..max_len} (a packed batch's mix)."""
+    g = _gen(seed)
+    return torch.randint(min_len, max_len + 1, (B,), generator=g).tolist()
+
+
+def varlen_inputs(lens_q, lens_k, Hq, Hkv, D, dtype="bf16", seed=0, amp=1.0):
+    """Packed (q, k, v, dout) host tensors (total, nheads, headdim) and the
+    (B+1) int32 cu_seqlens offsets of the query and key sequences."""
+    dt = DTYPES[dtype] if isinstance(dtype, str) else dtype
+    g = _gen(seed)
+    tq, tk = int(sum(lens_q)), int(sum(lens_k))
+    q = randn((tq, Hq, D), g, dt, amp)
+    k = randn((tk, Hkv, D), g, dt, amp)
+    v = randn((tk, Hkv, D), g, dt, amp)
+    dout = randn((tq, Hq, D), g, dt, amp)
+    cu_q = torch.tensor([0] + list(torch.tensor(lens_q).cumsum(0).tolist()), dtype=torch.int32)
+    cu_k = torch.tensor([0] + list(torch.tensor(lens_k).cumsum(0).tolist()), dtype=torch.int32)
+    return q, k, v, dout, cu_q, cu_k
+
+
+def varlen_config():
+    """Packed training batch at hidden 2048 (Hq=Hkv=16, D=128, bf16, causal):
+    32 sequences with lengths U{64..1024} (seed 6), as a document-packing mix."""
+    lens = varlen_lengths(32, 64, 1024, seed=6)
+    return dict(lens=lens, Hq=16, Hkv=16, D=128, dtype="bf16", causal=True, window=(-1, -1), softcap=0.0,
+                scale=1.0 / math.sqrt(128), seed=7, amp=1.0)

@@ -109,6 +109,53 @@ fa_status fa_bwd(const void* dout, const void* q, const void* k, const void* v,
                  float scale, int causal, int window_left, int window_right, float softcap,
                  int deterministic, void* workspace, size_t ws_bytes, fa_stream_t stream);
 
+/*
+ * Forward attention on a packed batch of variable-length sequences (the
+ * pages' "varlen" variant).  The B sequences are concatenated along the token
+ * axis:
+ *   q   (total_q, Hq, D)  16-bit, read;  k, v (total_k, Hkv, D) 16-bit, read
+ *   out (total_q, Hq, D)  16-bit, written
+ *   lse (Hq, total_q)     float32, written
+ *   cu_seqlens_q, cu_seqlens_k: (B+1) int32 device offsets, cu[0] = 0,
+ *     non-decreasing, cu[B] = total; sequence b owns query tokens
+ *     cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 and key tokens likewise.
+ *   max_seqlen_q / max_seqlen_k: upper bounds of the sequence lengths (they
+ *     size the grid).
+ * Each sequence is attended on its own, masks and bottom-right alignment
+ * taken from its own lengths (causal: query i of a sequence with Sq_b
+ * queries and Sk_b keys sees keys j <= i + Sk_b - Sq_b).  A sequence with no
+ * keys gets O = 0 and LSE = -inf.  Offsets that do not satisfy the contract
+ * are clamped on the device (no access leaves the tensors) and record
+ * FA_ERR_INVALID_ARG in the device status word.  Runs on the tcgen05 kernel
+ * only: FA_ERR_UNSUPPORTED where it is not available or the mma.sync kernel
+ * was selected.  Pointers are device pointers the caller owns.
+ */
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
+                        const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int max_seqlen_q,
+                        int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, int D, fa_dtype dt,
+                        float scale, int causal, int window_left, int window_right, float softcap,
+                        fa_stream_t stream);
+
+/*
+ * Workspace of fa_bwd_varlen: the float32 dQ accumulator (total_q, Hq, D),
+ * Delta (Hq, total_q) and, when deterministic, one ordering counter per
+ * (sequence, q-head, 64-row query block of max_seqlen_q) plus a work counter.
+ */
+size_t fa_bwd_varlen_workspace_size(int B, int max_seqlen_q, int total_q, int Hq, int D, int deterministic);
+
+/*
+ * Backward of fa_fwd_varlen (same packed layouts; lse from fa_fwd_varlen with
+ * the same arguments).  dq (total_q, Hq, D), dk, dv (total_k, Hkv, D) written.
+ * workspace >= fa_bwd_varlen_workspace_size(...) bytes, 256-byte aligned.
+ * max_seqlen_k >= 1.  deterministic as in fa_bwd.  tcgen05 kernel only.
+ */
+fa_status fa_bwd_varlen(const void* dout, const void* q, const void* k, const void* v,
+                        const void* out, const float* lse, void* dq, void* dk, void* dv,
+                        const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int max_seqlen_q,
+                        int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, int D, fa_dtype dt,
+                        float scale, int causal, int window_left, int window_right, float softcap,
+                        int deterministic, void* workspace, size_t ws_bytes, fa_stream_t stream);
+
 /* Largest split count fa_fwd_kvcache accepts; num_splits <= 0 picks one. */
 #define FA_MAX_SPLITS 64
 

@@ -450,8 +450,8 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale=None, causal=Fals
     lse = np.full((Hq, q.shape[0]), NEG_INF)
     for b in range(len(cq) - 1):
         q0, q1, k0, k1 = int(cq[b]), int(cq[b + 1]), int(ck[b]), int(ck[b + 1])
-        if q1 == q0:
-            continue
+        if q1 == q0 or k1 == k0:
+            continue  # no queries, or no keys: rows stay O = 0, LSE = -inf
         o_b, l_b = attn_fwd(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1], scale, causal, window_left,
                             window_right, softcap)
         out[q0:q1] = o_b[0]

@@ -508,3 +508,15 @@ def test_varlen_backward_finite_differences():
             args_m[which][idx] -= h
             num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
         np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-8)
+
+
+def test_varlen_sequence_without_keys():
+    rng = np.random.default_rng(44)
+    cq, ck = np.array([0, 3, 7]), np.array([0, 0, 5])
+    q, k, v = _rand((7, 2, 4), rng), _rand((5, 1, 4), rng), _rand((5, 1, 4), rng)
+    o, l = attn64.attn_fwd_varlen(q, k, v, cq, ck)
+    assert np.all(o[:3] == 0) and np.all(l[:, :3] == -np.inf)
+    o_s, l_s = attn64.attn_fwd(q[None, 3:], k[None], v[None])
+    np.testing.assert_allclose(o[3:], o_s[0], atol=1e-13)
+    dq, dk, dv = attn64.attn_bwd_varlen(_rand((7, 2, 4), rng), q, k, v, cq, ck)
+    assert np.all(dq[:3] == 0)
