@@ -44,6 +44,7 @@ ROOFLINE_UNIT = {"fwd": "H16D128S4096n", "bwd": "H16D128S4096n", "decode": "deco
 # entry must be removed whenever its kernel changes.
 TRAFFIC_PER_LAUNCH = {
     ("fwd", "H16D128S4096n"): 201.683712e6 + 51.086592e6,
+    ("bwd", "H16D128S4096n"): 416.537088e6 + 236.700928e6,
     ("decode", "decode"): 521.946368e6 + 7.995904e6,
 }
 
