@@ -24,12 +24,15 @@ def _stream(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def _check_tensor(t, name, dtype=None, device=None):
+def _check_tensor(t, name, dtype=None, device=None, strided=False):
     if t is None:
         return
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
-    if not t.is_contiguous():
+    if strided:
+        if t.dim() != 4 or t.stride(3) != 1:
+            raise ValueError(f"{name} must be (B, S, H, D) with a contiguous last dimension")
+    elif not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
@@ -55,9 +58,19 @@ def fa_last_launch_count():
     return int(_lib.load().fa_last_launch_count())
 
 
+def _stride_array(tensors):
+    """(batch, token, head) element strides of (B, S, H, D) tensors, as int64."""
+    vals = [int(x) for t in tensors for x in t.stride()[:3]]
+    return (ctypes.c_longlong * len(vals))(*vals)
+
+
 def fa_fwd(q, k, v, out=None, lse=None, scale=None, causal=False, window=(-1, -1), softcap=0.0,
            stream=None):
-    """Forward attention; returns (out, lse).  lse is fp32 (B, Hq, Sq)."""
+    """Forward attention; returns (out, lse).  lse is fp32 (B, Hq, Sq).
+
+    q, k, v (and out) may be views with any strides as long as the head
+    dimension is contiguous (e.g. slices of a packed qkv tensor); those go
+    through fa_fwd_strided."""
     lib = _lib.load()
     B, Sq, Hq, D = q.shape
     Sk, Hkv = k.shape[1], k.shape[2]
@@ -65,17 +78,21 @@ def fa_fwd(q, k, v, out=None, lse=None, scale=None, causal=False, window=(-1, -1
     if dt not in _DT:
         raise ValueError(f"unsupported dtype {dt}")
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
-        _check_tensor(t, n, dt, q.device)
+        _check_tensor(t, n, dt, q.device, strided=True)
     if out is None:
-        out = torch.empty_like(q)
+        out = torch.empty(q.shape, dtype=dt, device=q.device)
     if lse is None:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
     _check_tensor(lse, "lse", torch.float32, q.device)
     wl, wr = _window(window)
-    code = lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq, Sk, Hq, Hkv, D, _DT[dt],
-                      float(scale or 0.0), int(bool(causal)), wl, wr, float(softcap or 0.0),
-                      _stream(stream))
-    _lib.check(code, "fa_fwd")
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq, Sk, Hq, Hkv, D, _DT[dt], float(scale or 0.0),
+            int(bool(causal)), wl, wr, float(softcap or 0.0))
+    if all(t.is_contiguous() for t in (q, k, v, out)):
+        code = lib.fa_fwd(*args, _stream(stream))
+        _lib.check(code, "fa_fwd")
+    else:
+        code = lib.fa_fwd_strided(*args, _stride_array((q, k, v, out)), _stream(stream))
+        _lib.check(code, "fa_fwd_strided")
     return out, lse
 
 
@@ -92,21 +109,41 @@ def fa_bwd(dout, q, k, v, out, lse, dq=None, dk=None, dv=None, scale=None, causa
     dt = q.dtype
     for t, n in ((dout, "dout"), (q, "q"), (k, "k"), (v, "v"), (out, "out"), (dq, "dq"), (dk, "dk"),
                  (dv, "dv")):
-        _check_tensor(t, n, dt, q.device)
+        _check_tensor(t, n, dt, q.device, strided=True)
     _check_tensor(lse, "lse", torch.float32, q.device)
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
+    dq = torch.empty(q.shape, dtype=dt, device=q.device) if dq is None else dq
+    dk = torch.empty(k.shape, dtype=dt, device=q.device) if dk is None else dk
+    dv = torch.empty(v.shape, dtype=dt, device=q.device) if dv is None else dv
     need = fa_bwd_workspace_size(B, Sq, Sk, Hq, Hkv, D, deterministic)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     wl, wr = _window(window)
-    code = lib.fa_bwd(_ptr(dout), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dq), _ptr(dk),
-                      _ptr(dv), B, Sq, Sk, Hq, Hkv, D, _DT[dt], float(scale or 0.0),
-                      int(bool(causal)), wl, wr, float(softcap or 0.0), int(bool(deterministic)),
-                      _ptr(workspace), workspace.numel(), _stream(stream))
-    _lib.check(code, "fa_bwd")
+    args = (_ptr(dout), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), B, Sq, Sk,
+            Hq, Hkv, D, _DT[dt], float(scale or 0.0), int(bool(causal)), wl, wr, float(softcap or 0.0),
+            int(bool(deterministic)), _ptr(workspace), workspace.numel())
+    tensors = (dout, q, k, v, out, dq, dk, dv)
+    if all(t.is_contiguous() for t in tensors):
+        code = lib.fa_bwd(*args, _stream(stream))
+        _lib.check(code, "fa_bwd")
+    else:
+        code = lib.fa_bwd_strided(*args, _stride_array(tensors), _stream(stream))
+        _lib.check(code, "fa_bwd_strided")
     return dq, dk, dv
+
+
+def fa_fwd_qkvpacked(qkv, **kw):
+    """Forward attention on a packed (B, S, 3, H, D) tensor; returns (out, lse)."""
+    q, k, v = qkv.unbind(2)
+    return fa_fwd(q, k, v, **kw)
+
+
+def fa_bwd_qkvpacked(dout, qkv, out, lse, dqkv=None, **kw):
+    """Backward of :func:`fa_fwd_qkvpacked`; returns dqkv (B, S, 3, H, D)."""
+    q, k, v = qkv.unbind(2)
+    dqkv = torch.empty_like(qkv) if dqkv is None else dqkv
+    dq, dk, dv = dqkv.unbind(2)
+    fa_bwd(dout, q, k, v, out, lse, dq=dq, dk=dk, dv=dv, **kw)
+    return dqkv
 
 
 def _cu(t, name, device):

@@ -149,9 +149,23 @@ void fa_set_bwd_kernel(int which) { g_bwd_kernel_choice = which; }
 
 int fa_last_launch_count(void) { return g_last_launches; }
 
-fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk,
-                 int Hq, int Hkv, int D, fa_dtype dt, float scale, int causal, int window_left, int window_right,
-                 float softcap, fa_stream_t stream) {
+// (batch, token, head) element strides of a packed (B, S, H, D) tensor
+static void contiguous_strides(long long st[3], int S, int H, int D) {
+  st[0] = (long long)S * H * D;
+  st[1] = (long long)H * D;
+  st[2] = D;
+}
+// user strides: non-negative multiples of 8 elements (16-byte rows for TMA)
+static bool strides_ok(const long long* st, int n) {
+  for (int i = 0; i < n; ++i)
+    if (st[i] < 0 || st[i] % 8 != 0) return false;
+  return true;
+}
+
+// strides: NULL (packed tensors) or 12 values, (batch, token, head) of q, k, v, out
+static fa_status fwd_impl(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk,
+                          int Hq, int Hkv, int D, fa_dtype dt, float scale, int causal, int window_left,
+                          int window_right, float softcap, const long long* strides, fa_stream_t stream) {
   g_last_launches = 0;
   fa_status st = check_common(B, Sq, Hq, Hkv, D, dt, scale, softcap);
   if (st != FA_OK) return st;
@@ -161,9 +175,19 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* 
   if (Sk > 0 && (!k || !v)) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
     return FA_ERR_INVALID_ARG;
+  if (strides && !strides_ok(strides, 12)) return FA_ERR_INVALID_ARG;
   fa::FwdParams p{};
   p.q = q; p.k = k; p.v = v; p.o = out; p.lse = lse;
   p.B = B; p.Sq = Sq; p.Sk = Sk; p.Hq = Hq; p.Hkv = Hkv; p.D = D; p.G = Hq / Hkv;
+  contiguous_strides(p.st_q, Sq, Hq, D);
+  contiguous_strides(p.st_k, Sk, Hkv, D);
+  contiguous_strides(p.st_v, Sk, Hkv, D);
+  contiguous_strides(p.st_o, Sq, Hq, D);
+  if (strides) {
+    long long* dst[4] = {p.st_q, p.st_k, p.st_v, p.st_o};
+    for (int t = 0; t < 4; ++t)
+      for (int i = 0; i < 3; ++i) dst[t][i] = strides[3 * t + i];
+  }
   fold_window(causal, window_left, window_right, &p.wl, &p.wr);
   scale = resolve_scale(scale, D);
   fill_cap(scale, softcap, &p.softcap, &p.cap_in, &p.cap_log2, &p.scale_log2);
@@ -171,15 +195,32 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* 
   if (!p.status) return FA_ERR_CUDA;
   int launches = 0;
   cudaError_t e;
-  const bool tc = (g_fwd_kernel_choice == 2) || (g_fwd_kernel_choice == 0 && kTcAuto);
+  // strided tensors run on the tcgen05 kernel only
+  const bool tc = (g_fwd_kernel_choice == 2) || (g_fwd_kernel_choice == 0 && kTcAuto) || strides;
   if (tc && fa::fwd_tc_supported(p)) {
     e = fa::launch_fwd_tc(p, dt, stream, &launches);
   } else {
-    if (g_fwd_kernel_choice == 2) return FA_ERR_UNSUPPORTED;
+    if (g_fwd_kernel_choice == 2 || strides) return FA_ERR_UNSUPPORTED;
     e = fa::launch_fwd_mma(p, dt, stream, &launches);
   }
   g_last_launches = launches;
+  if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk,
+                 int Hq, int Hkv, int D, fa_dtype dt, float scale, int causal, int window_left, int window_right,
+                 float softcap, fa_stream_t stream) {
+  return fwd_impl(q, k, v, out, lse, B, Sq, Sk, Hq, Hkv, D, dt, scale, causal, window_left, window_right, softcap,
+                  nullptr, stream);
+}
+
+fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk,
+                         int Hq, int Hkv, int D, fa_dtype dt, float scale, int causal, int window_left,
+                         int window_right, float softcap, const long long* strides, fa_stream_t stream) {
+  if (!strides) return FA_ERR_INVALID_ARG;
+  return fwd_impl(q, k, v, out, lse, B, Sq, Sk, Hq, Hkv, D, dt, scale, causal, window_left, window_right, softcap,
+                  strides, stream);
 }
 
 size_t fa_bwd_workspace_size(int B, int Sq, int Sk, int Hq, int Hkv, int D, int deterministic) {
@@ -190,10 +231,13 @@ size_t fa_bwd_workspace_size(int B, int Sq, int Sk, int Hq, int Hkv, int D, int 
   return n;
 }
 
-fa_status fa_bwd(const void* dout, const void* q, const void* k, const void* v, const void* out, const float* lse,
-                 void* dq, void* dk, void* dv, int B, int Sq, int Sk, int Hq, int Hkv, int D, fa_dtype dt,
-                 float scale, int causal, int window_left, int window_right, float softcap, int deterministic,
-                 void* workspace, size_t ws_bytes, fa_stream_t stream) {
+// strides: NULL (packed tensors) or 24 values, (batch, token, head) of dout,
+// q, k, v, out, dq, dk, dv
+static fa_status bwd_impl(const void* dout, const void* q, const void* k, const void* v, const void* out,
+                          const float* lse, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int Hq, int Hkv,
+                          int D, fa_dtype dt, float scale, int causal, int window_left, int window_right,
+                          float softcap, int deterministic, void* workspace, size_t ws_bytes,
+                          const long long* strides, fa_stream_t stream) {
   g_last_launches = 0;
   fa_status st = check_common(B, Sq, Hq, Hkv, D, dt, scale, softcap);
   if (st != FA_OK) return st;
@@ -219,18 +263,61 @@ fa_status fa_bwd(const void* dout, const void* q, const void* k, const void* v, 
     p.work_counter = p.sem + (size_t)B * Hq * fa::bwd_num_qblocks(Sq);
   }
   p.B = B; p.Sq = Sq; p.Sk = Sk; p.Hq = Hq; p.Hkv = Hkv; p.D = D; p.G = Hq / Hkv;
+  if (strides && !strides_ok(strides, 24)) return FA_ERR_INVALID_ARG;
+  if ((long long)B * Sq * Hq >= (1LL << 31)) return FA_ERR_UNSUPPORTED;  // row index of the dQ accumulator
+  {
+    long long* dst[8] = {p.st_do, p.st_q, p.st_k, p.st_v, p.st_o, p.st_dq, p.st_dk, p.st_dv};
+    const bool is_q[8] = {true, true, false, false, true, true, false, false};
+    for (int t = 0; t < 8; ++t) {
+      if (strides)
+        for (int i = 0; i < 3; ++i) dst[t][i] = strides[3 * t + i];
+      else
+        contiguous_strides(dst[t], is_q[t] ? Sq : Sk, is_q[t] ? Hq : Hkv, D);
+    }
+  }
+  {
+    long long c[3];
+    contiguous_strides(c, Sq, Hq, D);
+    p.rows_packed = 1;
+    for (const long long* st : {p.st_do, p.st_o, p.st_dq})
+      if (st[0] != c[0] || st[1] != c[1] || st[2] != c[2]) p.rows_packed = 0;
+  }
   fold_window(causal, window_left, window_right, &p.wl, &p.wr);
   scale = resolve_scale(scale, D);
   p.scale = scale;
   fill_cap(scale, softcap, &p.softcap, &p.cap_in, &p.cap_log2, &p.scale_log2);
   p.deterministic = deterministic ? 1 : 0;
   p.kernel_choice = g_bwd_kernel_choice;
+  // strided tensors run on the tcgen05 kernel only
+  if (strides) {
+    if (g_bwd_kernel_choice == 1) return FA_ERR_UNSUPPORTED;
+    p.kernel_choice = 2;
+  }
   p.status = status_ptr();
   if (!p.status) return FA_ERR_CUDA;
   int launches = 0;
   cudaError_t e = fa::launch_bwd(p, dt, stream, &launches);
   g_last_launches = launches;
+  if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_bwd(const void* dout, const void* q, const void* k, const void* v, const void* out, const float* lse,
+                 void* dq, void* dk, void* dv, int B, int Sq, int Sk, int Hq, int Hkv, int D, fa_dtype dt,
+                 float scale, int causal, int window_left, int window_right, float softcap, int deterministic,
+                 void* workspace, size_t ws_bytes, fa_stream_t stream) {
+  return bwd_impl(dout, q, k, v, out, lse, dq, dk, dv, B, Sq, Sk, Hq, Hkv, D, dt, scale, causal, window_left,
+                  window_right, softcap, deterministic, workspace, ws_bytes, nullptr, stream);
+}
+
+fa_status fa_bwd_strided(const void* dout, const void* q, const void* k, const void* v, const void* out,
+                         const float* lse, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int Hq, int Hkv,
+                         int D, fa_dtype dt, float scale, int causal, int window_left, int window_right,
+                         float softcap, int deterministic, void* workspace, size_t ws_bytes,
+                         const long long* strides, fa_stream_t stream) {
+  if (!strides) return FA_ERR_INVALID_ARG;
+  return bwd_impl(dout, q, k, v, out, lse, dq, dk, dv, B, Sq, Sk, Hq, Hkv, D, dt, scale, causal, window_left,
+                  window_right, softcap, deterministic, workspace, ws_bytes, strides, stream);
 }
 
 // ---------------------------------------------------------------- packed batches
@@ -261,6 +348,9 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* out, 
   p.q = q; p.k = k; p.v = v; p.o = out; p.lse = lse;
   p.B = B; p.Sq = max_seqlen_q; p.Sk = max_seqlen_k; p.Hq = Hq; p.Hkv = Hkv; p.D = D; p.G = Hq / Hkv;
   p.cu_q = cu_seqlens_q; p.cu_k = cu_seqlens_k; p.total_q = total_q; p.total_k = total_k;
+  // packed tensors: one batch of tokens (batch stride 0)
+  for (long long* st : {p.st_q, p.st_o}) { st[0] = 0; st[1] = (long long)Hq * D; st[2] = D; }
+  for (long long* st : {p.st_k, p.st_v}) { st[0] = 0; st[1] = (long long)Hkv * D; st[2] = D; }
   fold_window(causal, window_left, window_right, &p.wl, &p.wr);
   scale = resolve_scale(scale, D);
   fill_cap(scale, softcap, &p.softcap, &p.cap_in, &p.cap_log2, &p.scale_log2);
@@ -299,6 +389,7 @@ fa_status fa_bwd_varlen(const void* dout, const void* q, const void* k, const vo
     if (!aligned16(ptr)) return FA_ERR_INVALID_ARG;
   if (total_q > 0 && (!dout || !q || !out || !lse || !dq)) return FA_ERR_INVALID_ARG;
   if (total_k > 0 && (!k || !v || !dk || !dv)) return FA_ERR_INVALID_ARG;
+  if ((long long)total_q * Hq >= (1LL << 31)) return FA_ERR_UNSUPPORTED;  // row index of the dQ accumulator
   const size_t need = fa_bwd_varlen_workspace_size(B, max_seqlen_q, total_q, Hq, D, deterministic);
   if (ws_bytes < need || (need > 0 && !workspace)) return FA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
@@ -315,6 +406,10 @@ fa_status fa_bwd_varlen(const void* dout, const void* q, const void* k, const vo
   }
   p.B = B; p.Sq = max_seqlen_q; p.Sk = max_seqlen_k; p.Hq = Hq; p.Hkv = Hkv; p.D = D; p.G = Hq / Hkv;
   p.cu_q = cu_seqlens_q; p.cu_k = cu_seqlens_k; p.total_q = total_q; p.total_k = total_k;
+  // packed tensors: one batch of tokens (batch stride 0)
+  for (long long* st : {p.st_do, p.st_q, p.st_o, p.st_dq}) { st[0] = 0; st[1] = (long long)Hq * D; st[2] = D; }
+  for (long long* st : {p.st_k, p.st_v, p.st_dk, p.st_dv}) { st[0] = 0; st[1] = (long long)Hkv * D; st[2] = D; }
+  p.rows_packed = 1;
   fold_window(causal, window_left, window_right, &p.wl, &p.wr);
   scale = resolve_scale(scale, D);
   p.scale = scale;

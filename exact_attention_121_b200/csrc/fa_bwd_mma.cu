@@ -35,7 +35,18 @@ constexpr int kBwdThreads = 128;
 // A row is D/8 lanes with 16-byte loads; a warp takes 32/(D/8) rows per step
 // and keeps kPreSteps steps of loads in flight (the kernel is HBM-bound).
 constexpr int kPreSteps = 4;
-template <typename T, int D>
+
+// Element offset of row r = (token, head) of a (B, S, H, D) tensor with
+// strides st (batch, token, head); packed batches have one batch of total_q
+// tokens.
+// Row counts stay below 2^31 (checked on the host): 32-bit division.
+__device__ __forceinline__ long long row_offset(const BwdParams& p, const long long st[3], unsigned r) {
+  const unsigned tok = r / (unsigned)p.Hq, h = r - tok * (unsigned)p.Hq;
+  if (p.cu_q) return (long long)tok * st[1] + (long long)h * st[2];
+  const unsigned b = tok / (unsigned)p.Sq, i = tok - b * (unsigned)p.Sq;
+  return (long long)b * st[0] + (long long)i * st[1] + (long long)h * st[2];
+}
+template <typename T, int D, bool kPacked>
 __global__ void bwd_preprocess_kernel(const BwdParams p, int n_sem) {
   constexpr int kLanesPerRow = D / 8;
   constexpr int kRowsPerStep = 32 / kLanesPerRow;
@@ -52,8 +63,10 @@ __global__ void bwd_preprocess_kernel(const BwdParams p, int n_sem) {
     for (int u = 0; u < kPreSteps; ++u) {
       const long long r = base + u * kRowsPerStep + sub;
       if (r < rows) {
-        a[u] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.dout) + r * D + l * 8));
-        c[u] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.o) + r * D + l * 8));
+        const long long off_do = (kPacked ? r * D : row_offset(p, p.st_do, (unsigned)r)) + l * 8;
+        const long long off_o = (kPacked ? r * D : row_offset(p, p.st_o, (unsigned)r)) + l * 8;
+        a[u] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.dout) + off_do));
+        c[u] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.o) + off_o));
       } else {
         a[u] = c[u] = make_uint4(0, 0, 0, 0);
       }
@@ -380,16 +393,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_main_kernel(const BwdParam
   }
 }
 
-template <typename T>
+template <typename T, bool kPacked>
 __global__ void bwd_convert_kernel(const BwdParams p) {
-  const long long n4 = (p.cu_q ? (long long)p.total_q : (long long)p.B * p.Sq) * p.Hq * p.D / 4;
+  // D/4 lanes per (token, head) row of the packed accumulator, four
+  // consecutive elements per lane; a warp takes 32/(D/4) rows per step
+  const unsigned rows = (unsigned)((p.cu_q ? (long long)p.total_q : (long long)p.B * p.Sq) * p.Hq);
+  const int lane = threadIdx.x & 31;
+  const int lanes_per_row = p.D / 4, rows_per_step = 32 / lanes_per_row;
+  const int sub = lane / lanes_per_row, l = lane - sub * lanes_per_row;
+  const unsigned warp0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, nwarps = (gridDim.x * blockDim.x) >> 5;
   T* dq = reinterpret_cast<T*>(p.dq);
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
-    const float4 a = reinterpret_cast<const float4*>(p.dq_accum)[i];
+  if (kPacked) {
+    const long long n4 = (long long)rows * p.D / 4;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
+         i += (long long)gridDim.x * blockDim.x) {
+      const float4 a = reinterpret_cast<const float4*>(p.dq_accum)[i];
+      uint2 v;
+      v.x = Elem<T>::pack(a.x * p.scale, a.y * p.scale);
+      v.y = Elem<T>::pack(a.z * p.scale, a.w * p.scale);
+      reinterpret_cast<uint2*>(dq)[i] = v;
+    }
+    return;
+  }
+  for (unsigned base = warp0 * rows_per_step; base < rows; base += nwarps * rows_per_step) {
+    const unsigned r = base + sub;
+    if (r >= rows) continue;
+    const float4 a = reinterpret_cast<const float4*>(p.dq_accum + (size_t)r * p.D)[l];
     uint2 v;
     v.x = Elem<T>::pack(a.x * p.scale, a.y * p.scale);
     v.y = Elem<T>::pack(a.z * p.scale, a.w * p.scale);
-    reinterpret_cast<uint2*>(dq)[i] = v;
+    *reinterpret_cast<uint2*>(dq + row_offset(p, p.st_dq, r) + l * 4) = v;
   }
 }
 
@@ -419,10 +452,13 @@ template <typename T>
 cudaError_t launch_bwd_t(const BwdParams& p, cudaStream_t s, int* launches) {
   const int nqb = (p.Sq + kQB - 1) / kQB;
   const int n_sem = p.B * p.Hq * nqb;
+  // packed dout/out rows: plain indexing (fewer registers, full occupancy)
   if (p.D == 64)
-    bwd_preprocess_kernel<T, 64><<<148 * 8, 256, 0, s>>>(p, n_sem);
+    p.rows_packed ? bwd_preprocess_kernel<T, 64, true><<<148 * 8, 256, 0, s>>>(p, n_sem)
+                  : bwd_preprocess_kernel<T, 64, false><<<148 * 8, 256, 0, s>>>(p, n_sem);
   else
-    bwd_preprocess_kernel<T, 128><<<148 * 8, 256, 0, s>>>(p, n_sem);
+    p.rows_packed ? bwd_preprocess_kernel<T, 128, true><<<148 * 8, 256, 0, s>>>(p, n_sem)
+                  : bwd_preprocess_kernel<T, 128, false><<<148 * 8, 256, 0, s>>>(p, n_sem);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   ++*launches;
@@ -434,7 +470,8 @@ cudaError_t launch_bwd_t(const BwdParams& p, cudaStream_t s, int* launches) {
     e = (p.D == 64) ? launch_main_d<T, 64>(p, s) : launch_main_d<T, 128>(p, s);
   if (e != cudaSuccess) return e;
   ++*launches;
-  bwd_convert_kernel<T><<<148 * 8, 256, 0, s>>>(p);
+  p.rows_packed ? bwd_convert_kernel<T, true><<<148 * 8, 256, 0, s>>>(p)
+                : bwd_convert_kernel<T, false><<<148 * 8, 256, 0, s>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   ++*launches;

@@ -456,9 +456,10 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     } else {
       // ---- dV and dK rows of this warp's keys, head-dim half hh
       tc_fence_after();
-      const size_t ks = (size_t)p.Hkv * D;
-      T* dVr = reinterpret_cast<T*>(p.dv) + (size_t)(seq.ktok + key) * ks + (size_t)hkv * D + hh * (D / 2);
-      T* dKr = reinterpret_cast<T*>(p.dk) + (size_t)(seq.ktok + key) * ks + (size_t)hkv * D + hh * (D / 2);
+      T* dVr = reinterpret_cast<T*>(p.dv) + (long long)b * p.st_dv[0] + (long long)(seq.ktma + key) * p.st_dv[1] +
+               (long long)hkv * p.st_dv[2] + hh * (D / 2);
+      T* dKr = reinterpret_cast<T*>(p.dk) + (long long)b * p.st_dk[0] + (long long)(seq.ktma + key) * p.st_dk[1] +
+               (long long)hkv * p.st_dk[2] + hh * (D / 2);
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const float mul = which ? p.scale : 1.f;
@@ -615,10 +616,10 @@ cudaError_t launch_bwd_main_tc(const BwdParams& p, fa_dtype dt, cudaStream_t s) 
   const bool bf = dt == FA_BF16;
   // a packed batch is one batch of total_q / total_k token rows
   const int mq_s = p.cu_q ? p.total_q : p.Sq, mk_s = p.cu_q ? p.total_k : p.Sk, mb = p.cu_q ? 1 : p.B;
-  if (!make_bshd_map(&mq, p.q, bf, p.D, p.Hq, mq_s, mb, kQ) ||
-      !make_bshd_map(&mdo, p.dout, bf, p.D, p.Hq, mq_s, mb, kQ) ||
-      !make_bshd_map(&mk, p.k, bf, p.D, p.Hkv, mk_s, mb, kKeys) ||
-      !make_bshd_map(&mv, p.v, bf, p.D, p.Hkv, mk_s, mb, kKeys) ||
+  if (!make_bshd_map_strided(&mq, p.q, bf, p.D, p.Hq, mq_s, mb, p.st_q, kQ) ||
+      !make_bshd_map_strided(&mdo, p.dout, bf, p.D, p.Hq, mq_s, mb, p.st_do, kQ) ||
+      !make_bshd_map_strided(&mk, p.k, bf, p.D, p.Hkv, mk_s, mb, p.st_k, kKeys) ||
+      !make_bshd_map_strided(&mv, p.v, bf, p.D, p.Hkv, mk_s, mb, p.st_v, kKeys) ||
       !make_bshd_map_f32(&mdq, p.dq_accum, p.D, p.Hq, mq_s, mb, kQ))
     return cudaErrorNotSupported;
   const bool cap = p.softcap > 0.f;

@@ -459,7 +459,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       // ---- epilogue: O / l in 16 bits, LSE
       tc_fence_after();
       const float inv = l_q > 0.f ? 1.f / l_q : 0.f;
-      T* orow = reinterpret_cast<T*>(p.o) + ((size_t)(seq.qtok + qi) * p.Hq + h) * D;
+      T* orow = reinterpret_cast<T*>(p.o) + (long long)b * p.st_o[0] + (long long)(seq.qtma + qi) * p.st_o[1] +
+                (long long)h * p.st_o[2];
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t u[32];
@@ -535,8 +536,9 @@ cudaError_t launch_fwd_tc(const FwdParams& p, fa_dtype dt, cudaStream_t s, int* 
   const bool bf = dt == FA_BF16;
   // a packed batch is one batch of total_q / total_k token rows
   const int mq_s = p.cu_q ? p.total_q : p.Sq, mk_s = p.cu_q ? p.total_k : p.Sk, mb = p.cu_q ? 1 : p.B;
-  if (!make_bshd_map(&mq, p.q, bf, p.D, p.Hq, mq_s, mb, 128) || !make_bshd_map(&mk, p.k, bf, p.D, p.Hkv, mk_s, mb, 128) ||
-      !make_bshd_map(&mv, p.v, bf, p.D, p.Hkv, mk_s, mb, 128))
+  if (!make_bshd_map_strided(&mq, p.q, bf, p.D, p.Hq, mq_s, mb, p.st_q, 128) ||
+      !make_bshd_map_strided(&mk, p.k, bf, p.D, p.Hkv, mk_s, mb, p.st_k, 128) ||
+      !make_bshd_map_strided(&mv, p.v, bf, p.D, p.Hkv, mk_s, mb, p.st_v, 128))
     return cudaErrorNotSupported;
   cudaError_t e = bf ? launch_dt<__nv_bfloat16>(p, mq, mk, mv, s) : launch_dt<__half>(p, mq, mk, mv, s);
   if (e == cudaSuccess) ++*launches;

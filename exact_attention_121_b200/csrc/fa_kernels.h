@@ -29,6 +29,9 @@ struct FwdParams {
   const int* cu_q;
   const int* cu_k;
   int total_q, total_k;
+  // element strides (batch, token, head) of q, k, v, out; the head dimension
+  // is contiguous.  Packed batches have batch stride 0.
+  long long st_q[3], st_k[3], st_v[3], st_o[3];
 };
 
 struct BwdParams {
@@ -58,6 +61,10 @@ struct BwdParams {
   const int* cu_q;
   const int* cu_k;
   int total_q, total_k;
+  // element strides (batch, token, head) of every (B, S, H, D) tensor; the
+  // workspace tensors (dq_accum, delta) are always packed
+  long long st_do[3], st_q[3], st_k[3], st_v[3], st_o[3], st_dq[3], st_dk[3], st_dv[3];
+  int rows_packed;       // dout, out and dq are packed (token, head) rows: plain indexing
 };
 
 struct DecodeParams {

@@ -28,10 +28,20 @@ EncodeTiledFn encode_fn() {
 bool tma_available() { return encode_fn() != nullptr; }
 
 bool make_bshd_map(CUtensorMap* m, const void* base, bool bf16, int D, int H, int S, int B, int box_rows) {
+  const long long st[3] = {(long long)S * H * D, (long long)H * D, (long long)D};
+  return make_bshd_map_strided(m, base, bf16, D, H, S, B, st, box_rows);
+}
+
+bool make_bshd_map_strided(CUtensorMap* m, const void* base, bool bf16, int D, int H, int S, int B,
+                           const long long st[3], int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
+  if (st[0] < 0 || st[1] < 0 || st[2] < 0 || (st[0] % 8) || (st[1] % 8) || (st[2] % 8)) return false;
   const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
-  const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)S * H * D * 2};
+  // a stride of a dimension of extent 1 is never used; the encoder still
+  // wants it non-zero and 16-byte aligned
+  const cuuint64_t strides[3] = {(cuuint64_t)(H > 1 ? st[2] : D) * 2, (cuuint64_t)(S > 1 ? st[1] : (long long)H * D) * 2,
+                                 (cuuint64_t)(B > 1 ? st[0] : (long long)S * H * D) * 2};
   const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(base),

@@ -15,6 +15,10 @@ bool tma_available();
 // 1 head x `box_rows` rows x 1 batch, 128-byte swizzle, zero fill outside the
 // tensor.  Returns false if the encoder is missing or rejects the map.
 bool make_bshd_map(CUtensorMap* m, const void* base, bool bf16, int D, int H, int S, int B, int box_rows);
+// Same with element strides (batch, token, head) of a tensor whose head
+// dimension is contiguous; every stride must be a multiple of 8 elements.
+bool make_bshd_map_strided(CUtensorMap* m, const void* base, bool bf16, int D, int H, int S, int B,
+                           const long long st[3], int box_rows);
 
 // 4-D map (D, H, S, B) of fp32 elements with a box of all D elements x 1 head
 // x `box_rows` rows x 1 batch, no swizzle (dense row-major box in shared

@@ -156,6 +156,36 @@ fa_status fa_bwd_varlen(const void* dout, const void* q, const void* k, const vo
                         float scale, int causal, int window_left, int window_right, float softcap,
                         int deterministic, void* workspace, size_t ws_bytes, fa_stream_t stream);
 
+/*
+ * fa_fwd on tensors with arbitrary layouts (the pages' qkvpacked variant is
+ * the case q, k, v = views of one (B, S, 3, H, D) tensor).  Same arguments as
+ * fa_fwd plus `strides`: 12 host int64 values, the element strides
+ * (batch, token, head) of q, k, v and out in that order; the head dimension
+ * of every tensor is contiguous.  Each stride must be a non-negative multiple
+ * of 8 elements (16-byte rows for the TMA unit) and every base pointer
+ * 16-byte aligned, else FA_ERR_INVALID_ARG; a layout the tensor-map encoder
+ * rejects gives FA_ERR_UNSUPPORTED.  lse stays (B, Hq, Sq) packed.  tcgen05
+ * kernel only.
+ */
+fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* out, float* lse,
+                         int B, int Sq, int Sk, int Hq, int Hkv, int D, fa_dtype dt,
+                         float scale, int causal, int window_left, int window_right, float softcap,
+                         const long long* strides, fa_stream_t stream);
+
+/*
+ * fa_bwd on tensors with arbitrary layouts: `strides` holds 24 host int64
+ * values, (batch, token, head) element strides of dout, q, k, v, out, dq, dk,
+ * dv in that order (qkvpacked: dq, dk, dv are views of one (B, S, 3, H, D)
+ * gradient).  Rules as fa_fwd_strided; the workspace is fa_bwd_workspace_size
+ * of the same sizes and stays packed.
+ */
+fa_status fa_bwd_strided(const void* dout, const void* q, const void* k, const void* v,
+                         const void* out, const float* lse, void* dq, void* dk, void* dv,
+                         int B, int Sq, int Sk, int Hq, int Hkv, int D, fa_dtype dt,
+                         float scale, int causal, int window_left, int window_right, float softcap,
+                         int deterministic, void* workspace, size_t ws_bytes,
+                         const long long* strides, fa_stream_t stream);
+
 /* Largest split count fa_fwd_kvcache accepts; num_splits <= 0 picks one. */
 #define FA_MAX_SPLITS 64
 

@@ -109,3 +109,30 @@ def test_kvcache_workspace(lib):
 
 def test_selftest_rejects_null_flag(lib):
     assert lib.fa_selftest_bounded_wait(None, 1, 1000, None) == _lib.FA_ERR_INVALID_ARG
+
+
+def test_strided_and_varlen_host_validation(lib):
+    p = ctypes.c_void_p(0x1000)
+    good = [16, 8, 8] * 4  # (batch, token, head) element strides of q, k, v, out
+    arr = lambda vals: (ctypes.c_longlong * len(vals))(*vals)
+    fwd = lambda st: lib.fa_fwd_strided(p, p, p, p, p, 1, 8, 8, 1, 1, 64, 1, 0.0, 0, -1, -1, 0.0, st, None)
+    bad = list(good)
+    bad[1] = 12  # token stride not a multiple of 8 elements
+    assert fwd(arr(bad)) == _lib.FA_ERR_INVALID_ARG
+    bad = list(good)
+    bad[5] = -8
+    assert fwd(arr(bad)) == _lib.FA_ERR_INVALID_ARG
+    assert fwd(None) == _lib.FA_ERR_INVALID_ARG
+    bst = arr([8] * 23 + [4])
+    assert lib.fa_bwd_strided(p, p, p, p, p, p, p, p, p, 1, 8, 8, 1, 1, 64, 1, 0.0, 0, -1, -1, 0.0, 0,
+                              ctypes.c_void_p(0x10000), 1 << 20, bst, None) == _lib.FA_ERR_INVALID_ARG
+    # packed batches: missing offsets, negative sizes, empty batch
+    vfwd = lambda cu, B=2, tq=16: lib.fa_fwd_varlen(p, p, p, p, p, cu, cu, B, 8, 8, tq, 16, 2, 2, 64, 1, 0.0, 0,
+                                                    -1, -1, 0.0, None)
+    assert vfwd(None) == _lib.FA_ERR_INVALID_ARG
+    assert vfwd(p, tq=-1) == _lib.FA_ERR_INVALID_ARG
+    assert vfwd(ctypes.c_void_p(0x1002)) == _lib.FA_ERR_INVALID_ARG  # offsets not 4-byte aligned
+    assert vfwd(p, B=0) == _lib.FA_OK
+    # the packed workspace is linear in the token count
+    w = [lib.fa_bwd_varlen_workspace_size(8, 1024, T, 16, 128, 0) for T in (4096, 8192)]
+    assert abs(w[1] / w[0] - 2.0) < 0.01
