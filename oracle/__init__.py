@@ -12,6 +12,7 @@ from .attn64 import (  # noqa: F401
     effective_window,
     gather_cache,
     kvcache_append,
+    rotary,
     split_token_ranges,
     visible,
     visible_rows,

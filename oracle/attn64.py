@@ -41,6 +41,10 @@ Readings where the pages are silent:
   ``cache_seqlens[b] + Snew`` keys and does not update ``cache_seqlens``.
 * split s of a sequence with P pages covers pages
   ``ceil(s*P/n) .. ceil((s+1)*P/n) - 1``.
+* rotary (kvcache call): new token t of sequence b and its query sit at
+  position ``cache_seqlens[b] + t``; pairs (j, j + r/2) are rotated, or
+  (2j, 2j+1) when interleaved, with r = 2 * rotary_cos.shape[1]; the cache
+  holds keys already rotated.
 * varlen: sequences packed along the token axis with ``cu_seqlens`` offsets
   (sequence b is tokens ``cu[b] .. cu[b+1]-1``); each sequence is attended on
   its own, with the masks and the bottom-right alignment of its own lengths;
@@ -342,19 +346,49 @@ def gather_cache(cache, b, L, block_table=None, page_size=None):
     return np.stack(rows).astype(np.float64)
 
 
+def rotary(x, cos, sin, positions, interleaved=False):
+    """Rotary position embedding of the rows of ``x`` (..., R, H, D) at
+    ``positions`` (..., R): the first ``r = 2 * cos.shape[1]`` dims of each
+    head are rotated pairwise by angle theta[pos, j] with cos/sin[pos, j]
+    given; non-interleaved pairs are (j, j + r/2), interleaved (2j, 2j+1).
+    Dims past r are unchanged."""
+    x = np.array(x, np.float64, copy=True)
+    c = np.asarray(cos, np.float64)[np.asarray(positions)][..., None, :]  # (..., R, 1, r/2)
+    s = np.asarray(sin, np.float64)[np.asarray(positions)][..., None, :]
+    half = c.shape[-1]
+    if interleaved:
+        a, b = x[..., 0:2 * half:2].copy(), x[..., 1:2 * half:2].copy()
+        x[..., 0:2 * half:2] = a * c - b * s
+        x[..., 1:2 * half:2] = b * c + a * s
+    else:
+        a, b = x[..., :half].copy(), x[..., half:2 * half].copy()
+        x[..., :half] = a * c - b * s
+        x[..., half:2 * half] = b * c + a * s
+    return x
+
+
 def attn_with_kvcache(q, k_cache, v_cache, k_new=None, v_new=None, cache_seqlens=None,
                       block_table=None, page_size=None, scale=None, causal=False,
-                      window_left=-1, window_right=-1, softcap=0.0):
+                      window_left=-1, window_right=-1, softcap=0.0, rotary_cos=None, rotary_sin=None,
+                      rotary_interleaved=False):
     """Append then attend: q (B, Sq, Hq, D) against each sequence's cache.
 
     Sequence b attends over L_b = cache_seqlens[b] + Snew keys (Snew = 0 when
     no new K/V is given), with the bottom-right alignment of
-    :func:`visible`.  Returns O (B, Sq, Hq, D), LSE (B, Hq, Sq) and the
-    updated caches.
+    :func:`visible`.  With rotary tables, new key row t of sequence b and
+    query row i are first rotated (:func:`rotary`) at positions
+    cache_seqlens[b] + t and cache_seqlens[b] + i (the queries are the new
+    tokens'); the cache already holds rotated keys.  Returns O
+    (B, Sq, Hq, D), LSE (B, Hq, Sq) and the updated caches.
     """
     q = np.asarray(q, np.float64)
     B, Sq, Hq, D = q.shape
     Snew = 0 if k_new is None else k_new.shape[1]
+    if rotary_cos is not None:
+        base = np.asarray(cache_seqlens, np.int64)[:, None]
+        q = rotary(q, rotary_cos, rotary_sin, base + np.arange(Sq)[None, :], rotary_interleaved)
+        if Snew:
+            k_new = rotary(k_new, rotary_cos, rotary_sin, base + np.arange(Snew)[None, :], rotary_interleaved)
     kc, vc = kvcache_append(k_cache, v_cache, k_new, v_new, cache_seqlens, block_table, page_size)
     out = np.zeros((B, Sq, Hq, D))
     lse = np.full((B, Hq, Sq), NEG_INF)

@@ -520,3 +520,71 @@ def test_varlen_sequence_without_keys():
     np.testing.assert_allclose(o[3:], o_s[0], atol=1e-13)
     dq, dk, dv = attn64.attn_bwd_varlen(_rand((7, 2, 4), rng), q, k, v, cq, ck)
     assert np.all(dq[:3] == 0)
+
+
+# ---------------------------------------------------------------------------
+# rotary position embedding in the kvcache call
+# ---------------------------------------------------------------------------
+
+def _rope_tables(n_pos, half, base=10000.0):
+    inv = base ** (-np.arange(half) / half)
+    ang = np.arange(n_pos)[:, None] * inv[None, :]
+    return np.cos(ang), np.sin(ang)
+
+
+def test_rotary_two_dims_is_a_rotation_matrix():
+    # D = 2, one pair: (x, y) -> (x cos t - y sin t, y cos t + x sin t)
+    t = 0.7
+    cos, sin = np.array([[1.0], [math.cos(t)]]), np.array([[0.0], [math.sin(t)]])
+    x = np.array([[[[3.0, -2.0]]]])  # (1, 1, 1, 2)
+    for inter in (False, True):
+        r = attn64.rotary(x, cos, sin, np.array([[1]]), inter)
+        np.testing.assert_allclose(r[0, 0, 0], [3 * math.cos(t) + 2 * math.sin(t), -2 * math.cos(t) + 3 * math.sin(t)],
+                                   atol=1e-15)
+        np.testing.assert_array_equal(attn64.rotary(x, cos, sin, np.array([[0]]), inter), x)  # angle 0
+
+
+@pytest.mark.parametrize("inter", [False, True])
+def test_rotary_keeps_norms_and_depends_on_relative_position(inter):
+    rng = np.random.default_rng(45)
+    D, half = 16, 6
+    cos, sin = _rope_tables(64, half)
+    q, k = _rand((1, 1, 1, D), rng), _rand((1, 1, 1, D), rng)
+    # pairwise rotation keeps the norm
+    r = attn64.rotary(q, cos, sin, np.array([[37]]), inter)
+    np.testing.assert_allclose(np.linalg.norm(r), np.linalg.norm(q), rtol=1e-13)
+    np.testing.assert_array_equal(r[..., 2 * half:], q[..., 2 * half:])  # dims past r untouched
+    # <R(p) q, R(p') k> depends on p - p' only
+    dots = [float(np.sum(attn64.rotary(q, cos, sin, np.array([[p + 5]]), inter) *
+                         attn64.rotary(k, cos, sin, np.array([[p]]), inter))) for p in (0, 9, 40)]
+    np.testing.assert_allclose(dots, dots[0], rtol=1e-12)
+
+
+def test_rotary_interleaved_is_a_permutation_of_halves():
+    rng = np.random.default_rng(46)
+    D, half = 8, 4
+    cos, sin = _rope_tables(10, half)
+    x = _rand((1, 3, 2, D), rng)
+    pos = np.array([[1, 4, 7]])
+    perm = np.concatenate([np.arange(0, D, 2), np.arange(1, D, 2)])  # interleaved -> halves
+    r_int = attn64.rotary(x, cos, sin, pos, True)
+    r_half = attn64.rotary(x[..., perm], cos, sin, pos, False)
+    np.testing.assert_allclose(r_int[..., perm], r_half, atol=1e-14)
+
+
+def test_kvcache_rotary_matches_prerotated_inputs():
+    rng = np.random.default_rng(47)
+    B, Hq, Hkv, D, Snew, L = 2, 4, 2, 8, 2, 6
+    cos, sin = _rope_tables(16, 3)
+    kc, vc = _rand((B, 12, Hkv, D), rng), _rand((B, 12, Hkv, D), rng)
+    q, kn, vn = _rand((B, Snew, Hq, D), rng), _rand((B, Snew, Hkv, D), rng), _rand((B, Snew, Hkv, D), rng)
+    sl = np.array([L, 3])
+    o1, l1, kc1, _ = attn64.attn_with_kvcache(q, kc, vc, kn, vn, sl, causal=True, rotary_cos=cos, rotary_sin=sin)
+    pos = sl[:, None] + np.arange(Snew)[None, :]
+    o2, l2, kc2, _ = attn64.attn_with_kvcache(attn64.rotary(q, cos, sin, pos), kc, vc, attn64.rotary(kn, cos, sin, pos),
+                                              vn, sl, causal=True)
+    np.testing.assert_allclose(o1, o2, atol=1e-13)
+    np.testing.assert_allclose(kc1, kc2, atol=1e-13)
+    # the appended keys are rotated, the old cache rows are not touched
+    np.testing.assert_array_equal(kc1[0, :L], kc[0, :L])
+    assert not np.allclose(kc1[0, L:L + Snew], kn[0])
