@@ -36,6 +36,9 @@ SIGNATURES = {
     "fa_kvcache_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "fa_fwd_kvcache": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _I, _I, _I, _I, _I, _I,
                             _I, _F, _I, _I, _I, _F, _I, _P, _Z, _P]),
+    "fa_kvcache_rotary_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
+    "fa_fwd_kvcache_rotary": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _I, _I, _I, _I, _I, _I,
+                                   _I, _F, _I, _I, _I, _F, _P, _P, _I, _I, _I, _I, _P, _Z, _P]),
     "fa_fwd_kvcache_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _I, _I, _I, _I, _I, _I,
                                     _I, _F, _I, _I, _I, _F, _I, _P]),
     "fa_last_device_status": (_I, [_P]),

@@ -225,13 +225,16 @@ def fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits):
 
 def fa_fwd_kvcache(q, k_cache, v_cache, k_new=None, v_new=None, cache_seqlens=None, block_table=None,
                    page_size=256, out=None, lse=None, scale=None, causal=False, window=(-1, -1),
-                   softcap=0.0, num_splits=0, workspace=None, stream=None, return_lse=True):
+                   softcap=0.0, num_splits=0, workspace=None, stream=None, return_lse=True, rotary_cos=None,
+                   rotary_sin=None, rotary_interleaved=False):
     """Append k_new/v_new into the cache (in place), then attend; returns (out, lse).
 
     Paged when ``block_table`` (B, max_pages_per_seq) int32 is given: caches
     are (num_pages, page_size, Hkv, D).  Otherwise caches are
     (B, max_seqlen, Hkv, D).  ``cache_seqlens`` (B,) int32 is the length
-    before the append and is not modified.
+    before the append and is not modified.  ``rotary_cos``/``rotary_sin``
+    (seqlen_ro, rotary_dim/2) float32 tables rotate the new keys and the
+    queries at positions cache_seqlens[b] + t (fa_fwd_kvcache_rotary).
     """
     lib = _lib.load()
     B, Sq, Hq, D = q.shape
@@ -253,17 +256,29 @@ def fa_fwd_kvcache(q, k_cache, v_cache, k_new=None, v_new=None, cache_seqlens=No
     out = torch.empty_like(q) if out is None else out
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
-    need = fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits)
-    if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wl, wr = _window(window)
-    code = lib.fa_fwd_kvcache(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_new), _ptr(v_new),
-                              _ptr(cache_seqlens), _ptr(block_table), int(page_size), int(max_pages_per_seq),
-                              int(cap), _ptr(out), _ptr(lse), B, Sq, Snew, Hq, Hkv, D, _DT[dt],
-                              float(scale or 0.0), int(bool(causal)), wl, wr, float(softcap or 0.0),
-                              int(num_splits), _ptr(workspace), 0 if workspace is None else workspace.numel(),
-                              _stream(stream))
-    _lib.check(code, "fa_fwd_kvcache")
+    head = (_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_new), _ptr(v_new), _ptr(cache_seqlens), _ptr(block_table),
+            int(page_size), int(max_pages_per_seq), int(cap), _ptr(out), _ptr(lse), B, Sq, Snew, Hq, Hkv, D, _DT[dt],
+            float(scale or 0.0), int(bool(causal)), wl, wr, float(softcap or 0.0))
+    if rotary_cos is None:
+        need = fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits)
+        if workspace is None and need > 0:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        code = lib.fa_fwd_kvcache(*head, int(num_splits), _ptr(workspace),
+                                  0 if workspace is None else workspace.numel(), _stream(stream))
+        _lib.check(code, "fa_fwd_kvcache")
+        return out, lse
+    for t, n in ((rotary_cos, "rotary_cos"), (rotary_sin, "rotary_sin")):
+        _check_tensor(t, n, torch.float32, q.device)
+    if rotary_cos.shape != rotary_sin.shape or rotary_cos.dim() != 2:
+        raise ValueError("rotary_cos and rotary_sin must be (seqlen_ro, rotary_dim/2) float32")
+    need = int(lib.fa_kvcache_rotary_workspace_size(B, Sq, Hq, D, num_splits))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    code = lib.fa_fwd_kvcache_rotary(*head, _ptr(rotary_cos), _ptr(rotary_sin), 2 * rotary_cos.shape[1],
+                                     rotary_cos.shape[0], int(bool(rotary_interleaved)), int(num_splits),
+                                     _ptr(workspace), workspace.numel(), _stream(stream))
+    _lib.check(code, "fa_fwd_kvcache_rotary")
     return out, lse
 
 

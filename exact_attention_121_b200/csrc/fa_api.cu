@@ -435,11 +435,20 @@ size_t fa_kvcache_workspace_size(int B, int Sq, int Hq, int D, int num_splits) {
   return round256(rows * D * sizeof(float)) + round256(rows * sizeof(float));
 }
 
-fa_status fa_fwd_kvcache(const void* q, void* k_cache, void* v_cache, const void* k_new, const void* v_new,
-                         const int* cache_seqlens, const int* block_table, int page_size, int max_pages_per_seq,
-                         int num_pages_or_max_seqlen, void* out, float* lse, int B, int Sq, int Snew, int Hq,
-                         int Hkv, int D, fa_dtype dt, float scale, int causal, int window_left, int window_right,
-                         float softcap, int num_splits, void* workspace, size_t ws_bytes, fa_stream_t stream) {
+struct RotaryArgs {
+  const float* cos;
+  const float* sin;
+  int dim, len, interleaved;
+};
+
+// rot: NULL, or rotary tables; their q copy takes the first
+// round256(B*Sq*Hq*D*2) bytes of the workspace
+static fa_status kvcache_impl(const void* q, void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                              const int* cache_seqlens, const int* block_table, int page_size, int max_pages_per_seq,
+                              int num_pages_or_max_seqlen, void* out, float* lse, int B, int Sq, int Snew, int Hq,
+                              int Hkv, int D, fa_dtype dt, float scale, int causal, int window_left,
+                              int window_right, float softcap, int num_splits, void* workspace, size_t ws_bytes,
+                              const RotaryArgs* rot, fa_stream_t stream) {
   g_last_launches = 0;
   fa_status st = check_common(B, Sq, Hq, Hkv, D, dt, scale, softcap);
   if (st != FA_OK) return st;
@@ -483,6 +492,20 @@ fa_status fa_fwd_kvcache(const void* q, void* k_cache, void* v_cache, const void
     num_splits = n < 1 ? 1 : (int)n;
   }
   p.num_splits = num_splits;
+  if (rot) {
+    if (!rot->cos || !rot->sin || rot->dim <= 0 || rot->dim % 2 || rot->dim > D || rot->len <= 0)
+      return FA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(rot->cos) & 3u) || (reinterpret_cast<uintptr_t>(rot->sin) & 3u))
+      return FA_ERR_INVALID_ARG;
+    const size_t qbytes = round256((size_t)B * Sq * Hq * D * 2);
+    if (!workspace || ws_bytes < qbytes || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      return FA_ERR_INVALID_ARG;
+    p.rot_cos = rot->cos; p.rot_sin = rot->sin; p.rot_half = rot->dim / 2; p.rot_len = rot->len;
+    p.rot_inter = rot->interleaved ? 1 : 0;
+    p.q_rot = workspace;
+    workspace = static_cast<uint8_t*>(workspace) + qbytes;
+    ws_bytes -= qbytes;
+  }
   if (num_splits > 1) {
     const size_t rows = (size_t)num_splits * B * Hq * Sq;
     const size_t need = round256(rows * D * sizeof(float)) + round256(rows * sizeof(float));
@@ -497,6 +520,34 @@ fa_status fa_fwd_kvcache(const void* q, void* k_cache, void* v_cache, const void
   cudaError_t e = fa::launch_decode(p, dt, stream, &launches);
   g_last_launches = launches;
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_fwd_kvcache(const void* q, void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                         const int* cache_seqlens, const int* block_table, int page_size, int max_pages_per_seq,
+                         int num_pages_or_max_seqlen, void* out, float* lse, int B, int Sq, int Snew, int Hq,
+                         int Hkv, int D, fa_dtype dt, float scale, int causal, int window_left, int window_right,
+                         float softcap, int num_splits, void* workspace, size_t ws_bytes, fa_stream_t stream) {
+  return kvcache_impl(q, k_cache, v_cache, k_new, v_new, cache_seqlens, block_table, page_size, max_pages_per_seq,
+                      num_pages_or_max_seqlen, out, lse, B, Sq, Snew, Hq, Hkv, D, dt, scale, causal, window_left,
+                      window_right, softcap, num_splits, workspace, ws_bytes, nullptr, stream);
+}
+
+size_t fa_kvcache_rotary_workspace_size(int B, int Sq, int Hq, int D, int num_splits) {
+  if (B < 0 || Sq < 0 || Hq <= 0 || (D != 64 && D != 128)) return 0;
+  return round256((size_t)B * Sq * Hq * D * 2) + fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits);
+}
+
+fa_status fa_fwd_kvcache_rotary(const void* q, void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                                const int* cache_seqlens, const int* block_table, int page_size,
+                                int max_pages_per_seq, int num_pages_or_max_seqlen, void* out, float* lse, int B,
+                                int Sq, int Snew, int Hq, int Hkv, int D, fa_dtype dt, float scale, int causal,
+                                int window_left, int window_right, float softcap, const float* rotary_cos,
+                                const float* rotary_sin, int rotary_dim, int seqlen_ro, int rotary_interleaved,
+                                int num_splits, void* workspace, size_t ws_bytes, fa_stream_t stream) {
+  const RotaryArgs rot{rotary_cos, rotary_sin, rotary_dim, seqlen_ro, rotary_interleaved};
+  return kvcache_impl(q, k_cache, v_cache, k_new, v_new, cache_seqlens, block_table, page_size, max_pages_per_seq,
+                      num_pages_or_max_seqlen, out, lse, B, Sq, Snew, Hq, Hkv, D, dt, scale, causal, window_left,
+                      window_right, softcap, num_splits, workspace, ws_bytes, &rot, stream);
 }
 
 fa_status fa_last_device_status(fa_stream_t stream) {

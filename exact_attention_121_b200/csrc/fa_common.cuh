@@ -66,6 +66,7 @@ struct Elem<__half> {
     return __half22float2(h);
   }
   __device__ static __forceinline__ __half from_float(float x) { return __float2half_rn(x); }
+  __device__ static __forceinline__ float to_float(__half x) { return __half2float(x); }
 };
 
 template <>
@@ -80,6 +81,7 @@ struct Elem<__nv_bfloat16> {
     return __bfloat1622float2(h);
   }
   __device__ static __forceinline__ __nv_bfloat16 from_float(float x) { return __float2bfloat16_rn(x); }
+  __device__ static __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
 };
 
 // ---------------------------------------------------------------------------

@@ -81,6 +81,79 @@ __global__ void kvcache_append_kernel(const DecodeParams p) {
   }
 }
 
+// Element d of a row of x rotated at table row `pos` (rotary position
+// embedding): pairs (j, j + half), or (2j, 2j + 1) when interleaved, turn by
+// the angle whose cosine and sine the tables hold; dims past 2 * half are
+// copied.  Computed in float32 from the 16-bit inputs.
+template <typename T>
+__device__ __forceinline__ float rotate_elem(const DecodeParams& p, const T* x, int d, int pos) {
+  const int half = p.rot_half;
+  const float xd = Elem<T>::to_float(x[d]);
+  if (d >= 2 * half) return xd;
+  int j, partner;
+  float sign;
+  if (p.rot_inter) {
+    j = d >> 1;
+    partner = d ^ 1;
+    sign = (d & 1) ? 1.f : -1.f;
+  } else {
+    j = d < half ? d : d - half;
+    partner = d < half ? d + half : d - half;
+    sign = d < half ? -1.f : 1.f;
+  }
+  const float c = __ldg(p.rot_cos + (size_t)pos * half + j), s = __ldg(p.rot_sin + (size_t)pos * half + j);
+  return xd * c + sign * Elem<T>::to_float(x[partner]) * s;
+}
+
+// q row (b, i, h) rotated at position cache_seqlens[b] + i into q_rot.
+template <typename T>
+__global__ void rotary_q_kernel(const DecodeParams p) {
+  const long long total = (long long)p.B * p.Sq * p.Hq * p.D;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int d = (int)(e % p.D);
+    const long long row = e / p.D;  // (b, i, h)
+    const int i = (int)((row / p.Hq) % p.Sq);
+    const int b = (int)(row / ((long long)p.Hq * p.Sq));
+    const T* x = reinterpret_cast<const T*>(p.q) + row * p.D;
+    int pos = __ldg(p.cache_seqlens + b) + i;
+    if (pos < 0 || pos >= p.rot_len) {
+      report_status(p.status, kStatusBadArg);
+      pos = min(max(pos, 0), p.rot_len - 1);
+    }
+    reinterpret_cast<T*>(p.q_rot)[e] = Elem<T>::from_float(rotate_elem<T>(p, x, d, pos));
+  }
+}
+
+// kvcache_append_kernel with k_new rotated at its position on the way in.
+template <typename T>
+__global__ void kvcache_append_rotary_kernel(const DecodeParams p) {
+  const long long total = (long long)p.B * p.Snew * p.Hkv * p.D;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int d = (int)(e % p.D);
+    long long r = e / p.D;
+    const int g = (int)(r % p.Hkv);
+    r /= p.Hkv;
+    const int t = (int)(r % p.Snew);
+    const int b = (int)(r / p.Snew);
+    const int pos = __ldg(p.cache_seqlens + b) + t;
+    if (pos < 0 || pos >= seq_capacity(p) || pos >= p.rot_len) {
+      report_status(p.status, kStatusBadArg);
+      continue;
+    }
+    const long long dst = cache_row(p, b, pos, g);
+    if (dst < 0) {
+      report_status(p.status, kStatusBadArg);
+      continue;
+    }
+    const size_t src = (((size_t)b * p.Snew + t) * p.Hkv + g) * p.D;
+    reinterpret_cast<T*>(p.k_cache)[dst + d] =
+        Elem<T>::from_float(rotate_elem<T>(p, reinterpret_cast<const T*>(p.k_new) + src, d, pos));
+    reinterpret_cast<T*>(p.v_cache)[dst + d] = reinterpret_cast<const T*>(p.v_new)[src + d];
+  }
+}
+
 template <typename T, int D, bool kCap>
 __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeParams p) {
   constexpr int CH = D / 8;
@@ -409,9 +482,29 @@ cudaError_t launch_split(const DecodeParams& p, cudaStream_t s) {
 }
 
 template <typename T>
-cudaError_t launch_decode_t(const DecodeParams& p, cudaStream_t s, int* launches) {
+cudaError_t launch_decode_t(const DecodeParams& p_in, cudaStream_t s, int* launches) {
   cudaError_t e;
-  if (p.Snew > 0) {
+  DecodeParams p = p_in;
+  if (p.rot_cos) {
+    // rotate q into the scratch copy the attention kernels then read
+    const long long total = (long long)p.B * p.Sq * p.Hq * p.D;
+    const int threads = 256;
+    const int blocks = (int)((total + threads - 1) / threads < 4096 ? (total + threads - 1) / threads : 4096);
+    rotary_q_kernel<T><<<blocks, threads, 0, s>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    ++*launches;
+    p.q = p.q_rot;
+  }
+  if (p.Snew > 0 && p.rot_cos) {
+    const long long total = (long long)p.B * p.Snew * p.Hkv * p.D;
+    const int threads = 256;
+    const int blocks = (int)((total + threads - 1) / threads < 4096 ? (total + threads - 1) / threads : 4096);
+    kvcache_append_rotary_kernel<T><<<blocks, threads, 0, s>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    ++*launches;
+  } else if (p.Snew > 0) {
     const long long total = (long long)p.B * p.Snew * p.Hkv * (p.D / 8);
     const int threads = 256;
     const int blocks = (int)((total + threads - 1) / threads < 4096 ? (total + threads - 1) / threads : 4096);

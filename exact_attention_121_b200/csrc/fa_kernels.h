@@ -87,6 +87,13 @@ struct DecodeParams {
   int wl, wr;
   float scale_log2, softcap, cap_in, cap_log2;
   int* status;
+  // rotary position embedding (rot_cos == null: off): float32 tables
+  // (rot_len, rot_half); q is rotated into q_rot, which the attention
+  // kernels then read as q, and k_new is rotated on its way into the cache
+  const float* rot_cos;
+  const float* rot_sin;
+  int rot_half, rot_len, rot_inter;
+  void* q_rot;
 };
 
 // Optional timing hooks around the dominant kernel of each call (events set

@@ -229,6 +229,38 @@ fa_status fa_fwd_kvcache(const void* q, void* k_cache, void* v_cache, const void
                          float softcap, int num_splits, void* workspace, size_t ws_bytes,
                          fa_stream_t stream);
 
+/*
+ * Workspace of fa_fwd_kvcache_rotary: the rotated copy of q (B, Sq, Hq, D
+ * 16-bit, rounded up to 256 bytes) followed by fa_kvcache_workspace_size of
+ * the same arguments.
+ */
+size_t fa_kvcache_rotary_workspace_size(int B, int Sq, int Hq, int D, int num_splits);
+
+/*
+ * fa_fwd_kvcache with the rotary position embedding the pages' kvcache call
+ * takes (rotary_cos / rotary_sin).  Arguments as fa_fwd_kvcache, plus:
+ *   rotary_cos, rotary_sin: float32 device tables (seqlen_ro, rotary_dim/2);
+ *     entry [pos][j] is the cosine / sine of pair j's angle at position pos.
+ *   rotary_dim: even, 0 < rotary_dim <= D; dims past it are not rotated.
+ *   rotary_interleaved: 0 rotates pairs (j, j + rotary_dim/2), 1 pairs
+ *     (2j, 2j+1).
+ * New key row t of sequence b and query row t sit at position
+ * cache_seqlens[b] + t: the keys are rotated on their way into the cache
+ * (the cache holds rotated keys), the queries into a copy at the start of
+ * the workspace.  Positions outside [0, seqlen_ro) record FA_ERR_INVALID_ARG
+ * in the device status word (such a key is not appended; such a query uses
+ * the nearest table row).  workspace >= fa_kvcache_rotary_workspace_size(...)
+ * bytes, 256-byte aligned.
+ */
+fa_status fa_fwd_kvcache_rotary(const void* q, void* k_cache, void* v_cache, const void* k_new,
+                                const void* v_new, const int* cache_seqlens, const int* block_table,
+                                int page_size, int max_pages_per_seq, int num_pages_or_max_seqlen,
+                                void* out, float* lse, int B, int Sq, int Snew, int Hq, int Hkv, int D,
+                                fa_dtype dt, float scale, int causal, int window_left, int window_right,
+                                float softcap, const float* rotary_cos, const float* rotary_sin,
+                                int rotary_dim, int seqlen_ro, int rotary_interleaved, int num_splits,
+                                void* workspace, size_t ws_bytes, fa_stream_t stream);
+
 /* Size of the fixed device scratch array behind fa_fwd_kvcache_noalloc. */
 #define FA_STATIC_SCRATCH_BYTES (8u * 1024u * 1024u)
 

@@ -10,6 +10,7 @@ failure run has already run every other test; it also passes alone.
 """
 
 import ctypes
+import gc
 
 import pytest
 import torch
@@ -53,12 +54,20 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
         out = torch.empty_like(d["q"])
         lse = torch.empty_like(ref_lse)
         torch.cuda.synchronize()
-        before = torch.cuda.memory_allocated()
-        code = _noalloc(lib, d, splits, out, lse)
-        torch.cuda.synchronize()
+        # tensors that earlier tests left in reference cycles must not be
+        # freed inside the measured call
+        gc.collect()
+        gc.disable()
+        try:
+            before = torch.cuda.memory_allocated()
+            code = _noalloc(lib, d, splits, out, lse)
+            torch.cuda.synchronize()
+            after = torch.cuda.memory_allocated()
+        finally:
+            gc.enable()
         assert code == _lib.FA_OK, api.fa_status_string(code)
         assert api.fa_last_device_status() == 0
-        assert torch.cuda.memory_allocated() == before
+        assert after == before
         check_out(out, f64(ref_out), torch.bfloat16)
         check_lse(lse, f64(ref_lse))
 
