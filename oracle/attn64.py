@@ -22,6 +22,9 @@ there, so each function states the reading it implements):
   appends the new K/V into the existing cache and attends in place,
   ``cache_seqlens`` marks each sample's valid length, ``block_table`` pages the
   cache, ``num_splits`` splits the KV range.  -> :func:`attn_with_kvcache`.
+* same page, advanced parameters: ``alibi_slopes`` adds an ALiBi position
+  bias that lowers the scores of distant keys, instead of an explicit
+  position encoding.  -> :func:`alibi_bias`.
 * same page, the three techniques: tiling, online softmax (running row max and
   running sum updated block by block), recomputation in the backward.
   -> :func:`attn_fwd_online` (used only to pin :func:`attn_fwd`).
@@ -45,6 +48,10 @@ Readings where the pages are silent:
   position ``cache_seqlens[b] + t``; pairs (j, j + r/2) are rotated, or
   (2j, 2j+1) when interleaved, with r = 2 * rotary_cos.shape[1]; the cache
   holds keys already rotated.
+* ALiBi: with slope m of (batch b, q-head h) the score of query i and key j
+  gains ``-m * |i + off - j|`` (``off`` of the bottom-right alignment),
+  added after the soft cap and before the mask; slopes are (Hq,) shared by
+  the batch or (B, Hq).
 * varlen: sequences packed along the token axis with ``cu_seqlens`` offsets
   (sequence b is tokens ``cu[b] .. cu[b+1]-1``); each sequence is attended on
   its own, with the masks and the bottom-right alignment of its own lengths;
@@ -129,11 +136,26 @@ def transform_scores(u, softcap):
     return u
 
 
+def head_slopes(alibi_slopes, B, h):
+    """Slope of q-head h for each of the B batch rows: slopes (Hq,) are
+    shared by the batch, (B, Hq) are per batch row."""
+    m = np.asarray(alibi_slopes, np.float64)
+    return np.full(B, m[h]) if m.ndim == 1 else m[:, h].copy()
+
+
+def alibi_bias(slope, rows, Sq, Sk):
+    """Bias ``-slope * |i + Sk - Sq - j|`` of query rows ``rows`` against keys
+    0..Sk-1 (distance at the bottom-right aligned positions)."""
+    qpos = np.asarray(rows)[:, None] + (Sk - Sq)
+    return -float(slope) * np.abs(qpos - np.arange(Sk)[None, :]).astype(np.float64)
+
+
 def attn_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1,
-             softcap=0.0, return_probs=False):
-    """Exact attention O = softmax(transform(scale * Q K^T) + mask) V.
+             softcap=0.0, return_probs=False, alibi_slopes=None):
+    """Exact attention O = softmax(transform(scale * Q K^T) [+ ALiBi] + mask) V.
 
     q: (B, Sq, Hq, D); k, v: (B, Sk, Hkv, D), any float dtype (upcast to f64).
+    ``alibi_slopes`` (Hq,) or (B, Hq) adds :func:`alibi_bias`.
     Returns O (B, Sq, Hq, D) f64 and LSE (B, Hq, Sq) f64 (natural log).
     With ``return_probs`` also returns P (B, Hq, Sq, Sk) and the raw
     scores u (B, Hq, Sq, Sk).
@@ -155,6 +177,9 @@ def attn_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1,
         g = h // G
         u = raw_scores(q, k, scale, h, g)              # (B, Sq, Sk)
         s = transform_scores(u, softcap)
+        if alibi_slopes is not None:
+            ms = head_slopes(alibi_slopes, B, h)
+            s = s + np.stack([alibi_bias(ms[b], np.arange(Sq), Sq, Sk) for b in range(B)])
         s = np.where(vis[None], s, NEG_INF)
         any_vis = vis.any(axis=1)                       # (Sq,)
         m = np.where(any_vis[None], s.max(axis=2), 0.0)  # row max over visible keys
@@ -173,7 +198,7 @@ def attn_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1,
 
 
 def attn_fwd_rows(q, k, v, b, h, rows, scale=None, causal=False, window_left=-1, window_right=-1,
-                  softcap=0.0):
+                  softcap=0.0, alibi_slopes=None):
     """O and LSE of selected query rows of one (batch b, q-head h).
 
     Each row is the plain definition on its own: its scores against every
@@ -194,6 +219,8 @@ def attn_fwd_rows(q, k, v, b, h, rows, scale=None, causal=False, window_left=-1,
     Vg = np.asarray(v[b, :, g, :], np.float64)
     u = scale * (np.asarray(q[b, rows, h, :], np.float64) @ Kg.T)   # (R, Sk)
     s = transform_scores(u, softcap)
+    if alibi_slopes is not None:
+        s = s + alibi_bias(head_slopes(alibi_slopes, B, h)[b], rows, Sq, Sk)
     vis = visible_rows(rows, Sq, Sk, causal, window_left, window_right)
     s = np.where(vis, s, NEG_INF)
     anyv = vis.any(axis=1)
@@ -258,13 +285,14 @@ def attn_fwd_online(q, k, v, scale=None, causal=False, window_left=-1, window_ri
 # ---------------------------------------------------------------------------
 
 def attn_bwd(dout, q, k, v, scale=None, causal=False, window_left=-1, window_right=-1,
-             softcap=0.0):
+             softcap=0.0, alibi_slopes=None):
     """Gradients of L = sum(dout * O) with respect to q, k, v.
 
     Steps (per q-head h reading kv-head g):
       dV_g += P^T dO ; dP = dO V^T ; Delta_i = sum_j P_ij dP_ij ;
       dS = P * (dP - Delta) ; dU = dS * (1 - tanh^2(u/softcap)) when capped ;
       dQ = scale * dU K ; dK_g += scale * dU^T Q.
+    The ALiBi bias is a constant of the inputs: it changes P, not the chain.
     Returns dq, dk, dv (f64, shapes of q, k, v) and Delta (B, Hq, Sq).
     """
     dout = np.asarray(dout, np.float64)
@@ -283,8 +311,9 @@ def attn_bwd(dout, q, k, v, scale=None, causal=False, window_left=-1, window_rig
     for h in range(Hq):
         g = h // G
         # forward of this head alone (same definition as attn_fwd)
+        sl_h = None if alibi_slopes is None else head_slopes(alibi_slopes, B, h)[:, None]
         _, _, P, U = attn_fwd(q[:, :, h:h + 1], k[:, :, g:g + 1], v[:, :, g:g + 1], scale, causal,
-                              window_left, window_right, softcap, return_probs=True)
+                              window_left, window_right, softcap, return_probs=True, alibi_slopes=sl_h)
         Ph, Uh = P[:, 0], U[:, 0]                       # (B, Sq, Sk)
         del P, U
         dO = dout[:, :, h, :]                           # (B, Sq, D)

@@ -588,3 +588,134 @@ def test_kvcache_rotary_matches_prerotated_inputs():
     # the appended keys are rotated, the old cache rows are not touched
     np.testing.assert_array_equal(kc1[0, :L], kc[0, :L])
     assert not np.allclose(kc1[0, L:L + Snew], kn[0])
+
+
+# ---------------------------------------------------------------------------
+# ALiBi (alibi_slopes): distance bias -m * |i + off - j|
+# ---------------------------------------------------------------------------
+
+def _geo(n, r):
+    """sum_{d=0}^{n} r^d and sum_{d=0}^{n} d r^d in closed form (n >= 0)."""
+    g0 = (1.0 - r ** (n + 1)) / (1.0 - r)
+    g1 = r * (1.0 - (n + 1) * r ** n + n * r ** (n + 1)) / (1.0 - r) ** 2
+    return g0, g1
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("Sq,Sk", [(9, 9), (4, 9)])
+def test_alibi_geometric_weights_closed_form(causal, Sq, Sk):
+    # q = 0: every raw score is 0 and the weights are r^distance with
+    # r = exp(-m); with V = key index the output is a mean position
+    slopes = np.array([[0.3, 1.1], [0.05, 2.0]])  # (B, Hq)
+    B, H = slopes.shape
+    q = np.zeros((B, Sq, H, 2))
+    k = np.ones((B, Sk, H, 2))
+    v = np.zeros((B, Sk, H, 2))
+    v[:, :, :, 0] = np.arange(Sk)[None, :, None]
+    v[:, :, :, 1] = 1.0
+    o, lse = oracle.attn_fwd(q, k, v, causal=causal, alibi_slopes=slopes)
+    for b in range(B):
+        for h in range(H):
+            r = math.exp(-slopes[b, h])
+            for i in range(Sq):
+                p = i + Sk - Sq
+                g0l, g1l = _geo(p, r)                      # keys p, p-1, ..., 0
+                if causal:
+                    s0, s1 = g0l, -g1l
+                else:
+                    g0r, g1r = _geo(Sk - 1 - p, r)         # keys p, p+1, ..., Sk-1
+                    s0, s1 = g0l + g0r - 1.0, g1r - g1l
+                assert lse[b, h, i] == pytest.approx(math.log(s0), abs=1e-12)
+                assert o[b, i, h, 0] == pytest.approx(p + s1 / s0, abs=1e-12)
+                assert o[b, i, h, 1] == pytest.approx(1.0, abs=1e-12)
+
+
+@pytest.mark.parametrize("wl", [-1, 3])
+def test_alibi_causal_equals_augmented_dot_product(wl):
+    # causal: -m (p - j) = m j - m p; the row constant -m p leaves P alone and
+    # m j is one more dot-product term: q' = [q, 1], k' = [k, m j / scale]
+    rng = np.random.default_rng(40)
+    B, Sq, Sk, H, D, sc = 2, 5, 8, 3, 4, 0.7
+    q, k, v = _rand((B, Sq, H, D), rng), _rand((B, Sk, H, D), rng), _rand((B, Sk, H, D), rng)
+    m = np.array([0.25, 0.5, 1.5])
+    o, lse = oracle.attn_fwd(q, k, v, sc, True, wl, -1, alibi_slopes=m)
+    qa = np.concatenate([q, np.ones((B, Sq, H, 1))], axis=3)
+    ka = np.concatenate([k, (m[None, None, :] * np.arange(Sk)[None, :, None] / sc)[..., None]
+                         * np.ones((B, 1, 1, 1))], axis=3)
+    va = np.concatenate([v, np.zeros((B, Sk, H, 1))], axis=3)
+    oa, la = oracle.attn_fwd(qa, ka, va, sc, True, wl, -1)
+    np.testing.assert_allclose(o, oa[..., :D], rtol=0, atol=1e-12)
+    p = np.arange(Sq) + Sk - Sq
+    np.testing.assert_allclose(lse, la - m[None, :, None] * p[None, None, :], rtol=0, atol=1e-11)
+
+
+def test_alibi_is_added_after_the_softcap():
+    # capped scores lie in [-c, c], so log(P_ij / P_il) differs from the bias
+    # difference by at most 2c, however far apart the keys are
+    rng = np.random.default_rng(41)
+    B, S, H, D, c = 1, 12, 2, 8, 0.5
+    q, k, v = _rand((B, S, H, D), rng, 3.0), _rand((B, S, H, D), rng, 3.0), _rand((B, S, H, D), rng)
+    m = np.array([1.0, 2.5])
+    _, _, P, _ = oracle.attn_fwd(q, k, v, None, False, softcap=c, return_probs=True, alibi_slopes=m)
+    for h in range(H):
+        for i in range(S):
+            bias = -m[h] * np.abs(i - np.arange(S))
+            lr = np.log(P[0, h, i]) - np.log(P[0, h, i, i])
+            assert np.all(np.abs(lr - (bias - bias[i])) <= 2 * c + 1e-12)
+
+
+def test_alibi_zero_slopes_and_rows():
+    rng = np.random.default_rng(42)
+    q, k, v = _rand((2, 6, 4, 8), rng), _rand((2, 9, 2, 8), rng), _rand((2, 9, 2, 8), rng)
+    o0, l0 = oracle.attn_fwd(q, k, v, causal=True)
+    o1, l1 = oracle.attn_fwd(q, k, v, causal=True, alibi_slopes=np.zeros(4))
+    np.testing.assert_array_equal(o0, o1)
+    np.testing.assert_array_equal(l0, l1)
+    # the row-wise form agrees with the whole-matrix form
+    m = np.array([[0.1, 0.2, 0.4, 0.8], [1.0, 0.5, 0.25, 0.125]])
+    o, l = oracle.attn_fwd(q, k, v, None, False, 3, 2, 1.5, alibi_slopes=m)
+    for b, h in ((0, 1), (1, 3)):
+        orow, lrow = oracle.attn_fwd_rows(q, k, v, b, h, np.arange(6), None, False, 3, 2, 1.5, alibi_slopes=m)
+        np.testing.assert_allclose(orow, o[b, :, h], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lrow, l[b, h], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal,cap", [(False, 0.0), (True, 1.5)])
+def test_alibi_gradients_match_finite_differences(causal, cap):
+    rng = np.random.default_rng(43)
+    q, k, v = _rand((2, 4, 2, 3), rng), _rand((2, 5, 1, 3), rng), _rand((2, 5, 1, 3), rng)
+    do = _rand((2, 4, 2, 3), rng)
+    kw = dict(scale=0.6, causal=causal, softcap=cap, alibi_slopes=np.array([[0.3, 0.9], [1.7, 0.1]]))
+
+    def loss(qq, kk, vv):
+        return float((oracle.attn_fwd(qq, kk, vv, **kw)[0] * do).sum())
+
+    dq, dk, dv, _ = oracle.attn_bwd(do, q, k, v, **kw)
+    h = 1e-6
+    for x, g in ((q, dq), (k, dk), (v, dv)):
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = [xp if x is t else t for t in (q, k, v)]
+            args_m = [xm if x is t else t for t in (q, k, v)]
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        err = np.linalg.norm(num - g) / max(np.linalg.norm(g), 1e-30)
+        assert err <= 1e-6, err
+
+
+def test_planted_alibi_sign_is_caught(monkeypatch):
+    orig = attn64.alibi_bias
+    monkeypatch.setattr(attn64, "alibi_bias", lambda m, rows, Sq, Sk: -orig(m, rows, Sq, Sk))
+    with pytest.raises(AssertionError):
+        test_alibi_geometric_weights_closed_form(True, 9, 9)
+
+
+def test_planted_alibi_top_left_alignment_is_caught(monkeypatch):
+    orig = attn64.alibi_bias
+    monkeypatch.setattr(attn64, "alibi_bias", lambda m, rows, Sq, Sk: orig(m, np.asarray(rows) - (Sk - Sq), Sq, Sk))
+    with pytest.raises(AssertionError):
+        test_alibi_geometric_weights_closed_form(False, 4, 9)
