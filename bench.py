@@ -158,10 +158,13 @@ class AttnUnit:
         self.ws = torch.empty(n, dtype=torch.uint8, device=dev)
         self.flops_fwd, self.flops_bwd = attn_flops(cfg)
         self.kw = dict(scale=cfg["scale"], causal=cfg["causal"], window=cfg["window"], softcap=cfg["softcap"])
+        if cfg.get("alibi"):
+            self.kw["alibi_slopes"] = inputs.alibi_slopes(cfg["Hq"]).to(dev)
 
     def name(self):
         c = self.cfg
-        return "H%dD%dS%d%s%s" % (c["Hq"], c["D"], c["Sq"], "c" if c["causal"] else "n", "-det" if self.det else "")
+        return "H%dD%dS%d%s%s%s" % (c["Hq"], c["D"], c["Sq"], "c" if c["causal"] else "n", "-det" if self.det else "",
+                                    "-alibi" if c.get("alibi") else "")
 
     def run(self, tracer):
         api = self.api
@@ -378,6 +381,8 @@ def build_units(dev, workload, point=None):
         units.append(AttnUnit(inputs.fwd_bwd_512_config(), dev))
     if workload == "varlen":
         units.append(VarlenUnit(inputs.varlen_config(), dev))
+    if workload == "alibi":
+        units.append(AttnUnit(inputs.alibi_config(), dev))
     return units
 
 
@@ -519,7 +524,8 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="full", choices=["full", "sweep", "gqa", "decode", "small", "point", "varlen"])
+    ap.add_argument("--workload", default="full", choices=["full", "sweep", "gqa", "decode", "small", "point", "varlen",
+                                                                   "alibi"])
     ap.add_argument("--point", default="H16D128S4096n", help="sweep point for --workload point")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -64,13 +64,25 @@ def _stride_array(tensors):
     return (ctypes.c_longlong * len(vals))(*vals)
 
 
+def _alibi(slopes, B, Hq, device):
+    """(pointer, batch stride) of ALiBi slopes: float32 (Hq,) or (B, Hq)."""
+    if slopes.dtype != torch.float32 or slopes.device != device:
+        raise ValueError("alibi_slopes must be a float32 tensor on the device of q")
+    if slopes.dim() == 1 and slopes.shape == (Hq,) and slopes.is_contiguous():
+        return _ptr(slopes), 0
+    if slopes.dim() == 2 and slopes.shape == (B, Hq) and slopes.stride(1) == 1:
+        return _ptr(slopes), slopes.stride(0)
+    raise ValueError(f"alibi_slopes must be ({Hq},) or ({B}, {Hq}) with contiguous heads")
+
+
 def fa_fwd(q, k, v, out=None, lse=None, scale=None, causal=False, window=(-1, -1), softcap=0.0,
-           stream=None):
+           stream=None, alibi_slopes=None):
     """Forward attention; returns (out, lse).  lse is fp32 (B, Hq, Sq).
 
     q, k, v (and out) may be views with any strides as long as the head
     dimension is contiguous (e.g. slices of a packed qkv tensor); those go
-    through fa_fwd_strided."""
+    through fa_fwd_strided.  ``alibi_slopes`` (float32 (Hq,) or (B, Hq))
+    adds the ALiBi bias through fa_fwd_alibi."""
     lib = _lib.load()
     B, Sq, Hq, D = q.shape
     Sk, Hkv = k.shape[1], k.shape[2]
@@ -87,7 +99,12 @@ def fa_fwd(q, k, v, out=None, lse=None, scale=None, causal=False, window=(-1, -1
     wl, wr = _window(window)
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq, Sk, Hq, Hkv, D, _DT[dt], float(scale or 0.0),
             int(bool(causal)), wl, wr, float(softcap or 0.0))
-    if all(t.is_contiguous() for t in (q, k, v, out)):
+    packed = all(t.is_contiguous() for t in (q, k, v, out))
+    if alibi_slopes is not None:
+        ap, ab = _alibi(alibi_slopes, B, Hq, q.device)
+        code = lib.fa_fwd_alibi(*args, None if packed else _stride_array((q, k, v, out)), ap, ab, _stream(stream))
+        _lib.check(code, "fa_fwd_alibi")
+    elif packed:
         code = lib.fa_fwd(*args, _stream(stream))
         _lib.check(code, "fa_fwd")
     else:
@@ -101,8 +118,9 @@ def fa_bwd_workspace_size(B, Sq, Sk, Hq, Hkv, D, deterministic=False):
 
 
 def fa_bwd(dout, q, k, v, out, lse, dq=None, dk=None, dv=None, scale=None, causal=False,
-           window=(-1, -1), softcap=0.0, deterministic=False, workspace=None, stream=None):
-    """Backward attention; returns (dq, dk, dv)."""
+           window=(-1, -1), softcap=0.0, deterministic=False, workspace=None, stream=None, alibi_slopes=None):
+    """Backward attention; returns (dq, dk, dv).  ``alibi_slopes`` as in
+    :func:`fa_fwd` (the same slopes the forward used)."""
     lib = _lib.load()
     B, Sq, Hq, D = q.shape
     Sk, Hkv = k.shape[1], k.shape[2]
@@ -122,7 +140,12 @@ def fa_bwd(dout, q, k, v, out, lse, dq=None, dk=None, dv=None, scale=None, causa
             Hq, Hkv, D, _DT[dt], float(scale or 0.0), int(bool(causal)), wl, wr, float(softcap or 0.0),
             int(bool(deterministic)), _ptr(workspace), workspace.numel())
     tensors = (dout, q, k, v, out, dq, dk, dv)
-    if all(t.is_contiguous() for t in tensors):
+    packed = all(t.is_contiguous() for t in tensors)
+    if alibi_slopes is not None:
+        ap, ab = _alibi(alibi_slopes, B, Hq, q.device)
+        code = lib.fa_bwd_alibi(*args, None if packed else _stride_array(tensors), ap, ab, _stream(stream))
+        _lib.check(code, "fa_bwd_alibi")
+    elif packed:
         code = lib.fa_bwd(*args, _stream(stream))
         _lib.check(code, "fa_bwd")
     else:

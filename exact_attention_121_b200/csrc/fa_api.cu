@@ -162,14 +162,24 @@ static bool strides_ok(const long long* st, int n) {
   return true;
 }
 
+// ALiBi slopes: null (off), else 4-byte aligned with batch stride 0 (one
+// slope per head) or >= Hq (one row of Hq slopes per batch element)
+static bool alibi_ok(const float* a, int bstride, int Hq) {
+  if (!a) return true;
+  if (reinterpret_cast<uintptr_t>(a) & 3u) return false;
+  return bstride == 0 || bstride >= Hq;
+}
+
 // strides: NULL (packed tensors) or 12 values, (batch, token, head) of q, k, v, out
 static fa_status fwd_impl(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk,
                           int Hq, int Hkv, int D, fa_dtype dt, float scale, int causal, int window_left,
-                          int window_right, float softcap, const long long* strides, fa_stream_t stream) {
+                          int window_right, float softcap, const long long* strides, const float* alibi,
+                          int alibi_bstride, fa_stream_t stream) {
   g_last_launches = 0;
   fa_status st = check_common(B, Sq, Hq, Hkv, D, dt, scale, softcap);
   if (st != FA_OK) return st;
   if (Sk < 0) return FA_ERR_INVALID_ARG;
+  if (!alibi_ok(alibi, alibi_bstride, Hq)) return FA_ERR_INVALID_ARG;
   if (B == 0 || Sq == 0) return FA_OK;
   if (!q || !out || !lse) return FA_ERR_INVALID_ARG;
   if (Sk > 0 && (!k || !v)) return FA_ERR_INVALID_ARG;
@@ -191,16 +201,21 @@ static fa_status fwd_impl(const void* q, const void* k, const void* v, void* out
   fold_window(causal, window_left, window_right, &p.wl, &p.wr);
   scale = resolve_scale(scale, D);
   fill_cap(scale, softcap, &p.softcap, &p.cap_in, &p.cap_log2, &p.scale_log2);
+  p.alibi = alibi;
+  p.alibi_bstride = alibi_bstride;
   p.status = status_ptr();
   if (!p.status) return FA_ERR_CUDA;
   int launches = 0;
   cudaError_t e;
-  // strided tensors run on the tcgen05 kernel only
-  const bool tc = (g_fwd_kernel_choice == 2) || (g_fwd_kernel_choice == 0 && kTcAuto) || strides;
+  // strided tensors and ALiBi run on the tcgen05 kernel only: refused when
+  // the mma.sync kernel is forced
+  const bool tc_only = strides || alibi;
+  if (tc_only && g_fwd_kernel_choice == 1) return FA_ERR_UNSUPPORTED;
+  const bool tc = (g_fwd_kernel_choice == 2) || (g_fwd_kernel_choice == 0 && kTcAuto) || tc_only;
   if (tc && fa::fwd_tc_supported(p)) {
     e = fa::launch_fwd_tc(p, dt, stream, &launches);
   } else {
-    if (g_fwd_kernel_choice == 2 || strides) return FA_ERR_UNSUPPORTED;
+    if (g_fwd_kernel_choice == 2 || tc_only) return FA_ERR_UNSUPPORTED;
     e = fa::launch_fwd_mma(p, dt, stream, &launches);
   }
   g_last_launches = launches;
@@ -212,7 +227,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* 
                  int Hq, int Hkv, int D, fa_dtype dt, float scale, int causal, int window_left, int window_right,
                  float softcap, fa_stream_t stream) {
   return fwd_impl(q, k, v, out, lse, B, Sq, Sk, Hq, Hkv, D, dt, scale, causal, window_left, window_right, softcap,
-                  nullptr, stream);
+                  nullptr, nullptr, 0, stream);
 }
 
 fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk,
@@ -220,7 +235,16 @@ fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* out,
                          int window_right, float softcap, const long long* strides, fa_stream_t stream) {
   if (!strides) return FA_ERR_INVALID_ARG;
   return fwd_impl(q, k, v, out, lse, B, Sq, Sk, Hq, Hkv, D, dt, scale, causal, window_left, window_right, softcap,
-                  strides, stream);
+                  strides, nullptr, 0, stream);
+}
+
+fa_status fa_fwd_alibi(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk,
+                       int Hq, int Hkv, int D, fa_dtype dt, float scale, int causal, int window_left,
+                       int window_right, float softcap, const long long* strides, const float* alibi_slopes,
+                       int alibi_batch_stride, fa_stream_t stream) {
+  if (!alibi_slopes) return FA_ERR_INVALID_ARG;
+  return fwd_impl(q, k, v, out, lse, B, Sq, Sk, Hq, Hkv, D, dt, scale, causal, window_left, window_right, softcap,
+                  strides, alibi_slopes, alibi_batch_stride, stream);
 }
 
 size_t fa_bwd_workspace_size(int B, int Sq, int Sk, int Hq, int Hkv, int D, int deterministic) {
@@ -237,11 +261,12 @@ static fa_status bwd_impl(const void* dout, const void* q, const void* k, const 
                           const float* lse, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int Hq, int Hkv,
                           int D, fa_dtype dt, float scale, int causal, int window_left, int window_right,
                           float softcap, int deterministic, void* workspace, size_t ws_bytes,
-                          const long long* strides, fa_stream_t stream) {
+                          const long long* strides, const float* alibi, int alibi_bstride, fa_stream_t stream) {
   g_last_launches = 0;
   fa_status st = check_common(B, Sq, Hq, Hkv, D, dt, scale, softcap);
   if (st != FA_OK) return st;
   if (Sk < 0) return FA_ERR_INVALID_ARG;
+  if (!alibi_ok(alibi, alibi_bstride, Hq)) return FA_ERR_INVALID_ARG;
   if (B == 0 || (Sq == 0 && Sk == 0)) return FA_OK;
   const void* ptrs[] = {dout, q, k, v, out, lse, dq, dk, dv, workspace};
   for (const void* ptr : ptrs)
@@ -288,8 +313,10 @@ static fa_status bwd_impl(const void* dout, const void* q, const void* k, const 
   fill_cap(scale, softcap, &p.softcap, &p.cap_in, &p.cap_log2, &p.scale_log2);
   p.deterministic = deterministic ? 1 : 0;
   p.kernel_choice = g_bwd_kernel_choice;
-  // strided tensors run on the tcgen05 kernel only
-  if (strides) {
+  p.alibi = alibi;
+  p.alibi_bstride = alibi_bstride;
+  // strided tensors and ALiBi run on the tcgen05 kernel only
+  if (strides || alibi) {
     if (g_bwd_kernel_choice == 1) return FA_ERR_UNSUPPORTED;
     p.kernel_choice = 2;
   }
@@ -307,7 +334,7 @@ fa_status fa_bwd(const void* dout, const void* q, const void* k, const void* v, 
                  float scale, int causal, int window_left, int window_right, float softcap, int deterministic,
                  void* workspace, size_t ws_bytes, fa_stream_t stream) {
   return bwd_impl(dout, q, k, v, out, lse, dq, dk, dv, B, Sq, Sk, Hq, Hkv, D, dt, scale, causal, window_left,
-                  window_right, softcap, deterministic, workspace, ws_bytes, nullptr, stream);
+                  window_right, softcap, deterministic, workspace, ws_bytes, nullptr, nullptr, 0, stream);
 }
 
 fa_status fa_bwd_strided(const void* dout, const void* q, const void* k, const void* v, const void* out,
@@ -317,7 +344,18 @@ fa_status fa_bwd_strided(const void* dout, const void* q, const void* k, const v
                          const long long* strides, fa_stream_t stream) {
   if (!strides) return FA_ERR_INVALID_ARG;
   return bwd_impl(dout, q, k, v, out, lse, dq, dk, dv, B, Sq, Sk, Hq, Hkv, D, dt, scale, causal, window_left,
-                  window_right, softcap, deterministic, workspace, ws_bytes, strides, stream);
+                  window_right, softcap, deterministic, workspace, ws_bytes, strides, nullptr, 0, stream);
+}
+
+fa_status fa_bwd_alibi(const void* dout, const void* q, const void* k, const void* v, const void* out,
+                       const float* lse, void* dq, void* dk, void* dv, int B, int Sq, int Sk, int Hq, int Hkv, int D,
+                       fa_dtype dt, float scale, int causal, int window_left, int window_right, float softcap,
+                       int deterministic, void* workspace, size_t ws_bytes, const long long* strides,
+                       const float* alibi_slopes, int alibi_batch_stride, fa_stream_t stream) {
+  if (!alibi_slopes) return FA_ERR_INVALID_ARG;
+  return bwd_impl(dout, q, k, v, out, lse, dq, dk, dv, B, Sq, Sk, Hq, Hkv, D, dt, scale, causal, window_left,
+                  window_right, softcap, deterministic, workspace, ws_bytes, strides, alibi_slopes,
+                  alibi_batch_stride, stream);
 }
 
 // ---------------------------------------------------------------- packed batches

@@ -86,7 +86,7 @@ struct BwdTcCfg {
 
 __device__ __forceinline__ float f32(uint32_t u) { return __uint_as_float(u); }
 
-template <typename T, int D_, bool kCap>
+template <typename T, int D_, bool kCap, bool kAlibi>
 __global__ void __launch_bounds__(kThreadsB, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -363,7 +363,8 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       const int x = it & 1, u = it >> 1;
       int h, q0;
       iter_q(it, h, q0);
-      (void)h;
+      // ALiBi slope of (b, h) as a log2-domain factor of |qpos - key|
+      const float mb = kAlibi ? -kLog2e * p.alibi[(long long)b * p.alibi_bstride + h] : 0.f;
       // S^T/dP^T(it) ready also means (commit order) that the products of
       // it-2 that read this TMEM buffer and the dQ^T that read this dS
       // buffer are done
@@ -398,6 +399,12 @@ __global__ void __launch_bounds__(kThreadsB, 1)
           const float4 a4 = nl4[j], b4 = dl4[j];
           nl[4 * j] = a4.x; nl[4 * j + 1] = a4.y; nl[4 * j + 2] = a4.z; nl[4 * j + 3] = a4.w;
           dlv[4 * j] = b4.x; dlv[4 * j + 1] = b4.y; dlv[4 * j + 2] = b4.z; dlv[4 * j + 3] = b4.w;
+        }
+        if (kAlibi) {
+          // the distance bias joins -LSE*log2e: query q0 + q16 + c
+          const float d0 = (float)(q0 + q16 + off - key);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) nl[c] = fmaf(mb, fabsf(d0 + (float)c), nl[c]);
         }
         tmem_wait_ld();
         reg_fence(s);
@@ -588,10 +595,10 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   }
 }
 
-template <typename T, int D, bool kCap>
+template <typename T, int D, bool kCap, bool kAlibi>
 cudaError_t launch_t(const BwdParams& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                      const CUtensorMap& mdo, const CUtensorMap& mdq, cudaStream_t s) {
-  auto kern = bwd_tc_kernel<T, D, kCap>;
+  auto kern = bwd_tc_kernel<T, D, kCap, kAlibi>;
   constexpr int smem = BwdTcCfg<D>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -603,6 +610,24 @@ cudaError_t launch_t(const BwdParams& p, const CUtensorMap& mq, const CUtensorMa
   kern<<<(unsigned)items, kThreadsB, smem, s>>>(mq, mk, mv, mdo, mdq, p);
   trace_end(s);
   return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_d(const BwdParams& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                     const CUtensorMap& mdo, const CUtensorMap& mdq, cudaStream_t s) {
+  const bool cap = p.softcap > 0.f;
+  if (p.alibi) {
+    if (p.D == 64)
+      return cap ? launch_t<T, 64, true, true>(p, mq, mk, mv, mdo, mdq, s)
+                 : launch_t<T, 64, false, true>(p, mq, mk, mv, mdo, mdq, s);
+    return cap ? launch_t<T, 128, true, true>(p, mq, mk, mv, mdo, mdq, s)
+               : launch_t<T, 128, false, true>(p, mq, mk, mv, mdo, mdq, s);
+  }
+  if (p.D == 64)
+    return cap ? launch_t<T, 64, true, false>(p, mq, mk, mv, mdo, mdq, s)
+               : launch_t<T, 64, false, false>(p, mq, mk, mv, mdo, mdq, s);
+  return cap ? launch_t<T, 128, true, false>(p, mq, mk, mv, mdo, mdq, s)
+             : launch_t<T, 128, false, false>(p, mq, mk, mv, mdo, mdq, s);
 }
 
 }  // namespace
@@ -622,15 +647,7 @@ cudaError_t launch_bwd_main_tc(const BwdParams& p, fa_dtype dt, cudaStream_t s) 
       !make_bshd_map_strided(&mv, p.v, bf, p.D, p.Hkv, mk_s, mb, p.st_v, kKeys) ||
       !make_bshd_map_f32(&mdq, p.dq_accum, p.D, p.Hq, mq_s, mb, kQ))
     return cudaErrorNotSupported;
-  const bool cap = p.softcap > 0.f;
-  if (p.D == 64) {
-    if (bf) return cap ? launch_t<__nv_bfloat16, 64, true>(p, mq, mk, mv, mdo, mdq, s)
-                       : launch_t<__nv_bfloat16, 64, false>(p, mq, mk, mv, mdo, mdq, s);
-    return cap ? launch_t<__half, 64, true>(p, mq, mk, mv, mdo, mdq, s) : launch_t<__half, 64, false>(p, mq, mk, mv, mdo, mdq, s);
-  }
-  if (bf) return cap ? launch_t<__nv_bfloat16, 128, true>(p, mq, mk, mv, mdo, mdq, s)
-                     : launch_t<__nv_bfloat16, 128, false>(p, mq, mk, mv, mdo, mdq, s);
-  return cap ? launch_t<__half, 128, true>(p, mq, mk, mv, mdo, mdq, s) : launch_t<__half, 128, false>(p, mq, mk, mv, mdo, mdq, s);
+  return bf ? launch_d<__nv_bfloat16>(p, mq, mk, mv, mdo, mdq, s) : launch_d<__half>(p, mq, mk, mv, mdo, mdq, s);
 }
 
 }  // namespace fa

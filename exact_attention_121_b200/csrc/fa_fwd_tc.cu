@@ -91,7 +91,7 @@ struct TcCfg {
 
 __device__ __forceinline__ float f32(uint32_t u) { return __uint_as_float(u); }
 
-template <typename T, int D, bool kCap>
+template <typename T, int D, bool kCap, bool kAlibi>
 __global__ void __launch_bounds__(kThreadsTC, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -127,6 +127,16 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   if (p.wr >= 0) kmax = min(kmax, qlast + off + p.wr);
   const int kt_begin = kmin / kRows;
   const int n_tiles = (kmax >= kmin) ? (kmax / kRows + 1 - kt_begin) : 0;
+  // Key-tile order.  Plain: ascending.  ALiBi: the tile at the diagonal of
+  // the CTA's rows first, then the rest in ascending order from the far end,
+  // so the running maximum is set at once and the (lower) bias of later
+  // tiles rarely moves it: few rescales of O.  The result does not depend
+  // on the order.
+  const int rot = kAlibi ? min(max((q0 + off + kRows) / kRows - kt_begin, 0), max(n_tiles - 1, 0)) : 0;
+  auto tile_k0 = [&](int j) {
+    const int t = (j + rot < n_tiles) ? j + rot : j + rot - n_tiles;
+    return (kt_begin + t) * kRows;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::B_Q), 1);
@@ -178,7 +188,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       for (int j = 0; j < n_tiles; ++j) {
         const int sk = j % C::NSK, uk = j / C::NSK;
         const int sv = j % C::NSV, uv = j / C::NSV;
-        const int k0 = (kt_begin + j) * kRows;
+        const int k0 = tile_k0(j);
         if (j >= C::NSK && !mbar_wait(bar(C::B_KE + sk), (uk - 1) & 1, abort_flag, kTcWaitNs)) {
           fail();
           break;
@@ -332,6 +342,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     const int qpos = qi + off;
     const int qpos_first = q0 + off, qpos_last = qlast + off;
     float m_run = -INFINITY, l_run = 0.f, l_q = 0.f;
+    // ALiBi slope of this (b, h), as a log2-domain factor of |qpos - key|
+    const float mb = kAlibi ? -kLog2e * p.alibi[(long long)b * p.alibi_bstride + h] : 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       // warp-uniform outcome: the TMEM accesses below are warp-collective
@@ -352,7 +364,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         tc_fence_before();
         mbar_arrive(bar(C::B_SF + t));
       }
-      const int k0 = (kt_begin + j) * kRows;
+      const int k0 = tile_k0(j);
       const bool full = (k0 + kRows <= Sk) && (p.wl < 0 || k0 >= qpos_last - p.wl) &&
                         (p.wr < 0 || k0 + kRows - 1 <= qpos_first + p.wr);
       // row maximum in the log2 domain (the scale is positive: max commutes)
@@ -360,6 +372,25 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       if (kCap) {
 #pragma unroll
         for (int i = 0; i < kRows; ++i) s[i] = __float_as_uint(p.cap_log2 * tanh_exp(f32(s[i]) * p.cap_in));
+      }
+      if (kAlibi) {
+        // to the log2 domain, plus the distance bias mb |qpos - key| of key
+        // k0 + i.  A tile on one side of every row of the warp has a bias
+        // linear in i: t0 + step i, one fma per key (without the softcap:
+        // beside the tanh the second copy of the loop costs spills).
+        const float in = kCap ? 1.f : p.scale_log2;
+        const bool left = !kCap && __all_sync(0xffffffffu, k0 + kRows - 1 <= qpos);
+        const bool right = !kCap && __all_sync(0xffffffffu, k0 >= qpos);
+        if (left || right) {
+          const float t0 = mb * fabsf((float)(qpos - k0));
+          const float step = left ? -mb : mb;
+#pragma unroll
+          for (int i = 0; i < kRows; ++i) s[i] = __float_as_uint(fmaf(f32(s[i]), in, fmaf(step, (float)i, t0)));
+        } else {
+          const float d0 = (float)(qpos - k0);
+#pragma unroll
+          for (int i = 0; i < kRows; ++i) s[i] = __float_as_uint(fmaf(f32(s[i]), in, mb * fabsf(d0 - (float)i)));
+        }
       }
       if (!full) {
 #pragma unroll
@@ -380,7 +411,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
         mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       }
-      const float sl = kCap ? 1.f : p.scale_log2;  // multiplier into the log2 domain
+      const float sl = (kCap || kAlibi) ? 1.f : p.scale_log2;  // multiplier into the log2 domain
       mx *= sl;
       // lazy rescale: move the running max only when it grows by > 2^8
       const bool move = (mx > m_run + kRescaleLog2) || (m_run == -INFINITY && mx != -INFINITY);
@@ -501,10 +532,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 // host side
 // ---------------------------------------------------------------------------
 
-template <typename T, int D, bool kCap>
+template <typename T, int D, bool kCap, bool kAlibi>
 cudaError_t launch_t(const FwdParams& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                      cudaStream_t s) {
-  auto kern = fwd_tc_kernel<T, D, kCap>;
+  auto kern = fwd_tc_kernel<T, D, kCap, kAlibi>;
   constexpr int smem = TcCfg<D>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -521,8 +552,14 @@ template <typename T>
 cudaError_t launch_dt(const FwdParams& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       cudaStream_t s) {
   const bool cap = p.softcap > 0.f;
-  if (p.D == 64) return cap ? launch_t<T, 64, true>(p, mq, mk, mv, s) : launch_t<T, 64, false>(p, mq, mk, mv, s);
-  return cap ? launch_t<T, 128, true>(p, mq, mk, mv, s) : launch_t<T, 128, false>(p, mq, mk, mv, s);
+  if (p.alibi) {
+    if (p.D == 64)
+      return cap ? launch_t<T, 64, true, true>(p, mq, mk, mv, s) : launch_t<T, 64, false, true>(p, mq, mk, mv, s);
+    return cap ? launch_t<T, 128, true, true>(p, mq, mk, mv, s) : launch_t<T, 128, false, true>(p, mq, mk, mv, s);
+  }
+  if (p.D == 64)
+    return cap ? launch_t<T, 64, true, false>(p, mq, mk, mv, s) : launch_t<T, 64, false, false>(p, mq, mk, mv, s);
+  return cap ? launch_t<T, 128, true, false>(p, mq, mk, mv, s) : launch_t<T, 128, false, false>(p, mq, mk, mv, s);
 }
 
 }  // namespace

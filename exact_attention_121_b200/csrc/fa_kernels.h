@@ -32,6 +32,10 @@ struct FwdParams {
   // element strides (batch, token, head) of q, k, v, out; the head dimension
   // is contiguous.  Packed batches have batch stride 0.
   long long st_q[3], st_k[3], st_v[3], st_o[3];
+  // ALiBi: slope of (batch b, q-head h) at alibi[b * alibi_bstride + h]
+  // (bstride 0: one slope per head for the whole batch); null = off
+  const float* alibi;
+  int alibi_bstride;
 };
 
 struct BwdParams {
@@ -65,6 +69,8 @@ struct BwdParams {
   // workspace tensors (dq_accum, delta) are always packed
   long long st_do[3], st_q[3], st_k[3], st_v[3], st_o[3], st_dq[3], st_dk[3], st_dv[3];
   int rows_packed;       // dout, out and dq are packed (token, head) rows: plain indexing
+  const float* alibi;    // ALiBi slopes as in FwdParams; null = off
+  int alibi_bstride;
 };
 
 struct DecodeParams {

@@ -47,6 +47,15 @@ def attention_inputs(B, Sq, Sk, Hq, Hkv, D, dtype="bf16", seed=0, amp=1.0, with_
     return q, k, v, dout
 
 
+def alibi_slopes(Hq, B=None, seed=None):
+    """ALiBi slopes, float32: the geometric sequence 2^(-8 (h+1) / Hq) of
+    the ALiBi paper shared by the batch (shape (Hq,)), or with ``B`` and
+    ``seed`` seeded draws U(0, 1) per (batch row, head) (shape (B, Hq))."""
+    if B is None:
+        return torch.tensor([2.0 ** (-8.0 * (h + 1) / Hq) for h in range(Hq)], dtype=torch.float32)
+    return torch.rand((B, Hq), generator=_gen(seed), dtype=torch.float32)
+
+
 def kvcache_inputs(B, Hq, Hkv, D, page_size, pages_per_seq, max_len, Sq=1, Snew=1,
                    dtype="bf16", seed=5, num_pages=None, paged=True, min_len=1,
                    seqlens=None):
@@ -153,3 +162,11 @@ def varlen_config():
     lens = varlen_lengths(32, 64, 1024, seed=6)
     return dict(lens=lens, Hq=16, Hkv=16, D=128, dtype="bf16", causal=True, window=(-1, -1), softcap=0.0,
                 scale=1.0 / math.sqrt(128), seed=7, amp=1.0)
+
+
+def alibi_config():
+    """ALiBi at hidden 2048: B=4, S=4096, Hq=Hkv=16, D=128, bf16, causal, the
+    geometric slopes of :func:`alibi_slopes`; the shape of the seqlen-sweep
+    point H16 D128 S4096 causal (seed 8)."""
+    return dict(B=4, Sq=4096, Sk=4096, Hq=16, Hkv=16, D=128, dtype="bf16", causal=True, window=(-1, -1),
+                softcap=0.0, scale=1.0 / math.sqrt(128), seed=8, amp=1.0, alibi=True)

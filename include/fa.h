@@ -186,6 +186,37 @@ fa_status fa_bwd_strided(const void* dout, const void* q, const void* k, const v
                          int deterministic, void* workspace, size_t ws_bytes,
                          const long long* strides, fa_stream_t stream);
 
+/*
+ * fa_fwd with ALiBi ("FlashAttention 实战指南", advanced parameters:
+ * alibi_slopes, a position bias that lowers the scores of distant keys).
+ * Query row i of (b, h) and key j get the bias -m * |i + Sk - Sq - j| added
+ * to the (soft-capped) scaled score before the mask, m = alibi_slopes[b *
+ * alibi_batch_stride + h]: a device float32 array, 4-byte aligned, borrowed
+ * for the call.  alibi_batch_stride is 0 (one slope per q-head for the whole
+ * batch, Hq values) or >= Hq (one row of Hq slopes per batch element);
+ * anything else, or a null alibi_slopes, gives FA_ERR_INVALID_ARG.  LSE
+ * includes the bias.  `strides` is NULL (packed tensors) or as in
+ * fa_fwd_strided.  tcgen05 kernel only.
+ */
+fa_status fa_fwd_alibi(const void* q, const void* k, const void* v, void* out, float* lse,
+                       int B, int Sq, int Sk, int Hq, int Hkv, int D, fa_dtype dt,
+                       float scale, int causal, int window_left, int window_right, float softcap,
+                       const long long* strides, const float* alibi_slopes, int alibi_batch_stride,
+                       fa_stream_t stream);
+
+/*
+ * fa_bwd of fa_fwd_alibi: the same slopes, and lse from fa_fwd_alibi.  The
+ * bias is a constant of the inputs, so the gradients flow as in fa_bwd with
+ * P recomputed including it.  `strides` is NULL or as in fa_bwd_strided;
+ * the workspace is fa_bwd_workspace_size.  tcgen05 kernel only.
+ */
+fa_status fa_bwd_alibi(const void* dout, const void* q, const void* k, const void* v,
+                       const void* out, const float* lse, void* dq, void* dk, void* dv,
+                       int B, int Sq, int Sk, int Hq, int Hkv, int D, fa_dtype dt,
+                       float scale, int causal, int window_left, int window_right, float softcap,
+                       int deterministic, void* workspace, size_t ws_bytes, const long long* strides,
+                       const float* alibi_slopes, int alibi_batch_stride, fa_stream_t stream);
+
 /* Largest split count fa_fwd_kvcache accepts; num_splits <= 0 picks one. */
 #define FA_MAX_SPLITS 64
 
@@ -306,16 +337,19 @@ fa_status fa_last_device_status(fa_stream_t stream);
 /*
  * Which forward kernel fa_fwd runs: 0 = automatic, 1 = the warp-level
  * mma.sync kernel, 2 = the tensor-memory tcgen05 kernel (fa_fwd returns
- * FA_ERR_UNSUPPORTED where it does not apply).  Process wide; meant for tests
+ * FA_ERR_UNSUPPORTED where it does not apply).  The calls that exist on the
+ * tcgen05 kernel only (strided, varlen, ALiBi) return FA_ERR_UNSUPPORTED
+ * under 1 rather than run another kernel.  Process wide; meant for tests
  * and benchmarks that compare the two.
  */
 void fa_set_fwd_kernel(int which);
 
 /*
  * Which main backward kernel fa_bwd runs: 0 = automatic, 1 = the warp-level
- * mma.sync kernel, 2 = the tensor-memory tcgen05 kernel (head dim 128, atomic
- * dQ mode; fa_bwd returns FA_ERR_CUDA where it does not apply).  Process wide;
- * meant for tests and benchmarks.
+ * mma.sync kernel, 2 = the tensor-memory tcgen05 kernel (head dim 64 and
+ * 128, atomic and ordered dQ).  The tcgen05-only calls (strided, varlen,
+ * ALiBi) return FA_ERR_UNSUPPORTED under 1.  Process wide; meant for tests
+ * and benchmarks.
  */
 void fa_set_bwd_kernel(int which);
 

@@ -136,3 +136,19 @@ def test_strided_and_varlen_host_validation(lib):
     # the packed workspace is linear in the token count
     w = [lib.fa_bwd_varlen_workspace_size(8, 1024, T, 16, 128, 0) for T in (4096, 8192)]
     assert abs(w[1] / w[0] - 2.0) < 0.01
+
+
+def test_alibi_host_validation(lib):
+    p = ctypes.c_void_p(0x1000)
+    fwd = lambda a, bs, Hq=4, B=1: lib.fa_fwd_alibi(p, p, p, p, p, B, 8, 8, Hq, 2, 64, 1, 0.0, 0, -1, -1, 0.0,
+                                                    None, a, bs, None)
+    assert fwd(None, 0) == _lib.FA_ERR_INVALID_ARG               # slopes are required
+    assert fwd(ctypes.c_void_p(0x1002), 0) == _lib.FA_ERR_INVALID_ARG  # not 4-byte aligned
+    assert fwd(p, 2) == _lib.FA_ERR_INVALID_ARG                  # batch stride between 0 and Hq
+    assert fwd(p, -4) == _lib.FA_ERR_INVALID_ARG
+    assert fwd(p, 0, B=0) == _lib.FA_OK                          # empty batch: nothing to do
+    assert fwd(p, 4, B=0) == _lib.FA_OK
+    bwd = lambda a, bs: lib.fa_bwd_alibi(p, p, p, p, p, p, p, p, p, 1, 8, 8, 4, 2, 64, 1, 0.0, 0, -1, -1, 0.0, 0,
+                                         ctypes.c_void_p(0x10000), 1 << 20, None, a, bs, None)
+    assert bwd(None, 0) == _lib.FA_ERR_INVALID_ARG
+    assert bwd(p, 3) == _lib.FA_ERR_INVALID_ARG
