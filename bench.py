@@ -256,7 +256,13 @@ class DecodeUnit:
         self.sl, self.bt = d["cache_seqlens"].to(dev), d["block_table"].to(dev)
         self.out = torch.empty_like(self.q)
         self.lse = torch.empty(cfg["B"], cfg["Hq"], 1, device=dev)
-        n = api.fa_kvcache_workspace_size(cfg["B"], 1, cfg["Hq"], cfg["D"], num_splits)
+        self.rot = {}
+        if cfg.get("rotary"):
+            cos, sin = inputs.rotary_tables(cfg["max_len"] + 1, cfg["D"])
+            self.rot = dict(rotary_cos=cos.to(dev), rotary_sin=sin.to(dev))
+            n = api.fa_kvcache_rotary_workspace_size(cfg["B"], 1, cfg["Hq"], cfg["D"], num_splits)
+        else:
+            n = api.fa_kvcache_workspace_size(cfg["B"], 1, cfg["Hq"], cfg["D"], num_splits)
         self.ws = torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
         lens = d["cache_seqlens"].numpy().astype(np.int64) + 1
         # algorithmic bytes: every attended K and V row once, plus q/out/new rows and the block table
@@ -266,14 +272,14 @@ class DecodeUnit:
         self.flops_dec = int(4 * cfg["D"] * cfg["Hq"] * lens.sum())
 
     def name(self):
-        return "decode"
+        return "decode-rotary" if self.rot else "decode"
 
     def run(self, tracer):
         tracer.arm("decode", self)
         self.api.fa_fwd_kvcache(self.q, self.kc, self.vc, self.kn, self.vn, self.sl, self.bt,
                                 page_size=self.cfg["page_size"], out=self.out, lse=self.lse,
                                 scale=self.cfg["scale"], causal=True, num_splits=self.num_splits,
-                                workspace=self.ws)
+                                workspace=self.ws, **self.rot)
         tracer.disarm()
         return self.api.fa_last_launch_count()
 
@@ -381,6 +387,8 @@ def build_units(dev, workload, point=None):
         units.append(AttnUnit(inputs.fwd_bwd_512_config(), dev))
     if workload == "varlen":
         units.append(VarlenUnit(inputs.varlen_config(), dev))
+    if workload == "decode_rotary":
+        units.append(DecodeUnit(inputs.paged_decode_rotary_config(), dev))
     if workload == "alibi":
         units.append(AttnUnit(inputs.alibi_config(), dev))
     return units
@@ -525,7 +533,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="full", choices=["full", "sweep", "gqa", "decode", "small", "point", "varlen",
-                                                                   "alibi"])
+                                                                   "alibi", "decode_rotary"])
     ap.add_argument("--point", default="H16D128S4096n", help="sweep point for --workload point")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -246,6 +246,10 @@ def fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits):
     return int(_lib.load().fa_kvcache_workspace_size(B, Sq, Hq, D, int(num_splits)))
 
 
+def fa_kvcache_rotary_workspace_size(B, Sq, Hq, D, num_splits):
+    return int(_lib.load().fa_kvcache_rotary_workspace_size(B, Sq, Hq, D, num_splits))
+
+
 def fa_fwd_kvcache(q, k_cache, v_cache, k_new=None, v_new=None, cache_seqlens=None, block_table=None,
                    page_size=256, out=None, lse=None, scale=None, causal=False, window=(-1, -1),
                    softcap=0.0, num_splits=0, workspace=None, stream=None, return_lse=True, rotary_cos=None,

@@ -56,6 +56,16 @@ def alibi_slopes(Hq, B=None, seed=None):
     return torch.rand((B, Hq), generator=_gen(seed), dtype=torch.float32)
 
 
+def rotary_tables(n_pos, rotary_dim, base=10000.0):
+    """Float32 (n_pos, rotary_dim/2) cos/sin tables of the usual rotary
+    frequencies base^(-2j/rotary_dim) at positions 0..n_pos-1 (inputs of the
+    kvcache call, like the caches; no draws)."""
+    half = rotary_dim // 2
+    inv = base ** (-torch.arange(half, dtype=torch.float64) / half)
+    ang = torch.arange(n_pos, dtype=torch.float64)[:, None] * inv[None, :]
+    return torch.cos(ang).float(), torch.sin(ang).float()
+
+
 def kvcache_inputs(B, Hq, Hkv, D, page_size, pages_per_seq, max_len, Sq=1, Snew=1,
                    dtype="bf16", seed=5, num_pages=None, paged=True, min_len=1,
                    seqlens=None):
@@ -170,3 +180,11 @@ def alibi_config():
     point H16 D128 S4096 causal (seed 8)."""
     return dict(B=4, Sq=4096, Sk=4096, Hq=16, Hkv=16, D=128, dtype="bf16", causal=True, window=(-1, -1),
                 softcap=0.0, scale=1.0 / math.sqrt(128), seed=8, amp=1.0, alibi=True)
+
+
+def paged_decode_rotary_config():
+    """The paged-decode workload with rotary tables over the full head dim
+    (halves pairing, base 10000, positions up to 32768 + 1)."""
+    cfg = paged_decode_config()
+    cfg["rotary"] = True
+    return cfg
