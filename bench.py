@@ -43,8 +43,8 @@ ROOFLINE_UNIT = {"fwd": "H16D128S4096n", "bwd": "H16D128S4096n", "decode": "deco
 # (profiles/*_H16D128S4096n.md, profiles/decode_tma_kernel_paged_B8.md).  An
 # entry must be removed whenever its kernel changes.
 TRAFFIC_PER_LAUNCH = {
-    ("fwd", "H16D128S4096n"): 201.683712e6 + 51.086592e6,
-    ("bwd", "H16D128S4096n"): 416.537088e6 + 236.700928e6,
+    ("fwd", "H16D128S4096n"): 201.704960e6 + 53.250816e6,
+    ("bwd", "H16D128S4096n"): 415.648512e6 + 231.981824e6,
     ("decode", "decode"): 521.946368e6 + 7.995904e6,
 }
 
