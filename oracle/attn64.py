@@ -25,6 +25,9 @@ there, so each function states the reading it implements):
 * same page, advanced parameters: ``alibi_slopes`` adds an ALiBi position
   bias that lowers the scores of distant keys, instead of an explicit
   position encoding.  -> :func:`alibi_bias`.
+* same page, versions: FlashAttention-3 adds an FP8 forward (and an AMD
+  backend's fp8 path keeps precision while lowering bandwidth).
+  -> :func:`attn_fwd_fp8`.
 * same page, the three techniques: tiling, online softmax (running row max and
   running sum updated block by block), recomputation in the backward.
   -> :func:`attn_fwd_online` (used only to pin :func:`attn_fwd`).
@@ -52,6 +55,10 @@ Readings where the pages are silent:
   gains ``-m * |i + off - j|`` (``off`` of the bottom-right alignment),
   added after the soft cap and before the mask; slopes are (Hq,) shared by
   the batch or (B, Hq).
+* FP8 forward: q, k, v are OCP FP8 E4M3 codes; each of the three tensors
+  has one float32 descale factor per (batch, kv-head) (a q-head uses the
+  factor of the kv-head it reads), default 1; the real inputs are code value
+  times factor, and the output is the exact attention of those real inputs.
 * varlen: sequences packed along the token axis with ``cu_seqlens`` offsets
   (sequence b is tokens ``cu[b] .. cu[b+1]-1``); each sequence is attended on
   its own, with the masks and the bottom-right alignment of its own lengths;
@@ -540,3 +547,41 @@ def attn_bwd_varlen(dout, q, k, v, cu_seqlens_q, cu_seqlens_k, scale=None, causa
         dq[q0:q1], dk[k0:k1], dv[k0:k1] = g[0][0], g[1][0], g[2][0]
     return dq, dk, dv
 
+
+# ---------------------------------------------------------------------------
+# FP8 (E4M3) forward
+# ---------------------------------------------------------------------------
+
+def e4m3_decode(codes):
+    """Float64 values of OCP FP8 E4M3 codes (uint8): sign in bit 7, a 4-bit
+    exponent (bits 6..3, bias 7) and a 3-bit mantissa; exponent 0 holds the
+    subnormals m * 2^-9; S.1111.111 is NaN and there is no infinity, so the
+    largest finite magnitude is 1.75 * 2^8 = 448."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2((e - 7).astype(np.float64)))
+    mag = np.where((e == 15) & (c & 0x7 == 7), np.nan, mag)
+    return sign * mag
+
+
+def attn_fwd_fp8(q8, k8, v8, descale_q=None, descale_k=None, descale_v=None, scale=None, causal=False,
+                 window_left=-1, window_right=-1, softcap=0.0):
+    """FP8 forward: q8 (B, Sq, Hq, D), k8/v8 (B, Sk, Hkv, D) E4M3 codes; the
+    descales are (B, Hkv) float arrays or None (factor 1).  Returns O and
+    LSE of :func:`attn_fwd` on the real inputs code * factor."""
+    q = e4m3_decode(q8)
+    k = e4m3_decode(k8)
+    v = e4m3_decode(v8)
+    B, Hq, Hkv = q.shape[0], q.shape[2], k.shape[2]
+    G = _check_heads(Hq, Hkv)
+
+    def fac(d, heads_per_factor, H):
+        if d is None:
+            return np.ones((B, 1, H, 1))
+        d = np.asarray(d, np.float64).reshape(B, Hkv)
+        return np.repeat(d, heads_per_factor, axis=1)[:, None, :, None]
+
+    return attn_fwd(q * fac(descale_q, G, Hq), k * fac(descale_k, 1, Hkv), v * fac(descale_v, 1, Hkv), scale,
+                    causal, window_left, window_right, softcap)

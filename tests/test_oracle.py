@@ -719,3 +719,94 @@ def test_planted_alibi_top_left_alignment_is_caught(monkeypatch):
     monkeypatch.setattr(attn64, "alibi_bias", lambda m, rows, Sq, Sk: orig(m, np.asarray(rows) - (Sk - Sq), Sq, Sk))
     with pytest.raises(AssertionError):
         test_alibi_geometric_weights_closed_form(False, 4, 9)
+
+
+# ---------------------------------------------------------------------------
+# FP8 E4M3 forward
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("code,value", [(0x00, 0.0), (0x01, 2.0 ** -9), (0x07, 7 * 2.0 ** -9), (0x08, 2.0 ** -6),
+                                        (0x38, 1.0), (0x3C, 1.5), (0x40, 2.0), (0x46, 3.5), (0x4B, 5.5), (0x7E, 448.0),
+                                        (0xB8, -1.0), (0xFE, -448.0)])
+def test_e4m3_known_codes(code, value):
+    # sign | exponent (bias 7) | 3-bit mantissa, worked by hand
+    assert oracle.e4m3_decode(np.array([code], np.uint8))[0] == value
+
+
+def test_e4m3_nan_and_negative_zero():
+    v = oracle.e4m3_decode(np.array([0x7F, 0xFF, 0x80], np.uint8))
+    assert np.isnan(v[0]) and np.isnan(v[1])
+    assert v[2] == 0.0 and math.copysign(1.0, v[2]) < 0
+
+
+def test_e4m3_decode_matches_torch_float8():
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    mine = oracle.e4m3_decode(codes)
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    np.testing.assert_array_equal(np.isnan(mine), np.isnan(lib))
+    fin = ~np.isnan(lib)
+    np.testing.assert_array_equal(mine[fin], lib[fin])
+
+
+def _codes(shape, rng):
+    # finite codes only (NaN codes 0x7F/0xFF excluded), magnitudes up to 8
+    c = rng.integers(0, 0x58, size=shape).astype(np.uint8)
+    return np.where(rng.random(shape) < 0.5, c | 0x80, c).astype(np.uint8)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_zero_queries_give_uniform_weights(causal):
+    # q = 0: every visible key gets the same weight, O is the mean of the
+    # visible V rows (times the V factor) and LSE = log(number visible)
+    rng = np.random.default_rng(60)
+    B, Sq, Sk, H, D = 2, 3, 7, 2, 4
+    q8 = np.zeros((B, Sq, H, D), np.uint8)
+    k8, v8 = _codes((B, Sk, H, D), rng), _codes((B, Sk, H, D), rng)
+    dv = np.array([[0.5, 2.0], [3.0, 0.25]])
+    o, lse = oracle.attn_fwd_fp8(q8, k8, v8, descale_v=dv, causal=causal)
+    vals = oracle.e4m3_decode(v8)
+    for b in range(B):
+        for h in range(H):
+            for i in range(Sq):
+                n = i + Sk - Sq + 1 if causal else Sk
+                np.testing.assert_allclose(o[b, i, h], dv[b, h] * vals[b, :n, h].mean(axis=0), rtol=0, atol=1e-12)
+                assert lse[b, h, i] == pytest.approx(math.log(n), abs=1e-12)
+
+
+def test_fp8_descales_act_per_batch_and_kv_head():
+    # the q and k factors of (b, kv-head g) only rescale the scores of the
+    # q-heads reading g: the same as a softmax scale times dq * dk for them
+    rng = np.random.default_rng(61)
+    B, S, Hq, Hkv, D = 2, 5, 4, 2, 8
+    q8, k8, v8 = _codes((B, S, Hq, D), rng), _codes((B, S, Hkv, D), rng), _codes((B, S, Hkv, D), rng)
+    dq = np.array([[0.5, 0.125], [0.25, 1.0]])
+    dk = np.array([[0.25, 0.5], [0.0625, 0.75]])
+    dv = np.array([[1.5, 0.5], [2.0, 0.25]])
+    sc = 0.2
+    o, lse = oracle.attn_fwd_fp8(q8, k8, v8, dq, dk, dv, scale=sc, causal=True)
+    qv, kv, vv = oracle.e4m3_decode(q8), oracle.e4m3_decode(k8), oracle.e4m3_decode(v8)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // (Hq // Hkv)
+            o1, l1 = oracle.attn_fwd(qv[b:b + 1, :, h:h + 1], kv[b:b + 1, :, g:g + 1], vv[b:b + 1, :, g:g + 1],
+                                     sc * dq[b, g] * dk[b, g], True)
+            np.testing.assert_allclose(o[b, :, h], dv[b, g] * o1[0, :, 0], rtol=1e-12, atol=1e-12)
+            np.testing.assert_allclose(lse[b, h], l1[0, 0], rtol=0, atol=1e-12)
+
+
+def test_planted_fp8_descale_by_q_head_is_caught(monkeypatch):
+    orig = oracle.attn_fwd_fp8
+
+    def bad(q8, k8, v8, descale_q=None, descale_k=None, descale_v=None, **kw):
+        # q factor taken by q-head index modulo Hkv instead of its kv-head
+        Hq, Hkv = q8.shape[2], k8.shape[2]
+        qv = oracle.e4m3_decode(q8) * np.asarray(descale_q)[:, None, [h % Hkv for h in range(Hq)], None]
+        return oracle.attn_fwd(qv, oracle.e4m3_decode(k8) * np.asarray(descale_k)[:, None, :, None],
+                               oracle.e4m3_decode(v8) * np.asarray(descale_v)[:, None, :, None], kw.get("scale"),
+                               kw.get("causal", False))
+
+    monkeypatch.setattr(oracle, "attn_fwd_fp8", bad)
+    with pytest.raises(AssertionError):
+        test_fp8_descales_act_per_batch_and_kv_head()
+    monkeypatch.setattr(oracle, "attn_fwd_fp8", orig)
