@@ -38,7 +38,10 @@ METRIC = "attention TFLOPs/s fwd+bwd (seqlen sweep 512-16k d64/d128, GQA+local, 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # Launch whose per-launch roofline is reported for each kernel class.
-ROOFLINE_UNIT = {"fwd": "H16D128S4096n", "bwd": "H16D128S4096n", "decode": "decode"}
+ROOFLINE_UNIT = {"fwd": "H16D128S4096n", "bwd": "H16D128S4096n", "fwd8": "fp8-H16D128S4096n", "decode": "decode"}
+# dense E4M3 tensor throughput over bf16 (nominal 4.5 / 2.25 PFLOP/s): the FP8
+# roofline peak is the measured bf16 figure times this ratio
+FP8_OVER_BF16 = 2.0
 # DRAM bytes (read + write) per launch from one ncu capture of that launch
 # (profiles/*_H16D128S4096n.md, profiles/decode_tma_kernel_paged_B8.md).  An
 # entry must be removed whenever its kernel changes.
@@ -302,6 +305,53 @@ class DecodeUnit:
                 self.out.numel() * self.out.element_size())
 
 
+class Fp8Unit:
+    """FP8 (E4M3) forward through fa_fwd_fp8: q, k, v in, bf16 O out."""
+    kind = "fp8"
+
+    def __init__(self, cfg, dev):
+        from exact_attention_121_b200 import api, inputs
+        self.api = api
+        self.cfg = cfg
+        q, k, v, dq, dk, dv = inputs.fp8_inputs(cfg["B"], cfg["Sq"], cfg["Sk"], cfg["Hq"], cfg["Hkv"], cfg["D"],
+                                                seed=cfg["seed"], amp=cfg["amp"])
+        self.host_in = (q, k, v)
+        self.q, self.k, self.v = (t.to(dev) for t in self.host_in)
+        self.dq, self.dk, self.dv = (t.to(dev) for t in (dq, dk, dv))
+        self.out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(cfg["B"], cfg["Hq"], cfg["Sq"], device=dev)
+        self.flops_fwd8 = attn_flops(cfg)[0]
+        self.kw = dict(scale=cfg["scale"], causal=cfg["causal"], window=cfg["window"], softcap=cfg["softcap"])
+
+    def name(self):
+        c = self.cfg
+        return "fp8-H%dD%dS%d%s" % (c["Hq"], c["D"], c["Sq"], "c" if c["causal"] else "n")
+
+    def run(self, tracer):
+        tracer.arm("fwd8", self)
+        self.api.fa_fwd_fp8(self.q, self.k, self.v, self.dq, self.dk, self.dv, out=self.out, lse=self.lse, **self.kw)
+        tracer.disarm()
+        return self.api.fa_last_launch_count()
+
+    def flops(self):
+        return self.flops_fwd8
+
+    def setup_e2e(self, pinned):
+        self.pin_in = [pinned.get(t, i) for i, t in enumerate(self.host_in)]
+        self.pin_out = [pinned.get_like(self.out)]
+
+    def copy_in(self):
+        for dst, src in zip((self.q, self.k, self.v), self.pin_in):
+            dst.copy_(src, non_blocking=True)
+
+    def copy_out(self):
+        self.pin_out[0].copy_(self.out, non_blocking=True)
+
+    def e2e_bytes(self):
+        return (sum(t.numel() * t.element_size() for t in (self.q, self.k, self.v)),
+                self.out.numel() * self.out.element_size())
+
+
 class Pinned:
     """Pinned host staging buffers: one per input tensor (each unit's own
     values), outputs shared between units of equal byte size (the copies out
@@ -344,7 +394,7 @@ class Tracer:
         b.record()
         self.lib.fa_set_trace_events(a.cuda_event, b.cuda_event)
         work = {"fwd": getattr(unit, "flops_fwd", 0), "bwd": getattr(unit, "flops_bwd", 0),
-                "decode": getattr(unit, "bytes", 0)}[cls]
+                "fwd8": getattr(unit, "flops_fwd8", 0), "decode": getattr(unit, "bytes", 0)}[cls]
         self.pending.append((cls, unit.name(), a, b, work))
 
     def disarm(self):
@@ -389,6 +439,8 @@ def build_units(dev, workload, point=None):
         units.append(VarlenUnit(inputs.varlen_config(), dev))
     if workload == "decode_rotary":
         units.append(DecodeUnit(inputs.paged_decode_rotary_config(), dev))
+    if workload == "fp8":
+        units.append(Fp8Unit(inputs.fp8_config(), dev))
     if workload == "alibi":
         units.append(AttnUnit(inputs.alibi_config(), dev))
     return units
@@ -533,7 +585,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="full", choices=["full", "sweep", "gqa", "decode", "small", "point", "varlen",
-                                                                   "alibi", "decode_rotary"])
+                                                                   "alibi", "decode_rotary", "fp8"])
     ap.add_argument("--point", default="H16D128S4096n", help="sweep point for --workload point")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -613,6 +665,9 @@ def main():
     if cls == "decode":
         pk = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk, "unit": "GB/s", "frac": achieved / pk}
+    elif cls == "fwd8":
+        pk = peaks["bf16_tflops_sustained"] * FP8_OVER_BF16
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s", "frac": achieved / pk}
     else:
         pk = peaks["bf16_tflops_sustained"]
         roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s", "frac": achieved / pk}
@@ -621,8 +676,10 @@ def main():
     roof["algorithmic_per_launch"] = work / cnt
     roof["achieved_all_launches"] = achieved_all
     roof["kernel"] = {"fwd": "fwd_tc_kernel (tcgen05 forward)", "bwd": "bwd_tc_kernel (tcgen05 backward)",
+                      "fwd8": "fwd_tc_kernel<E4M3> (tcgen05 kind::f8f6f4 forward)",
                       "decode": "decode_tma_kernel (split-KV decode)"}[cls]
-    roof["peak_source"] = f"{peak_src} ({'bf16_tflops_sustained' if cls != 'decode' else 'hbm_gbs'})"
+    roof["peak_source"] = f"{peak_src} " + {"decode": "(hbm_gbs)", "fwd8": "(bf16_tflops_sustained x 2, e4m3/bf16 "
+                                                       "nominal ratio)"}.get(cls, "(bf16_tflops_sustained)")
     kernels = {c: {"ms_total": v[0], "launches": v[1],
                    ("gbs" if c == "decode" else "tflops"): v[2] / (v[0] / 1e3) / (1e9 if c == "decode" else 1e12)}
                for c, v in totals.items()}
@@ -634,7 +691,8 @@ def main():
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if args.workload == "fp8" else "bf16",
+                "data": "synthetic",
                 "config": {"workload": args.workload + ": " + ", ".join(u.name() for u in units),
                            "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}",
                            "flops_per_step": flops_step},

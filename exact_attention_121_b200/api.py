@@ -113,6 +113,33 @@ def fa_fwd(q, k, v, out=None, lse=None, scale=None, causal=False, window=(-1, -1
     return out, lse
 
 
+def fa_fwd_fp8(q, k, v, descale_q=None, descale_k=None, descale_v=None, out=None, lse=None, scale=None,
+               causal=False, window=(-1, -1), softcap=0.0, stream=None):
+    """FP8 forward: q, k, v torch.float8_e4m3fn (B, S, H, D), head dim 128;
+    descales float32 (B, Hkv) or None.  Returns (out bf16, lse fp32)."""
+    lib = _lib.load()
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check_tensor(t, n, torch.float8_e4m3fn, q.device)
+    for t, n in ((descale_q, "descale_q"), (descale_k, "descale_k"), (descale_v, "descale_v")):
+        _check_tensor(t, n, torch.float32, q.device)
+        if t is not None and t.shape != (B, Hkv):
+            raise ValueError(f"{n} must be ({B}, {Hkv})")
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    _check_tensor(out, "out", torch.bfloat16, q.device)
+    _check_tensor(lse, "lse", torch.float32, q.device)
+    wl, wr = _window(window)
+    code = lib.fa_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq, Sk, Hq, Hkv, D,
+                          _ptr(descale_q), _ptr(descale_k), _ptr(descale_v), float(scale or 0.0),
+                          int(bool(causal)), wl, wr, float(softcap or 0.0), _stream(stream))
+    _lib.check(code, "fa_fwd_fp8")
+    return out, lse
+
+
 def fa_bwd_workspace_size(B, Sq, Sk, Hq, Hkv, D, deterministic=False):
     return int(_lib.load().fa_bwd_workspace_size(B, Sq, Sk, Hq, Hkv, D, int(bool(deterministic))))
 

@@ -247,6 +247,44 @@ fa_status fa_fwd_alibi(const void* q, const void* k, const void* v, void* out, f
                   strides, alibi_slopes, alibi_batch_stride, stream);
 }
 
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Sq, int Sk,
+                     int Hq, int Hkv, int D, const float* descale_q, const float* descale_k,
+                     const float* descale_v, float scale, int causal, int window_left, int window_right,
+                     float softcap, fa_stream_t stream) {
+  g_last_launches = 0;
+  fa_status st = check_common(B, Sq, Hq, Hkv, D, FA_BF16, scale, softcap);
+  if (st != FA_OK) return st;
+  if (Sk < 0) return FA_ERR_INVALID_ARG;
+  for (const float* d : {descale_q, descale_k, descale_v})
+    if (reinterpret_cast<uintptr_t>(d) & 3u) return FA_ERR_INVALID_ARG;
+  if (D != 128) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || Sq == 0) return FA_OK;
+  if (Sk == 0) return FA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !out || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return FA_ERR_INVALID_ARG;
+  if (g_fwd_kernel_choice == 1) return FA_ERR_UNSUPPORTED;  // tcgen05 kernel only
+  fa::FwdParams p{};
+  p.q = q; p.k = k; p.v = v; p.o = out; p.lse = lse;
+  p.B = B; p.Sq = Sq; p.Sk = Sk; p.Hq = Hq; p.Hkv = Hkv; p.D = D; p.G = Hq / Hkv;
+  contiguous_strides(p.st_q, Sq, Hq, D);
+  contiguous_strides(p.st_k, Sk, Hkv, D);
+  contiguous_strides(p.st_v, Sk, Hkv, D);
+  contiguous_strides(p.st_o, Sq, Hq, D);
+  p.descale_q = descale_q; p.descale_k = descale_k; p.descale_v = descale_v;
+  fold_window(causal, window_left, window_right, &p.wl, &p.wr);
+  scale = resolve_scale(scale, D);
+  fill_cap(scale, softcap, &p.softcap, &p.cap_in, &p.cap_log2, &p.scale_log2);
+  p.status = status_ptr();
+  if (!p.status) return FA_ERR_CUDA;
+  if (!fa::fwd_tc_supported(p)) return FA_ERR_UNSUPPORTED;
+  int launches = 0;
+  const cudaError_t e = fa::launch_fwd_tc_fp8(p, stream, &launches);
+  g_last_launches = launches;
+  if (e == cudaErrorNotSupported) return FA_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 size_t fa_bwd_workspace_size(int B, int Sq, int Sk, int Hq, int Hkv, int D, int deterministic) {
   if (B < 0 || Sq < 0 || Sk < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || (D != 64 && D != 128)) return 0;
   size_t n = round256((size_t)B * Sq * Hq * D * sizeof(float));   // dQ accumulator

@@ -60,10 +60,11 @@ __host__ __device__ constexpr bool poly_pair(int i) { return ((i * FA_POLY_PAIRS
 
 constexpr unsigned long long kTcWaitNs = kWaitLimitNs;
 
-template <int D>
+template <int D, bool kF8 = false>
 struct TcCfg {
-  static constexpr int CHUNK = kRows * 128;          // one 64-column, 128-row swizzled chunk (16 KB)
-  static constexpr int NCHUNK = D / 64;
+  static constexpr int CHUNK = kRows * 128;          // one 128-byte-wide, 128-row swizzled chunk (16 KB)
+  static constexpr int CHUNK_ELEMS = kF8 ? 128 : 64; // head-dim elements per chunk
+  static constexpr int NCHUNK = D / CHUNK_ELEMS;
   static constexpr int TILE = CHUNK * NCHUNK;        // one 128-row tile
   static constexpr int NSK = (D == 128) ? 3 : 4;     // K stages
   static constexpr int NSV = (D == 128) ? 2 : 4;     // V stages
@@ -91,11 +92,19 @@ struct TcCfg {
 
 __device__ __forceinline__ float f32(uint32_t u) { return __uint_as_float(u); }
 
-template <typename T, int D, bool kCap, bool kAlibi>
+// factor of (batch b, kv-head g) in a (B, Hkv) array; none given = 1
+__device__ __forceinline__ float descale_of(const float* d, int b, int g, int Hkv) {
+  return d ? d[(long long)b * Hkv + g] : 1.f;
+}
+
+// kFp8: q, k, v are E4M3 codes (T is the 16-bit output type), the two
+// products run as kind::f8f6f4 and P is quantised to E4M3 in TMEM.
+template <typename T, int D, bool kCap, bool kAlibi, bool kFp8>
 __global__ void __launch_bounds__(kThreadsTC, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using C = TcCfg<D>;
+  using C = TcCfg<D, kFp8>;
+  static_assert(!kFp8 || D == 128, "the 8-bit path is laid out for head dim 128");
   // Head dim 64 leaves TMEM room for P beside O (P_t at [256+128t+64, +64)),
   // so S_t can be refilled while P_t still feeds the PV product.
   constexpr bool kSepP = (D == 64);
@@ -182,8 +191,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       mbar_expect_tx(bar(C::B_Q), 2 * C::TILE);
       for (int t = 0; t < 2; ++t)
         for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_4d(sb + C::OFF_Q + t * C::TILE + c * C::CHUNK, &tmQ, c * 64, h, seq.qtma + q0 + t * kRows, seq.tb,
-                      bar(C::B_Q));
+          tma_load_4d(sb + C::OFF_Q + t * C::TILE + c * C::CHUNK, &tmQ, c * C::CHUNK_ELEMS, h,
+                      seq.qtma + q0 + t * kRows, seq.tb, bar(C::B_Q));
       int issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
         const int sk = j % C::NSK, uk = j / C::NSK;
@@ -195,8 +204,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
         mbar_expect_tx(bar(C::B_KF + sk), C::TILE);
         for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_4d(sb + C::OFF_K + sk * C::TILE + c * C::CHUNK, &tmK, c * 64, g, seq.ktma + k0, seq.tb,
-                      bar(C::B_KF + sk));
+          tma_load_4d(sb + C::OFF_K + sk * C::TILE + c * C::CHUNK, &tmK, c * C::CHUNK_ELEMS, g, seq.ktma + k0,
+                      seq.tb, bar(C::B_KF + sk));
         if (j >= C::NSV && !mbar_wait(bar(C::B_VE + sv), (uv - 1) & 1, abort_flag, kTcWaitNs)) {
           fail();
           issued = -(j + 1);  // K of tile j is in flight, V is not
@@ -204,8 +213,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
         mbar_expect_tx(bar(C::B_VF + sv), C::TILE);
         for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_4d(sb + C::OFF_V + sv * C::TILE + c * C::CHUNK, &tmV, c * 64, g, seq.ktma + k0, seq.tb,
-                      bar(C::B_VF + sv));
+          tma_load_4d(sb + C::OFF_V + sv * C::TILE + c * C::CHUNK, &tmV, c * C::CHUNK_ELEMS, g, seq.ktma + k0,
+                      seq.tb, bar(C::B_VF + sv));
         issued = j + 1;
       }
       if (*abort_flag) {
@@ -223,26 +232,36 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0 && n_tiles > 0) {
-      constexpr bool kBf = Elem<T>::kBf16;
+      // format fields: bf16 / f16 for kind::f16, E4M3 (0) for kind::f8f6f4
+      constexpr bool kBf = !kFp8 && Elem<T>::kBf16;
       constexpr uint32_t idesc_qk = make_idesc(kBf, 128, 128, false);
       constexpr uint32_t idesc_pv = make_idesc(kBf, 128, D, true);
+      constexpr int KS = kFp8 ? 32 : 16;  // elements per MMA k-step (32 bytes either way)
       const uint32_t tS[2] = {tmem, tmem + 128};
       const uint32_t tO[2] = {tmem + 256, tmem + 384};
       const uint32_t tP[2] = {kSepP ? tmem + 256 + D : tS[0], kSepP ? tmem + 384 + D : tS[1]};
       auto issue_qk = [&](int t, int st) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < D / KS; ++kk) {
           const uint32_t koff = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
           const uint64_t ad = make_sdesc_sw128(sb + C::OFF_Q + t * C::TILE + koff, 16, 1024);
           const uint64_t bd = make_sdesc_sw128(sb + C::OFF_K + st * C::TILE + koff, 16, 1024);
-          mma_ss(tS[t], ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          if constexpr (kFp8)
+            mma_ss_f8(tS[t], ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          else
+            mma_ss(tS[t], ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, int st, bool acc) {
 #pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk) {
-          const uint64_t bd = make_sdesc_sw128(sb + C::OFF_V + st * C::TILE + kk * 16 * 128, C::CHUNK, 1024);
-          mma_ts(tO[t], tP[t] + kk * 8, bd, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kRows / KS; ++kk) {
+          // KS keys of V (MN-major: 128-byte rows of head-dim elements); P
+          // packs KS keys into 8 TMEM columns
+          const uint64_t bd = make_sdesc_sw128(sb + C::OFF_V + st * C::TILE + kk * KS * 128, C::CHUNK, 1024);
+          if constexpr (kFp8)
+            mma_ts_f8(tO[t], tP[t] + kk * 8, bd, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+          else
+            mma_ts(tO[t], tP[t] + kk * 8, bd, idesc_pv, (acc || kk > 0) ? 1u : 0u);
         }
       };
       bool ok = mbar_wait(bar(C::B_Q), 0, abort_flag, kTcWaitNs);
@@ -344,6 +363,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     float m_run = -INFINITY, l_run = 0.f, l_q = 0.f;
     // ALiBi slope of this (b, h), as a log2-domain factor of |qpos - key|
     const float mb = kAlibi ? -kLog2e * p.alibi[(long long)b * p.alibi_bstride + h] : 0.f;
+    // 8-bit inputs: the q and k factors of (b, kv-head g) scale the raw scores
+    const float qk_f = kFp8 ? descale_of(p.descale_q, b, g, p.Hkv) * descale_of(p.descale_k, b, g, p.Hkv) : 1.f;
+    const float scale_log2 = p.scale_log2 * qk_f, cap_in = p.cap_in * qk_f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       // warp-uniform outcome: the TMEM accesses below are warp-collective
@@ -371,14 +393,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       float mx = -INFINITY;
       if (kCap) {
 #pragma unroll
-        for (int i = 0; i < kRows; ++i) s[i] = __float_as_uint(p.cap_log2 * tanh_exp(f32(s[i]) * p.cap_in));
+        for (int i = 0; i < kRows; ++i) s[i] = __float_as_uint(p.cap_log2 * tanh_exp(f32(s[i]) * cap_in));
       }
       if (kAlibi) {
         // to the log2 domain, plus the distance bias mb |qpos - key| of key
         // k0 + i.  A tile on one side of every row of the warp has a bias
         // linear in i: t0 + step i, one fma per key (without the softcap:
         // beside the tanh the second copy of the loop costs spills).
-        const float in = kCap ? 1.f : p.scale_log2;
+        const float in = kCap ? 1.f : scale_log2;
         const bool left = !kCap && __all_sync(0xffffffffu, k0 + kRows - 1 <= qpos);
         const bool right = !kCap && __all_sync(0xffffffffu, k0 >= qpos);
         if (left || right) {
@@ -411,7 +433,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
         mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       }
-      const float sl = (kCap || kAlibi) ? 1.f : p.scale_log2;  // multiplier into the log2 domain
+      const float sl = (kCap || kAlibi) ? 1.f : scale_log2;  // multiplier into the log2 domain
       mx *= sl;
       // lazy rescale: move the running max only when it grows by > 2^8
       const bool move = (mx > m_run + kRescaleLog2) || (m_run == -INFINITY && mx != -INFINITY);
@@ -443,11 +465,22 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
             p1 = fast_exp2(x1);
           }
           rs2 = f2_add(rs2, f2_pack(p0, p1));
-          pk[i] = Elem<T>::pack(p0, p1);
-          const float2 pr = Elem<T>::unpack(pk[i]);
+          float2 pr;
+          if constexpr (kFp8) {
+            // four E4M3 keys per TMEM column, lowest key in the low byte
+            const uint32_t h8 = f32x2_to_e4m3x2(p0, p1);
+            pk[i >> 1] = (i & 1) ? (pk[i >> 1] | (h8 << 16)) : h8;
+            pr = e4m3x2_to_f32x2(h8);
+          } else {
+            pk[i] = Elem<T>::pack(p0, p1);
+            pr = Elem<T>::unpack(pk[i]);
+          }
           rq2 = f2_add(rq2, f2_pack(pr.x, pr.y));
         }
-        if (!kSepP) tmem_st16(tP + c * 16, pk);
+        if constexpr (kFp8)
+          tmem_st8(tP + c * 8, *reinterpret_cast<uint32_t(*)[8]>(&pk[0]));
+        else if (!kSepP)
+          tmem_st16(tP + c * 16, pk);
       }
       if (kSepP) {
         // P_t and O_t are free once PV_t(j-1) has completed
@@ -489,7 +522,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     } else {
       // ---- epilogue: O / l in 16 bits, LSE
       tc_fence_after();
-      const float inv = l_q > 0.f ? 1.f / l_q : 0.f;
+      // O / l (times the v factor of (b, g) for 8-bit inputs)
+      const float ov = kFp8 ? descale_of(p.descale_v, b, g, p.Hkv) : 1.f;
+      const float inv = l_q > 0.f ? ov / l_q : 0.f;
       T* orow = reinterpret_cast<T*>(p.o) + (long long)b * p.st_o[0] + (long long)(seq.qtma + qi) * p.st_o[1] +
                 (long long)h * p.st_o[2];
 #pragma unroll
@@ -532,11 +567,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 // host side
 // ---------------------------------------------------------------------------
 
-template <typename T, int D, bool kCap, bool kAlibi>
+template <typename T, int D, bool kCap, bool kAlibi, bool kFp8 = false>
 cudaError_t launch_t(const FwdParams& p, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                      cudaStream_t s) {
-  auto kern = fwd_tc_kernel<T, D, kCap, kAlibi>;
-  constexpr int smem = TcCfg<D>::SMEM;
+  auto kern = fwd_tc_kernel<T, D, kCap, kAlibi, kFp8>;
+  constexpr int smem = TcCfg<D, kFp8>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const long long ctas = (long long)((p.Sq + 255) / 256) * p.Hq * p.B;
@@ -566,6 +601,18 @@ cudaError_t launch_dt(const FwdParams& p, const CUtensorMap& mq, const CUtensorM
 
 bool fwd_tc_supported(const FwdParams& p) {
   return (p.D == 64 || p.D == 128) && p.Sk >= 1 && p.Sq >= 1 && tma_available();
+}
+
+cudaError_t launch_fwd_tc_fp8(const FwdParams& p, cudaStream_t s, int* launches) {
+  if (p.D != 128 || p.cu_q || p.alibi) return cudaErrorNotSupported;
+  CUtensorMap mq, mk, mv;
+  if (!make_bshd_map_u8(&mq, p.q, p.D, p.Hq, p.Sq, p.B, 128) || !make_bshd_map_u8(&mk, p.k, p.D, p.Hkv, p.Sk, p.B, 128) ||
+      !make_bshd_map_u8(&mv, p.v, p.D, p.Hkv, p.Sk, p.B, 128))
+    return cudaErrorNotSupported;
+  const cudaError_t e = p.softcap > 0.f ? launch_t<__nv_bfloat16, 128, true, false, true>(p, mq, mk, mv, s)
+                                        : launch_t<__nv_bfloat16, 128, false, false, true>(p, mq, mk, mv, s);
+  if (e == cudaSuccess) ++*launches;
+  return e;
 }
 
 cudaError_t launch_fwd_tc(const FwdParams& p, fa_dtype dt, cudaStream_t s, int* launches) {

@@ -36,6 +36,11 @@ struct FwdParams {
   // (bstride 0: one slope per head for the whole batch); null = off
   const float* alibi;
   int alibi_bstride;
+  // FP8 (E4M3) inputs: one float32 factor per (batch, kv-head) for q, k, v
+  // ((B, Hkv) arrays, null = 1); out is then bf16
+  const float* descale_q;
+  const float* descale_k;
+  const float* descale_v;
 };
 
 struct BwdParams {
@@ -112,6 +117,8 @@ void trace_end(cudaStream_t s);
 cudaError_t launch_fwd_mma(const FwdParams& p, fa_dtype dt, cudaStream_t s, int* launches);
 bool fwd_tc_supported(const FwdParams& p);
 cudaError_t launch_fwd_tc(const FwdParams& p, fa_dtype dt, cudaStream_t s, int* launches);
+// E4M3 q, k, v (head dim 128, dense batch), bf16 out
+cudaError_t launch_fwd_tc_fp8(const FwdParams& p, cudaStream_t s, int* launches);
 cudaError_t launch_bwd(const BwdParams& p, fa_dtype dt, cudaStream_t s, int* launches);
 bool bwd_tc_supported(const BwdParams& p);
 cudaError_t launch_bwd_main_tc(const BwdParams& p, fa_dtype dt, cudaStream_t s);

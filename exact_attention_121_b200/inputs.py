@@ -188,3 +188,22 @@ def paged_decode_rotary_config():
     cfg = paged_decode_config()
     cfg["rotary"] = True
     return cfg
+
+
+def fp8_inputs(B, Sq, Sk, Hq, Hkv, D, seed=0, amp=1.0):
+    """E4M3 q, k, v (torch.float8_e4m3fn, rounded from N(0, amp^2) draws in
+    the order q, k, v) and float32 (B, Hkv) descale factors U(0.5, 2) for q,
+    k, v, drawn after them."""
+    g = _gen(seed)
+    q = (amp * torch.randn((B, Sq, Hq, D), generator=g)).to(torch.float8_e4m3fn)
+    k = (amp * torch.randn((B, Sk, Hkv, D), generator=g)).to(torch.float8_e4m3fn)
+    v = (amp * torch.randn((B, Sk, Hkv, D), generator=g)).to(torch.float8_e4m3fn)
+    d = [0.5 + 1.5 * torch.rand((B, Hkv), generator=g) for _ in range(3)]
+    return q, k, v, d[0], d[1], d[2]
+
+
+def fp8_config():
+    """FP8 forward at hidden 2048: B=4, S=4096, Hq=Hkv=16, D=128, non-causal,
+    N(0,1) inputs rounded to E4M3 with U(0.5, 2) descales (seed 9)."""
+    return dict(B=4, Sq=4096, Sk=4096, Hq=16, Hkv=16, D=128, causal=False, window=(-1, -1), softcap=0.0,
+                scale=1.0 / math.sqrt(128), seed=9, amp=1.0)

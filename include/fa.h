@@ -217,6 +217,27 @@ fa_status fa_bwd_alibi(const void* dout, const void* q, const void* k, const voi
                        int deterministic, void* workspace, size_t ws_bytes, const long long* strides,
                        const float* alibi_slopes, int alibi_batch_stride, fa_stream_t stream);
 
+/*
+ * FP8 forward ("FlashAttention 实战指南", versions: FlashAttention-3 adds an
+ * FP8 forward; an fp8 path keeps precision and lowers bandwidth).  q
+ * (B, Sq, Hq, D), k and v (B, Sk, Hkv, D) hold OCP FP8 E4M3 codes, one byte
+ * each, packed, 16-byte aligned.  descale_q, descale_k, descale_v are device
+ * float32 (B, Hkv) arrays (a q-head uses the factor of its kv-head) or NULL
+ * for 1: the inputs are code value x factor, and the call computes the
+ * exact attention of those inputs as fa_fwd does (scale, causal, window,
+ * softcap alike).  out (B, Sq, Hq, D) is bf16; lse (B, Hq, Sq) fp32.
+ * Internally P is quantised to E4M3 for the P.V product and O is divided by
+ * the sum of the quantised P, so each output row is a convex combination of
+ * V rows whose weights are off by at most the E4M3 rounding of P.  Head dim
+ * 128 and Sk >= 1 only (FA_ERR_UNSUPPORTED otherwise); misaligned pointers
+ * give FA_ERR_INVALID_ARG.  tcgen05 kernel only.
+ */
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, float* lse,
+                     int B, int Sq, int Sk, int Hq, int Hkv, int D,
+                     const float* descale_q, const float* descale_k, const float* descale_v,
+                     float scale, int causal, int window_left, int window_right, float softcap,
+                     fa_stream_t stream);
+
 /* Largest split count fa_fwd_kvcache accepts; num_splits <= 0 picks one. */
 #define FA_MAX_SPLITS 64
 

@@ -152,3 +152,14 @@ def test_alibi_host_validation(lib):
                                          ctypes.c_void_p(0x10000), 1 << 20, None, a, bs, None)
     assert bwd(None, 0) == _lib.FA_ERR_INVALID_ARG
     assert bwd(p, 3) == _lib.FA_ERR_INVALID_ARG
+
+
+def test_fp8_host_validation(lib):
+    p = ctypes.c_void_p(0x1000)
+    fwd = lambda D=128, B=1, Sk=8, d=None: lib.fa_fwd_fp8(p, p, p, p, p, B, 8, Sk, 2, 2, D, d, None, None, 0.0, 0,
+                                                          -1, -1, 0.0, None)
+    assert fwd(D=64) == _lib.FA_ERR_UNSUPPORTED                   # laid out for head dim 128
+    assert fwd(d=ctypes.c_void_p(0x1002)) == _lib.FA_ERR_INVALID_ARG  # descale not 4-byte aligned
+    assert fwd(B=0) == _lib.FA_OK                                 # nothing to do
+    assert fwd(Sk=0) == _lib.FA_ERR_UNSUPPORTED
+    assert fwd(Sk=-1) == _lib.FA_ERR_INVALID_ARG
