@@ -48,6 +48,7 @@ FP8_OVER_BF16 = 2.0
 TRAFFIC_PER_LAUNCH = {
     ("fwd", "H16D128S4096n"): 201.704960e6 + 53.250816e6,
     ("bwd", "H16D128S4096n"): 415.648512e6 + 231.981824e6,
+    ("fwd8", "fp8-H16D128S4096n"): 100.751104e6 + 37.022720e6,
     ("decode", "decode"): 521.946368e6 + 7.995904e6,
 }
 
