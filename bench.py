@@ -672,6 +672,15 @@ def main():
     else:
         pk = peaks["bf16_tflops_sustained"]
         roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s", "frac": achieved / pk}
+    if cls != "decode":
+        # exponentials: one per visible (query, key) pair in either pass, i.e.
+        # flops / (4 D) forward, flops / (10 D) backward, head dim 128 here;
+        # nominal MUFU rate 16 per clock per SM at the sampled SM clock
+        exps = (work / cnt) / ((10 if cls == "bwd" else 4) * 128)
+        exp_rate = exps / (kms / cnt / 1e3)
+        exp_peak = 16 * 148 * ((clk or {}).get("sm_mhz") or 1965.0) * 1e6
+        roof["sfu"] = {"exp_per_launch": exps, "exp_per_s": exp_rate, "peak_exp_per_s": exp_peak,
+                       "frac": exp_rate / exp_peak, "peak_source": "nominal 16/clk/SM x 148 SMs x sampled SM clock"}
     roof["traffic"] = TRAFFIC_PER_LAUNCH.get((cls, rep))
     roof["launch"] = rep
     roof["algorithmic_per_launch"] = work / cnt

@@ -163,3 +163,12 @@ def test_fp8_host_validation(lib):
     assert fwd(B=0) == _lib.FA_OK                                 # nothing to do
     assert fwd(Sk=0) == _lib.FA_ERR_UNSUPPORTED
     assert fwd(Sk=-1) == _lib.FA_ERR_INVALID_ARG
+
+
+def test_backward_workspace_is_linear_in_sequence_length(lib):
+    # O(S) memory: the dQ accumulator, Delta and (deterministic) one counter
+    # per 64-row query block grow linearly with S; nothing is S x S
+    for det in (0, 1):
+        w = [lib.fa_bwd_workspace_size(2, S, S, 16, 16, 128, det) for S in (4096, 8192, 16384)]
+        assert abs(w[1] / w[0] - 2.0) < 0.01 and abs(w[2] / w[1] - 2.0) < 0.01
+        assert w[2] < 2 * 16384 * 16 * 128 * 4 * 1.01 + 2 * 16 * 16384 * 4 * 2  # ~ fp32 dQ + Delta + counters
