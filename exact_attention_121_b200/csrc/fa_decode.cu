@@ -15,6 +15,8 @@
 // is read once for the whole group.
 #include <math.h>
 
+#include <type_traits>
+
 #include "fa_common.cuh"
 #include "fa_kernels.h"
 
@@ -421,38 +423,64 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecodeP
   }
 }
 
-// One warp per (b, q-head, query row): LSE = ln sum_s e^{LSE_s},
-// O = sum_s e^{LSE_s - LSE} O_s.
+// One 4-warp block per (b, q-head, query row): LSE = ln sum_s e^{LSE_s},
+// O = sum_s e^{LSE_s - LSE} O_s.  Warp w takes splits w, w+4, ...; every
+// lane loads its D/32 contiguous floats of O_s as one vector, and the loads
+// do not depend on the split's weight (an empty split's weight 0 selects
+// nothing), so consecutive splits' loads are in flight together; the four
+// partial sums meet in shared memory.
+constexpr int kCombineWarps = 4;
+
 template <typename T, int D>
-__global__ void decode_combine_kernel(const DecodeParams p) {
-  constexpr int PER_LANE = D / 32;
-  const int warps_per_block = blockDim.x / 32;
-  const long long row = (long long)blockIdx.x * warps_per_block + threadIdx.x / 32;
-  const int lane = threadIdx.x & 31;
-  const long long nrows = (long long)p.B * p.Hq * p.Sq;
-  if (row >= nrows) return;
-  const size_t split_stride = (size_t)nrows;
-  float M = -INFINITY;
-  for (int s = lane; s < p.num_splits; s += 32) M = fmaxf(M, p.lse_part[s * split_stride + row]);
+__global__ void __launch_bounds__(kCombineWarps * 32) decode_combine_kernel(const DecodeParams p) {
+  constexpr int PER_LANE = D / 32;  // 4 at head dim 128, 2 at 64
+  using Vec = typename std::conditional<PER_LANE == 4, float4, float2>::type;
+  __shared__ float s_acc[kCombineWarps][D];
+  __shared__ float s_w[kCombineWarps], s_m[kCombineWarps];
+  const long long row = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t split_stride = (size_t)p.B * p.Hq * p.Sq;
+  // largest split LSE (num_splits <= FA_MAX_SPLITS < the block's threads)
+  float m = (int)threadIdx.x < p.num_splits ? p.lse_part[threadIdx.x * split_stride + row] : -INFINITY;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) s_m[warp] = m;
+  __syncthreads();
+  float M = s_m[0];
+#pragma unroll
+  for (int w = 1; w < kCombineWarps; ++w) M = fmaxf(M, s_m[w]);
   float acc[PER_LANE];
 #pragma unroll
   for (int j = 0; j < PER_LANE; ++j) acc[j] = 0.f;
   float wsum = 0.f;
   if (M != -INFINITY) {
-    for (int s = 0; s < p.num_splits; ++s) {
-      const float ls = p.lse_part[s * split_stride + row];
-      const float w = fast_exp2((ls - M) * kLog2e);
+#pragma unroll 4
+    for (int sp = warp; sp < p.num_splits; sp += kCombineWarps) {
+      const float ls = p.lse_part[sp * split_stride + row];
+      const Vec v = *reinterpret_cast<const Vec*>(p.o_part + (sp * split_stride + row) * D + lane * PER_LANE);
+      const float w = fast_exp2((ls - M) * kLog2e);  // 0 for an empty split (LSE -inf)
+      const float* vf = reinterpret_cast<const float*>(&v);
       wsum += w;
-      if (w > 0.f) {
-        const float* o = p.o_part + (s * split_stride + row) * D + lane * PER_LANE;
 #pragma unroll
-        for (int j = 0; j < PER_LANE; ++j) acc[j] += w * o[j];
-      }
+      for (int j = 0; j < PER_LANE; ++j) acc[j] = w > 0.f ? fmaf(w, vf[j], acc[j]) : acc[j];
     }
   }
-  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+  for (int j = 0; j < PER_LANE; ++j) s_acc[warp][lane * PER_LANE + j] = acc[j];
+  if (lane == 0) s_w[warp] = wsum;
+  __syncthreads();
+  if (warp != 0) return;
+  float W = 0.f;
+#pragma unroll
+  for (int w = 0; w < kCombineWarps; ++w) W += s_w[w];
+#pragma unroll
+  for (int j = 0; j < PER_LANE; ++j) {
+    float a = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCombineWarps; ++w) a += s_acc[w][lane * PER_LANE + j];
+    acc[j] = a;
+  }
+  const float inv = W > 0.f ? 1.f / W : 0.f;
   // row = (b * Hq + h) * Sq + sq
   const int sq = (int)(row % p.Sq);
   const long long bh = row / p.Sq;
@@ -464,7 +492,7 @@ __global__ void decode_combine_kernel(const DecodeParams p) {
     const uint32_t v = Elem<T>::pack(acc[j] * inv, acc[j + 1] * inv);
     *reinterpret_cast<uint32_t*>(out + j) = v;
   }
-  if (p.lse && lane == 0) p.lse[row] = wsum > 0.f ? M + logf(wsum) : -INFINITY;
+  if (p.lse && lane == 0) p.lse[row] = W > 0.f ? M + logf(W) : -INFINITY;
 }
 
 template <typename T, int D, bool kCap>
@@ -527,12 +555,12 @@ cudaError_t launch_decode_t(const DecodeParams& p_in, cudaStream_t s, int* launc
   ++*launches;
   if (p.num_splits > 1) {
     const long long rows = (long long)p.B * p.Hq * p.Sq;
-    const int wpb = 8;
-    const int blocks = (int)((rows + wpb - 1) / wpb);
+    if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;  // one block per row
+    static_assert(FA_MAX_SPLITS <= kCombineWarps * 32, "one thread per split for the LSE maximum");
     if (p.D == 64)
-      decode_combine_kernel<T, 64><<<blocks, wpb * 32, 0, s>>>(p);
+      decode_combine_kernel<T, 64><<<(unsigned)rows, kCombineWarps * 32, 0, s>>>(p);
     else
-      decode_combine_kernel<T, 128><<<blocks, wpb * 32, 0, s>>>(p);
+      decode_combine_kernel<T, 128><<<(unsigned)rows, kCombineWarps * 32, 0, s>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     ++*launches;
