@@ -57,7 +57,7 @@ typedef struct CUstream_st* fa_stream_t;
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment or Hq % Hkv != 0 */
-  FA_ERR_UNSUPPORTED = 2, /* valid request this build does not implement (e.g. D=96) */
+  FA_ERR_UNSUPPORTED = 2, /* valid request the library does not implement (e.g. D=96) */
   FA_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
   FA_ERR_TIMEOUT = 4      /* a bounded device wait ran out (device status word) */
 } fa_status;
