@@ -47,9 +47,10 @@ def _rand(shape, rng, amp=1.0):
 @pytest.mark.parametrize("ex", _load()["examples"], ids=lambda e: e["name"])
 def test_hand_examples_forward(ex):
     q, k, v = _arr(ex["q"]), _arr(ex["k"]), _arr(ex["v"])
+    extra = {"alibi_slopes": _arr(ex["alibi_slopes"])} if "alibi_slopes" in ex else {}
     o, lse = oracle.attn_fwd(q, k, v, scale=_ev(ex["scale"]), causal=ex["causal"],
                              window_left=ex["window"][0], window_right=ex["window"][1],
-                             softcap=_ev(ex["softcap"]))
+                             softcap=_ev(ex["softcap"]), **extra)
     np.testing.assert_allclose(o, _arr(ex["out"]), rtol=0, atol=1e-13)
     np.testing.assert_allclose(lse, _arr(ex["lse"]), rtol=0, atol=1e-13)
 
@@ -712,6 +713,8 @@ def test_planted_alibi_sign_is_caught(monkeypatch):
     monkeypatch.setattr(attn64, "alibi_bias", lambda m, rows, Sq, Sk: -orig(m, rows, Sq, Sk))
     with pytest.raises(AssertionError):
         test_alibi_geometric_weights_closed_form(True, 9, 9)
+    with pytest.raises(AssertionError):
+        test_hand_examples_forward(_hand("alibi_causal_two_keys"))
 
 
 def test_planted_alibi_top_left_alignment_is_caught(monkeypatch):
