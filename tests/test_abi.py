@@ -46,6 +46,33 @@ def test_every_declared_symbol_is_exported_with_its_arity(lib):
         assert len(_lib.SIGNATURES[name][1]) == nargs, name
 
 
+def _ctype_of(param):
+    """ctypes class a C parameter declaration binds to: pointers (and the
+    stream handle) as c_void_p, float as c_float, size_t as c_size_t, int
+    and the enums as c_int."""
+    decl = param.strip()
+    if "*" in decl or decl.startswith("fa_stream_t"):
+        return ctypes.c_void_p
+    words = decl.replace("const ", "").split()
+    base = " ".join(words[:-1])
+    return {"float": ctypes.c_float, "size_t": ctypes.c_size_t, "int": ctypes.c_int, "fa_dtype": ctypes.c_int,
+            "fa_status": ctypes.c_int, "long long": ctypes.c_longlong}[base]
+
+
+def test_every_binding_matches_the_declared_parameter_types():
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    seen = 0
+    for m in re.finditer(r"^\s*(?:const\s+char\s*\*|fa_status|size_t|void|int)\s+(fa_\w+)\s*\(([^)]*)\)\s*;",
+                         text, flags=re.M):
+        args = m.group(2).strip()
+        params = [] if args in ("", "void") else args.split(",")
+        want = [_ctype_of(a) for a in params]
+        got = _lib.SIGNATURES[m.group(1)][1]
+        assert got == want, (m.group(1), [t.__name__ for t in got], [t.__name__ for t in want])
+        seen += 1
+    assert seen == len(_lib.SIGNATURES)
+
+
 def test_status_strings(lib):
     assert lib.fa_status_string(0) == b"FA_OK"
     assert lib.fa_status_string(4) == b"FA_ERR_TIMEOUT"
