@@ -78,3 +78,37 @@ def test_rotary_position_outside_table_is_reported():
                        rotary_sin=torch.from_numpy(sin).cuda())
     torch.cuda.synchronize()
     assert api.fa_last_device_status() == 1  # FA_ERR_INVALID_ARG
+
+
+def test_rotary_paged_decode_full_size():
+    # the bench's paged-decode workload with full-width tables: every
+    # sequence against the oracle on its gathered prefix plus the rotated
+    # new token (rows rounded to bf16 as stored and multiplied)
+    cfg = inputs.paged_decode_rotary_config()
+    d = inputs.kvcache_inputs(cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["D"], cfg["page_size"], cfg["pages_per_seq"],
+                              cfg["max_len"], Sq=1, Snew=1, dtype="bf16", seed=cfg["seed"])
+    cos_t, sin_t = inputs.rotary_tables(cfg["max_len"] + 1, cfg["D"])
+    q, kc, vc, kn, vn = (d[n].cuda() for n in ("q", "k_cache", "v_cache", "k_new", "v_new"))
+    out, lse = api.fa_fwd_kvcache(q, kc, vc, kn, vn, d["cache_seqlens"].cuda(), d["block_table"].cuda(),
+                                  page_size=cfg["page_size"], scale=cfg["scale"], causal=True,
+                                  rotary_cos=cos_t.cuda(), rotary_sin=sin_t.cuda())
+    torch.cuda.synchronize()
+    assert api.fa_last_device_status() == 0
+    cos, sin = cos_t.numpy(), sin_t.numpy()
+    rnd = lambda x: torch.from_numpy(x).to(torch.bfloat16).double().numpy()
+    bt = d["block_table"].numpy()
+    kc_h, vc_h = d["k_cache"].float().numpy(), d["v_cache"].float().numpy()
+    ps = cfg["page_size"]
+    for b in range(cfg["B"]):
+        L0 = int(d["cache_seqlens"][b])
+        pos = np.array([[L0]])
+        k_rot = oracle.rotary(d["k_new"][b:b + 1].float().numpy(), cos, sin, pos)[0]
+        q_rot = rnd(oracle.rotary(d["q"][b:b + 1].float().numpy(), cos, sin, pos))
+        K = np.concatenate([oracle.gather_cache(kc_h, b, L0, bt, ps), rnd(k_rot)])[None]
+        V = np.concatenate([oracle.gather_cache(vc_h, b, L0, bt, ps), d["v_new"][b].float().numpy()])[None]
+        o_r, l_r = oracle.attn_fwd(q_rot, K, V, cfg["scale"], True)
+        check_out(out[b:b + 1], o_r, torch.bfloat16)
+        check_lse(lse[b:b + 1], l_r)
+        page, slot = bt[b, L0 // ps], L0 % ps
+        assert torch.equal(vc[page, slot].cpu(), d["v_new"][b, 0])
+        check_out(kc[page, slot], k_rot[0], torch.bfloat16, "rotated K slot")
