@@ -71,8 +71,10 @@ import math
 
 import numpy as np
 
-# -inf arithmetic on masked entries is intended; the results are selected away.
-np.seterr(invalid="ignore", divide="ignore")
+# -inf arithmetic on masked entries is intended (the results are selected
+# away): the functions that do it silence NumPy's warnings for their own
+# duration only, leaving the caller's error state alone.
+_masked_math = np.errstate(invalid="ignore", divide="ignore")
 
 NEG_INF = -np.inf
 
@@ -157,6 +159,7 @@ def alibi_bias(slope, rows, Sq, Sk):
     return -float(slope) * np.abs(qpos - np.arange(Sk)[None, :]).astype(np.float64)
 
 
+@_masked_math
 def attn_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1,
              softcap=0.0, return_probs=False, alibi_slopes=None):
     """Exact attention O = softmax(transform(scale * Q K^T) [+ ALiBi] + mask) V.
@@ -204,6 +207,7 @@ def attn_fwd(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1,
     return out, lse
 
 
+@_masked_math
 def attn_fwd_rows(q, k, v, b, h, rows, scale=None, causal=False, window_left=-1, window_right=-1,
                   softcap=0.0, alibi_slopes=None):
     """O and LSE of selected query rows of one (batch b, q-head h).
@@ -243,6 +247,7 @@ def attn_fwd_rows(q, k, v, b, h, rows, scale=None, causal=False, window_left=-1,
 # forward: the tiled online-softmax algorithm (pins attn_fwd, never the GPU)
 # ---------------------------------------------------------------------------
 
+@_masked_math
 def attn_fwd_online(q, k, v, scale=None, causal=False, window_left=-1, window_right=-1,
                     softcap=0.0, block=16):
     """Same result as :func:`attn_fwd`, reached block by block.
@@ -291,6 +296,7 @@ def attn_fwd_online(q, k, v, scale=None, causal=False, window_left=-1, window_ri
 # backward: chain rule on the materialised tensors
 # ---------------------------------------------------------------------------
 
+@_masked_math
 def attn_bwd(dout, q, k, v, scale=None, causal=False, window_left=-1, window_right=-1,
              softcap=0.0, alibi_slopes=None):
     """Gradients of L = sum(dout * O) with respect to q, k, v.
@@ -403,6 +409,7 @@ def rotary(x, cos, sin, positions, interleaved=False):
     return x
 
 
+@_masked_math
 def attn_with_kvcache(q, k_cache, v_cache, k_new=None, v_new=None, cache_seqlens=None,
                       block_table=None, page_size=None, scale=None, causal=False,
                       window_left=-1, window_right=-1, softcap=0.0, rotary_cos=None, rotary_sin=None,
@@ -458,6 +465,7 @@ def split_token_ranges(L, unit, num_splits):
     return out
 
 
+@_masked_math
 def attn_partial(q, K, V, t0, t1, scale, causal=False, window_left=-1, window_right=-1,
                  softcap=0.0):
     """Attention of q (Sq, Hq, D) over keys [t0, t1) of K, V (L, Hkv, D).
@@ -487,6 +495,7 @@ def attn_partial(q, K, V, t0, t1, scale, causal=False, window_left=-1, window_ri
     return o, lse
 
 
+@_masked_math
 def combine_splits(o_parts, lse_parts):
     """Merge split results: LSE = ln sum_s e^{LSE_s}; O = sum_s e^{LSE_s-LSE} O_s.
 
@@ -509,6 +518,7 @@ def combine_splits(o_parts, lse_parts):
 # variable-length (packed) batches
 # ---------------------------------------------------------------------------
 
+@_masked_math
 def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale=None, causal=False, window_left=-1,
                     window_right=-1, softcap=0.0):
     """Packed batch: q (total_q, Hq, D), k/v (total_k, Hkv, D).  Every
@@ -529,6 +539,7 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale=None, causal=Fals
     return out, lse
 
 
+@_masked_math
 def attn_bwd_varlen(dout, q, k, v, cu_seqlens_q, cu_seqlens_k, scale=None, causal=False, window_left=-1,
                     window_right=-1, softcap=0.0):
     """Gradients of sum(dout * O) for a packed batch; each sequence is the
@@ -552,6 +563,7 @@ def attn_bwd_varlen(dout, q, k, v, cu_seqlens_q, cu_seqlens_k, scale=None, causa
 # FP8 (E4M3) forward
 # ---------------------------------------------------------------------------
 
+@_masked_math
 def e4m3_decode(codes):
     """Float64 values of OCP FP8 E4M3 codes (uint8): sign in bit 7, a 4-bit
     exponent (bits 6..3, bias 7) and a 3-bit mantissa; exponent 0 holds the
@@ -566,6 +578,7 @@ def e4m3_decode(codes):
     return sign * mag
 
 
+@_masked_math
 def attn_fwd_fp8(q8, k8, v8, descale_q=None, descale_k=None, descale_v=None, scale=None, causal=False,
                  window_left=-1, window_right=-1, softcap=0.0):
     """FP8 forward: q8 (B, Sq, Hq, D), k8/v8 (B, Sk, Hkv, D) E4M3 codes; the
