@@ -192,10 +192,26 @@ def test_fp8_host_validation(lib):
     assert fwd(Sk=-1) == _lib.FA_ERR_INVALID_ARG
 
 
-def test_backward_workspace_is_linear_in_sequence_length(lib):
-    # O(S) memory: the dQ accumulator, Delta and (deterministic) one counter
-    # per 64-row query block grow linearly with S; nothing is S x S
-    for det in (0, 1):
-        w = [lib.fa_bwd_workspace_size(2, S, S, 16, 16, 128, det) for S in (4096, 8192, 16384)]
-        assert abs(w[1] / w[0] - 2.0) < 0.01 and abs(w[2] / w[1] - 2.0) < 0.01
-        assert w[2] < 2 * 16384 * 16 * 128 * 4 * 1.01 + 2 * 16 * 16384 * 4 * 2  # ~ fp32 dQ + Delta + counters
+def test_kvcache_rotary_host_validation(lib):
+    p = ctypes.c_void_p(0x1000)
+    ws = ctypes.c_void_p(0x100000)  # 256-byte aligned
+    # B=2 Sq=Snew=1 Hq=8 Hkv=2 D=128 bf16, paged (page 256, 4 pages/seq, 8 pages), causal, one split
+    head = [p, p, p, p, p, p, p, 256, 4, 8, p, p, 2, 1, 1, 8, 2, 128, 1, 0.0, 1, -1, -1, 0.0]
+
+    def call(cos=p, sin=p, dim=128, seqlen_ro=100, w=ws, nbytes=1 << 20):
+        return lib.fa_fwd_kvcache_rotary(*head, cos, sin, dim, seqlen_ro, 0, 1, w, nbytes, None)
+
+    bad = _lib.FA_ERR_INVALID_ARG
+    assert call(cos=None) == bad and call(sin=None) == bad       # tables required
+    assert call(dim=0) == bad and call(dim=127) == bad            # even and positive
+    assert call(dim=256) == bad                                   # at most the head dim
+    assert call(seqlen_ro=0) == bad                               # at least one position
+    assert call(cos=ctypes.c_void_p(0x1002)) == bad               # 4-byte aligned tables
+    assert call(w=None) == bad                                    # the rotated q copy needs room
+    assert call(w=ctypes.c_void_p(0x100010)) == bad               # 256-byte aligned workspace
+    assert call(nbytes=16) == bad
+    # workspace: the 16-bit q copy rounded to 256 bytes, then the split partials
+    r256 = lambda n: (n + 255) // 256 * 256
+    for splits in (1, 4, 0):
+        assert lib.fa_kvcache_rotary_workspace_size(2, 1, 8, 128, splits) == \
+            r256(2 * 1 * 8 * 128 * 2) + lib.fa_kvcache_workspace_size(2, 1, 8, 128, splits)
