@@ -344,6 +344,90 @@ def attn_bwd(dout, q, k, v, scale=None, causal=False, window_left=-1, window_rig
     return dq, dk, dv, delta
 
 
+@_masked_math
+def _bwd_row_terms(dout, q, k, v, b, h, rows, scale, causal, window_left, window_right, softcap,
+                   alibi_slopes):
+    """Per-row backward quantities of query ``rows`` of (batch b, q-head h),
+    each row on its own with the definitions of :func:`attn_bwd`: the raw
+    scores u against every key, P, dP = dO V^T, Delta = sum_j P dP and
+    dU = P (dP - Delta) [* (1 - tanh^2(u/softcap))].  Returns (P, dU, LSE,
+    Delta) with P and dU of shape (len(rows), Sk)."""
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    g = h // _check_heads(Hq, Hkv)
+    rows = np.asarray(rows)
+    Kg = np.asarray(k[b, :, g, :], np.float64)
+    Vg = np.asarray(v[b, :, g, :], np.float64)
+    u = scale * (np.asarray(q[b, rows, h, :], np.float64) @ Kg.T)      # (R, Sk)
+    s = transform_scores(u, softcap)
+    if alibi_slopes is not None:
+        s = s + alibi_bias(head_slopes(alibi_slopes, B, h)[b], rows, Sq, Sk)
+    vis = visible_rows(rows, Sq, Sk, causal, window_left, window_right)
+    s = np.where(vis, s, NEG_INF)
+    anyv = vis.any(axis=1)
+    m = np.where(anyv, s.max(axis=1), 0.0)
+    l = np.where(vis, np.exp(s - m[:, None]), 0.0).sum(axis=1)
+    lse = np.where(anyv, m + np.log(np.where(anyv, l, 1.0)), NEG_INF)
+    P = np.where(vis, np.exp(s - np.where(anyv, lse, 0.0)[:, None]), 0.0)
+    dP = np.asarray(dout[b, rows, h, :], np.float64) @ Vg.T             # (R, Sk)
+    delta = (P * dP).sum(axis=1)
+    dU = P * (dP - delta[:, None])
+    if softcap is not None and softcap > 0:
+        t = np.tanh(u / softcap)
+        dU = dU * (1.0 - t * t)
+    return P, dU, lse, delta
+
+
+def attn_bwd_rows(dout, q, k, v, b, h, rows, scale=None, causal=False, window_left=-1, window_right=-1,
+                  softcap=0.0, alibi_slopes=None):
+    """dQ of selected query rows of one (batch b, q-head h).
+
+    dQ_i = scale * sum_j dU_ij K_j, with dU of the row from the chain rule of
+    :func:`attn_bwd` (each row needs only its own scores).  Returns dq
+    (len(rows), D), LSE and Delta (len(rows),).  Used to check gradients of
+    problems too large to evaluate whole.
+    """
+    q = np.asarray(q)
+    D = q.shape[3]
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(D)
+    g = h // _check_heads(q.shape[2], k.shape[2])
+    _, dU, lse, delta = _bwd_row_terms(dout, q, k, v, b, h, rows, scale, causal, window_left, window_right,
+                                       softcap, alibi_slopes)
+    dq = scale * (dU @ np.asarray(k[b, :, g, :], np.float64))
+    return dq, lse, delta
+
+
+def attn_bwd_cols(dout, q, k, v, b, g, cols, scale=None, causal=False, window_left=-1, window_right=-1,
+                  softcap=0.0, alibi_slopes=None, row_chunk=1024):
+    """dK and dV of selected key rows ``cols`` of one (batch b, kv-head g).
+
+    dV_j = sum_{h in g} sum_i P_ij dO_i and dK_j = scale * sum_{h in g}
+    sum_i dU_ij Q_i: the sums of :func:`attn_bwd` over every query row i of
+    every q-head of the group.  A column needs the row statistics (LSE,
+    Delta) of every query, so all rows are evaluated with the per-row
+    definitions, ``row_chunk`` rows at a time to bound memory (the rows are
+    independent; only the sums over i run across chunks).  Returns dk, dv
+    (len(cols), D).
+    """
+    q = np.asarray(q)
+    B, Sq, Hq, D = q.shape
+    G = _check_heads(Hq, k.shape[2])
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(D)
+    cols = np.asarray(cols)
+    dk = np.zeros((len(cols), D))
+    dv = np.zeros((len(cols), D))
+    for h in range(g * G, (g + 1) * G):
+        for r0 in range(0, Sq, row_chunk):
+            rows = np.arange(r0, min(Sq, r0 + row_chunk))
+            P, dU, _, _ = _bwd_row_terms(dout, q, k, v, b, h, rows, scale, causal, window_left, window_right,
+                                         softcap, alibi_slopes)
+            dv += P[:, cols].T @ np.asarray(dout[b, rows, h, :], np.float64)
+            dk += scale * (dU[:, cols].T @ np.asarray(q[b, rows, h, :], np.float64))
+    return dk, dv
+
+
 # ---------------------------------------------------------------------------
 # incremental decoding with a (paged) KV cache
 # ---------------------------------------------------------------------------

@@ -422,6 +422,65 @@ def test_rows_equal_full_forward():
             np.testing.assert_allclose(lrow, lse[b, h, rows], atol=1e-14)
 
 
+@pytest.mark.parametrize("kw", [
+    dict(scale=0.3, causal=True, window_left=9, window_right=0, softcap=2.0),
+    dict(scale=0.4, causal=False, window_left=-1, window_right=-1, softcap=0.0),
+    dict(scale=0.5, causal=False, window_left=4, window_right=6, softcap=0.0),
+    dict(scale=0.2, causal=True, softcap=0.0, alibi_slopes=np.array([0.5, 0.25, 0.125, 1.0])),
+], ids=["causal-window-cap", "full", "two-sided-window", "alibi"])
+@pytest.mark.parametrize("Sq,Sk", [(37, 41), (41, 37), (30, 30)])
+def test_sampled_gradients_equal_full_backward(kw, Sq, Sk):
+    """attn_bwd_rows / attn_bwd_cols give the rows and columns of attn_bwd
+    (itself pinned by finite differences), GQA group sums included; a row
+    chunk smaller than Sq exercises sums that run across chunks."""
+    rng = np.random.default_rng(51)
+    q, k, v = _rand((2, Sq, 4, 8), rng), _rand((2, Sk, 2, 8), rng), _rand((2, Sk, 2, 8), rng)
+    do = _rand((2, Sq, 4, 8), rng)
+    dq, dk, dv, delta = oracle.attn_bwd(do, q, k, v, **kw)
+    _, lse = oracle.attn_fwd(q, k, v, **kw)
+    rows = np.array([0, 5, Sq // 2, Sq - 1])
+    cols = np.array([0, 3, Sk // 2, Sk - 1])
+    for b in range(2):
+        for h in range(4):
+            dq_r, lse_r, delta_r = oracle.attn_bwd_rows(do, q, k, v, b, h, rows, **kw)
+            np.testing.assert_allclose(dq_r, dq[b, rows, h], atol=1e-12)
+            np.testing.assert_allclose(lse_r, lse[b, h, rows], atol=1e-12)
+            np.testing.assert_allclose(delta_r, delta[b, h, rows], atol=1e-12)
+        for g in range(2):
+            dk_c, dv_c = oracle.attn_bwd_cols(do, q, k, v, b, g, cols, row_chunk=7, **kw)
+            np.testing.assert_allclose(dk_c, dk[b, cols, g], atol=1e-12)
+            np.testing.assert_allclose(dv_c, dv[b, cols, g], atol=1e-12)
+
+
+def test_sampled_gradients_match_finite_differences():
+    """Direct pin of the sampled-row and sampled-column gradients: central
+    differences of sum(dO * O) in one query row and one key/value row."""
+    rng = np.random.default_rng(52)
+    q, k, v = _rand((1, 6, 2, 4), rng), _rand((1, 7, 1, 4), rng), _rand((1, 7, 1, 4), rng)
+    do = _rand((1, 6, 2, 4), rng)
+    kw = dict(scale=0.7, causal=True, window_left=3, window_right=0, softcap=1.5)
+
+    def loss(qq, kk, vv):
+        return float((oracle.attn_fwd(qq, kk, vv, **kw)[0] * do).sum())
+
+    def num_grad(x, idx):
+        g = np.zeros(x.shape[-1])
+        for d in range(x.shape[-1]):
+            xp, xm = x.copy(), x.copy()
+            xp[idx + (d,)] += 1e-6
+            xm[idx + (d,)] -= 1e-6
+            a = [xp if x is t else t for t in (q, k, v)]
+            m = [xm if x is t else t for t in (q, k, v)]
+            g[d] = (loss(*a) - loss(*m)) / 2e-6
+        return g
+
+    dq_r, _, _ = oracle.attn_bwd_rows(do, q, k, v, 0, 1, np.array([4]), **kw)
+    np.testing.assert_allclose(dq_r[0], num_grad(q, (0, 4, 1)), rtol=1e-6, atol=1e-9)
+    dk_c, dv_c = oracle.attn_bwd_cols(do, q, k, v, 0, 0, np.array([3]), row_chunk=2, **kw)
+    np.testing.assert_allclose(dk_c[0], num_grad(k, (0, 3, 0)), rtol=1e-6, atol=1e-9)
+    np.testing.assert_allclose(dv_c[0], num_grad(v, (0, 3, 0)), rtol=1e-6, atol=1e-9)
+
+
 # ---------------------------------------------------------------------------
 # variable-length (packed) batches
 # ---------------------------------------------------------------------------
