@@ -128,3 +128,41 @@ def test_bwd_seqlen_sweep_head_slices(cfg):
         check_grad(dq[b:b + 1, :, h:h + 1], dq_r, "dQ")
         check_grad(dk[b:b + 1, :, h:h + 1], dk_r, "dK")
         check_grad(dv[b:b + 1, :, h:h + 1], dv_r, "dV")
+
+
+def _sample(S, rng, n):
+    idx = set([0, 1, S // 2, S - 2, S - 1]) | set(rng.integers(0, S, n).tolist())
+    return np.array(sorted(i for i in idx if 0 <= i < S))
+
+
+@pytest.mark.parametrize("cfg", [c for c in inputs.seqlen_sweep_configs() if c["Sq"] >= 4096],
+                         ids=lambda c: "H%dD%dS%d%s" % (c["Hq"], c["D"], c["Sq"], "c" if c["causal"] else "n"))
+def test_bwd_seqlen_sweep_sampled(cfg):
+    """Long sweep points (S = 4k, 8k, 16k) in the benchmark's launch
+    configuration: dQ of sampled query rows of two (batch, head) slices and
+    dK/dV of sampled key rows of one, against the oracle's per-row chain
+    rule, for the atomic and the ordered dQ accumulation."""
+    q, k, v, do = inputs.attention_inputs(cfg["B"], cfg["Sq"], cfg["Sk"], cfg["Hq"], cfg["Hkv"], cfg["D"],
+                                          cfg["dtype"], seed=cfg["seed"])
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    kw = dict(scale=cfg["scale"], causal=cfg["causal"])
+    out, lse = api.fa_fwd(qd, kd, vd, **kw)
+    grads = {}
+    for det in (False, True):
+        grads[det] = [t.cpu() for t in api.fa_bwd(dod, qd, kd, vd, out, lse, deterministic=det, **kw)]
+        torch.cuda.synchronize()
+        assert api.fa_last_device_status() == 0
+    Q, K, V, DO = (t.to(torch.float64).numpy() for t in (q, k, v, do))
+    rng = np.random.default_rng(cfg["seed"])
+    B, Hq, S = cfg["B"], cfg["Hq"], cfg["Sq"]
+    for b, h in ((0, 0), (B - 1, Hq - 1)):
+        rows = _sample(S, rng, 24)
+        dq_r, _, _ = oracle.attn_bwd_rows(DO, Q, K, V, b, h, rows, cfg["scale"], cfg["causal"])
+        for det, (dq, _, _) in grads.items():
+            check_grad(dq[b, rows, h], dq_r, f"dQ b{b} h{h} det={det}")
+    b, g = B - 1, cfg["Hkv"] - 1
+    cols = _sample(S, rng, 12)
+    dk_r, dv_r = oracle.attn_bwd_cols(DO, Q, K, V, b, g, cols, cfg["scale"], cfg["causal"])
+    for det, (_, dk, dv) in grads.items():
+        check_grad(dk[b, cols, g], dk_r, f"dK b{b} g{g} det={det}")
+        check_grad(dv[b, cols, g], dv_r, f"dV b{b} g{g} det={det}")
