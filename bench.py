@@ -34,7 +34,7 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-METRIC = "attention TFLOPs/s fwd+bwd (seqlen sweep 512-16k d64/d128, GQA+local, paged decode)"
+METRIC = "attention TFLOPs/s fwd & fwd+bwd at seqlen 512–16k, d64/128 (% of tensor peak)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # Launch whose per-launch roofline is reported for each kernel class.
@@ -276,7 +276,8 @@ class DecodeUnit:
         self.flops_dec = int(4 * cfg["D"] * cfg["Hq"] * lens.sum())
 
     def name(self):
-        return "decode-rotary" if self.rot else "decode"
+        base = "decode-rotary" if self.rot else "decode"
+        return base + ("-s%d" % self.num_splits if self.num_splits > 0 else "")
 
     def run(self, tracer):
         tracer.arm("decode", self)
@@ -378,33 +379,58 @@ class Pinned:
 
 
 class Tracer:
-    """Per-call CUDA event pairs around each call's dominant kernel (set through
-    fa_set_trace_events), accumulated per kernel class over the timed region."""
+    """Two kinds of CUDA event pairs, accumulated per kernel class over the
+    timed region: one immediately around each call's dominant kernel (set
+    through fa_set_trace_events, recorded by the library on the launching
+    stream), and one around the whole API call (every kernel of the call,
+    recorded on the same stream).  A call span runs from arm() to the next
+    arm() or disarm()."""
 
     def __init__(self, lib, enabled=False):
         self.lib = lib
         self.enabled = enabled
         self.pending = []
+        self.pending_calls = []
         self.totals = {}
+        self.per_unit = {}
+        self.per_call = {}
+        self._open = None
+
+    def _work(self, cls, unit):
+        return {"fwd": getattr(unit, "flops_fwd", 0), "bwd": getattr(unit, "flops_bwd", 0),
+                "fwd8": getattr(unit, "flops_fwd8", 0), "decode": getattr(unit, "bytes", 0)}[cls]
+
+    def _close_call(self):
+        if self._open is not None:
+            cls, name, a, work = self._open
+            b = torch.cuda.Event(enable_timing=True)
+            b.record()
+            self.pending_calls.append((cls, name, a, b, work))
+            self._open = None
 
     def arm(self, cls, unit):
         if not self.enabled:
             return
+        self._close_call()
+        work = self._work(cls, unit)
+        c = torch.cuda.Event(enable_timing=True)
+        c.record()
+        self._open = (cls, unit.name(), c, work)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         b.record()
         self.lib.fa_set_trace_events(a.cuda_event, b.cuda_event)
-        work = {"fwd": getattr(unit, "flops_fwd", 0), "bwd": getattr(unit, "flops_bwd", 0),
-                "fwd8": getattr(unit, "flops_fwd8", 0), "decode": getattr(unit, "bytes", 0)}[cls]
         self.pending.append((cls, unit.name(), a, b, work))
 
     def disarm(self):
         if self.enabled:
             self.lib.fa_set_trace_events(None, None)
+            self._close_call()
 
     def collect(self):
-        """Totals per kernel class; per (class, unit) totals in self.per_unit."""
-        self.per_unit = getattr(self, "per_unit", {})
+        """Totals per kernel class; per (class, unit) kernel totals in
+        self.per_unit and whole-call totals in self.per_call, each
+        [ms, count, work]."""
         for cls, name, a, b, work in self.pending:
             ms = a.elapsed_time(b)
             for d, key in ((self.totals, cls), (self.per_unit, (cls, name))):
@@ -412,7 +438,13 @@ class Tracer:
                 t[0] += ms
                 t[1] += 1
                 t[2] += work
+        for cls, name, a, b, work in self.pending_calls:
+            t = self.per_call.setdefault((cls, name), [0.0, 0, 0])
+            t[0] += a.elapsed_time(b)
+            t[1] += 1
+            t[2] += work
         self.pending = []
+        self.pending_calls = []
         return self.totals
 
 
@@ -434,6 +466,8 @@ def build_units(dev, workload, point=None):
         units.append(AttnUnit(inputs.gqa_local_config(), dev, deterministic=True))
     if workload in ("full", "decode"):
         units.append(DecodeUnit(inputs.paged_decode_config(), dev))
+        for n in (1, 4, 16):
+            units.append(DecodeUnit(inputs.paged_decode_config(), dev, num_splits=n))
     if workload == "small":
         units.append(AttnUnit(inputs.fwd_bwd_512_config(), dev))
     if workload == "varlen":
@@ -541,6 +575,59 @@ def cpu_oracle_sample(budget_s=12.0):
                        f"{el:.1f} s", elapsed_s=el, flops=n * flops)
 
 
+def _r(x, n=4):
+    return float(f"{x:.{n}g}")
+
+
+def per_config(tracer, peaks):
+    """Per workload point, from the whole-call event spans of the timed
+    region: forward and forward+backward TFLOP/s of every attention point
+    and their fractions of the measured bf16 tensor rates (sustained and
+    burst); GB/s of every paged-decode call (append + split-KV attention +
+    combine) beside its split kernel's, as fractions of the measured HBM
+    copy bandwidth."""
+    sus, burst, hbm = peaks["bf16_tflops_sustained"], peaks["bf16_tflops"], peaks["hbm_gbs"]
+    out = {}
+    for name in sorted({n for (_, n) in tracer.per_call}):
+        e = {}
+        f = tracer.per_call.get(("fwd", name)) or tracer.per_call.get(("fwd8", name))
+        bw = tracer.per_call.get(("bwd", name))
+        dc = tracer.per_call.get(("decode", name))
+        if f:
+            peak_scale = FP8_OVER_BF16 if ("fwd8", name) in tracer.per_call else 1.0
+            ms_f = f[0] / f[1]
+            tf = f[2] / f[1] / (ms_f / 1e3) / 1e12
+            e.update(fwd_ms=_r(ms_f), fwd_tflops=_r(tf), fwd_frac=_r(tf / (sus * peak_scale), 3),
+                     fwd_frac_burst=_r(tf / (burst * peak_scale), 3))
+        if f and bw:
+            ms_b = bw[0] / bw[1]
+            tb = bw[2] / bw[1] / (ms_b / 1e3) / 1e12
+            tfb = (f[2] / f[1] + bw[2] / bw[1]) / ((ms_f + ms_b) / 1e3) / 1e12
+            e.update(bwd_ms=_r(ms_b), bwd_tflops=_r(tb), fwdbwd_tflops=_r(tfb), fwdbwd_frac=_r(tfb / sus, 3),
+                     fwdbwd_frac_burst=_r(tfb / burst, 3))
+        if dc:
+            ms = dc[0] / dc[1]
+            gbs = dc[2] / dc[1] / (ms / 1e3) / 1e9
+            e.update(call_ms=_r(ms), call_gbs=_r(gbs), call_frac=_r(gbs / hbm, 3))
+            kt = tracer.per_unit.get(("decode", name))
+            if kt:
+                kg = kt[2] / kt[1] / (kt[0] / kt[1] / 1e3) / 1e9
+                e.update(split_kernel_gbs=_r(kg), split_kernel_frac=_r(kg / hbm, 3))
+        out[name] = e
+    # the long-sequence head-dim-128 sweep points (S >= 4096), both masks
+    long128 = [v for n, v in out.items() if n.startswith("H16D128S") and "-" not in n
+               and int(n[8:-1]) >= 4096 and "fwd_frac" in v]
+    summary = {}
+    if long128:
+        summary["d128_s4k_plus"] = {"fwd_frac_min": min(v["fwd_frac"] for v in long128),
+                                    "fwdbwd_frac_min": min(v["fwdbwd_frac"] for v in long128 if "fwdbwd_frac" in v),
+                                    "points": len(long128)}
+    dec = [v["call_frac"] for n, v in out.items() if n.startswith("decode") and "call_frac" in v]
+    if dec:
+        summary["decode_call_frac_min"] = min(dec)
+    return out, summary
+
+
 def max_over_ranks(ms, pg, dev):
     """The slowest rank's time: every rank contributes its own device-timed
     milliseconds (one all-reduce, taken in the same order on every rank)."""
@@ -625,6 +712,7 @@ def main():
     ms, launches = time_steps(units, args.steps, args.warmup, tracer, barrier=barrier)
     clk = clocks.stop()
     totals = tracer.collect()
+    points, points_summary = per_config(tracer, peaks)
     ms_max = max_over_ranks(ms, pg, dev)
     value = whole_job_tflops(world, flops_step, args.steps, ms_max)
 
@@ -709,8 +797,10 @@ def main():
                 "gpu_launches": launches,
                 "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h, "steps": args.e2e_steps},
-                "roofline": roof, "kernels": kernels, "cpu_baseline": cpu,
-                "clocks": clk}
+                "roofline": roof, "kernels": kernels, "per_config": points, "per_config_summary": points_summary,
+                "peaks": {"source": peak_src, "bf16_tflops_sustained": peaks["bf16_tflops_sustained"],
+                          "bf16_tflops": peaks["bf16_tflops"], "hbm_gbs": peaks["hbm_gbs"]},
+                "cpu_baseline": cpu, "clocks": clk}
         if detail:
             line["detail"] = detail
         print(json.dumps(line))
