@@ -682,3 +682,56 @@ def attn_fwd_fp8(q8, k8, v8, descale_q=None, descale_k=None, descale_v=None, sca
 
     return attn_fwd(q * fac(descale_q, G, Hq), k * fac(descale_k, 1, Hkv), v * fac(descale_v, 1, Hkv), scale,
                     causal, window_left, window_right, softcap)
+
+
+def e4m3_spacing(x):
+    """Distance between adjacent E4M3 values around non-negative x (the OCP
+    format of :func:`e4m3_decode`): 2^(e-3) for a normal value with exponent
+    e (x >= 2^-6), 2^-9 in the subnormal range."""
+    x = np.asarray(x, np.float64)
+    e = np.floor(np.log2(np.maximum(x, 2.0 ** -6)))
+    return np.where(x >= 2.0 ** -6, np.exp2(e - 3.0), 2.0 ** -9)
+
+
+@_masked_math
+def fp8_p_rounding_sigma(q, k, v, b, h, rows, scale=None, causal=False, window_left=-1, window_right=-1,
+                         softcap=0.0):
+    """Scale of the output error that rounding the probabilities to E4M3
+    introduces, per element of selected query rows of (batch b, q-head h).
+
+    q, k, v are the real inputs (decoded codes times their factors).  An
+    FP8 forward that forms O = sum_j R(P_j) v_j / sum_j R(P_j), with R the
+    round-to-nearest onto E4M3 and P_j = c e^{s_j - max s} for some factor c,
+    is off by sum_j (R(P_j) - P_j)(v_j - O) / sum_j R(P_j).  Each rounding
+    error lies within half the E4M3 spacing u_j at P_j; taking the errors as
+    independent and uniform (variance u_j^2 / 12) gives
+        sigma_id = sqrt(sum_j u_j^2 / 12 (v_jd - O_id)^2) / sum_j P_j,
+    evaluated here with c = 1 (the row's largest P equal to 1).  A factor
+    c >= 1 never more than doubles u_j / c (normal values keep a relative
+    spacing within [2^-4, 2^-3]; the fixed subnormal spacing only shrinks
+    relative to c P_j), so 2 sigma bounds the scale for every c >= 1.
+    Returns O (R, D), LSE (R,) and sigma (R, D).
+    """
+    q = np.asarray(q, np.float64)
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    g = h // _check_heads(Hq, Hkv)
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(D)
+    rows = np.asarray(rows)
+    Kg = np.asarray(k[b, :, g, :], np.float64)
+    Vg = np.asarray(v[b, :, g, :], np.float64)
+    s = transform_scores(scale * (q[b, rows, h, :] @ Kg.T), softcap)
+    vis = visible_rows(rows, Sq, Sk, causal, window_left, window_right)
+    s = np.where(vis, s, NEG_INF)
+    anyv = vis.any(axis=1)
+    m = np.where(anyv, s.max(axis=1), 0.0)
+    P = np.where(vis, np.exp(s - m[:, None]), 0.0)                      # largest P of a row = 1
+    l = np.where(anyv, P.sum(axis=1), 1.0)
+    o = np.where(anyv[:, None], (P @ Vg) / l[:, None], 0.0)
+    lse = np.where(anyv, m + np.log(l), NEG_INF)
+    var = np.where(vis, e4m3_spacing(P) ** 2 / 12.0, 0.0)                # (R, Sk)
+    sigma = np.zeros_like(o)
+    for r in range(len(rows)):                                          # one row at a time: (Sk, D) terms
+        sigma[r] = np.sqrt(var[r] @ (Vg - o[r]) ** 2) / l[r]
+    return o, lse, sigma

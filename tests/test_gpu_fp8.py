@@ -1,11 +1,16 @@
 """FP8 (E4M3) forward on the tcgen05 kernel against the float64 oracle.
 
 The scores are exact products of E4M3 values, so LSE is held to the usual
-1e-4.  O goes through P quantised to E4M3 (relative rounding <= 2^-4 per
-weight, zero mean): the expected relative RMS error of O from that alone is
-about 2^-4 / sqrt(3) ~ 0.036, and the bound used is 0.05.  A second case
-makes every P exactly representable (integer scores spanning <= 8 with
-scale ln 2, so P = 2^k with |k| <= 8) and holds O to the bf16 bound.
+1e-4.  O goes through P rounded to E4M3, so every element of O is held to a
+bound derived from that rounding: the oracle's fp8_p_rounding_sigma gives,
+per element, the scale sigma of the error that rounding the weights of its
+row to the E4M3 grid leaves in O (at any running-maximum factor the scale
+is at most 2 sigma), and each element must lie within 7 x 2 sigma plus half
+a bf16 unit of the oracle; the root mean square of error / sigma over all
+checked elements must stay below 2.5 (an error twice the E4M3 scale would
+fail it).  A second case makes every P exactly representable (integer
+scores spanning <= 8 with scale ln 2, so P = 2^k with |k| <= 8) and holds O
+to the bf16 bound.
 """
 
 import math
@@ -15,12 +20,49 @@ import pytest
 import torch
 
 import oracle
-from _parity import check_lse, check_out, f64, rel_fro
+from _parity import check_lse, check_out, f64, ulp
 from exact_attention_121_b200 import _lib, api, inputs
 
 pytestmark = pytest.mark.gpu
 
-FP8_REL_RMS = 0.05
+SIGMA_K = 7.0          # elementwise bound: SIGMA_K x (2 sigma) + half a bf16 unit
+RMS_RATIO_MAX = 2.5    # root mean square of error / sigma over the checked elements
+
+
+def _real(q8, k8, v8, dq, dk, dv):
+    """Real inputs: decoded codes times the (batch, kv-head) factors."""
+    q, k, v = (oracle.e4m3_decode(_codes(t)) for t in (q8, k8, v8))
+    B, Hq, Hkv = q.shape[0], q.shape[2], k.shape[2]
+    G = Hq // Hkv
+
+    def fac(d, rep):
+        if d is None:
+            return 1.0
+        return np.repeat(d.double().numpy().reshape(B, Hkv), rep, axis=1)[:, None, :, None]
+
+    return q * fac(dq, G), k * fac(dk, 1), v * fac(dv, 1)
+
+
+def check_fp8_rows(out, lse, real, b, h, rows, ratios, **kw):
+    """O of the given rows of (b, h) elementwise within the E4M3 rounding
+    bound, LSE within 1e-4; appends error / sigma to `ratios`."""
+    o_r, l_r, sig = oracle.fp8_p_rounding_sigma(*real, b, h, rows, **kw)
+    g = f64(out[b, rows, h])
+    assert np.isfinite(g).all()
+    err = np.abs(g - o_r)
+    half_ulp = 0.5 * ulp(o_r, torch.bfloat16)
+    tol = SIGMA_K * 2.0 * sig + half_ulp + 1e-6
+    bad = err > tol
+    assert not bad.any(), (f"O b{b} h{h}: {int(bad.sum())} elements outside the E4M3 bound; "
+                           f"worst err/tol {float((err / tol).max()):.2f}")
+    check_lse(lse[b, h, rows], l_r)
+    ratios.append((np.maximum(err - half_ulp, 0.0) / np.maximum(sig, 1e-12)).ravel())
+
+
+def check_rms_ratio(ratios):
+    r = float(np.sqrt(np.mean(np.concatenate(ratios) ** 2)))
+    assert r <= RMS_RATIO_MAX, f"RMS of error / sigma {r:.2f}"
+    return r
 
 # (B, Sq, Sk, Hq, Hkv, causal, window, softcap, with descales)
 CASES = [
@@ -36,9 +78,11 @@ def _codes(t):
     return t.view(torch.uint8).numpy()
 
 
-def _run(case, seed=70):
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "B%dS%dx%dH%d-%d%s%s" % (
+    c[0], c[1], c[2], c[3], c[4], "c" if c[5] else "", "w" if c[6] != (-1, -1) else ""))
+def test_fp8_forward_vs_oracle(case):
     B, Sq, Sk, Hq, Hkv, causal, window, cap, desc = case
-    q, k, v, dq, dk, dv = inputs.fp8_inputs(B, Sq, Sk, Hq, Hkv, 128, seed=seed)
+    q, k, v, dq, dk, dv = inputs.fp8_inputs(B, Sq, Sk, Hq, Hkv, 128, seed=70)
     if not desc:
         dq = dk = dv = None
     dev = lambda t: None if t is None else t.cuda()
@@ -46,21 +90,18 @@ def _run(case, seed=70):
                               softcap=cap)
     torch.cuda.synchronize()
     assert api.fa_last_device_status() == 0
+    real = _real(q, k, v, dq, dk, dv)
+    # the whole-tensor definition and the per-row one agree (LSE of every row)
     npd = lambda t: None if t is None else t.double().numpy()
-    o_r, l_r = oracle.attn_fwd_fp8(_codes(q), _codes(k), _codes(v), npd(dq), npd(dk), npd(dv), None, causal,
+    _, l_all = oracle.attn_fwd_fp8(_codes(q), _codes(k), _codes(v), npd(dq), npd(dk), npd(dv), None, causal,
                                    window[0], window[1], cap)
-    return out, lse, o_r, l_r
-
-
-@pytest.mark.parametrize("case", CASES, ids=lambda c: "B%dS%dx%dH%d-%d%s%s" % (
-    c[0], c[1], c[2], c[3], c[4], "c" if c[5] else "", "w" if c[6] != (-1, -1) else ""))
-def test_fp8_forward_vs_oracle(case):
-    out, lse, o_r, l_r = _run(case)
-    check_lse(lse, l_r)
-    g = f64(out)
-    assert np.isfinite(g).all()
-    e = rel_fro(out, o_r)
-    assert e <= FP8_REL_RMS, f"O relative RMS error {e:.3e}"
+    check_lse(lse, l_all)
+    ratios = []
+    for b in range(B):
+        for h in range(Hq):
+            check_fp8_rows(out, lse, real, b, h, np.arange(Sq), ratios, causal=causal, window_left=window[0],
+                           window_right=window[1], softcap=cap)
+    check_rms_ratio(ratios)
 
 
 def test_fp8_exact_powers_of_two_match_to_bf16():
@@ -95,13 +136,15 @@ def test_fp8_full_size_sampled_rows():
                                             seed=cfg["seed"], amp=cfg["amp"])
     out, lse = api.fa_fwd_fp8(q.cuda(), k.cuda(), v.cuda(), dq.cuda(), dk.cuda(), dv.cuda())
     torch.cuda.synchronize()
-    rows = np.array([0, 1, 255, 2048, 4095])
-    qv, kv, vv = (oracle.e4m3_decode(_codes(t)) for t in (q, k, v))
-    for b, h in ((0, 0), (3, 15)):
-        f = lambda d: float(d[b, h])
-        o_r, l_r = oracle.attn_fwd_rows(qv * f(dq), kv * f(dk), vv * f(dv), b, h, rows)
-        check_lse(lse[b, h, rows], l_r)
-        assert rel_fro(out[b, rows, h], o_r) <= FP8_REL_RMS
+    assert api.fa_last_device_status() == 0
+    rng = np.random.default_rng(cfg["seed"])
+    real = _real(q, k, v, dq, dk, dv)
+    ratios = []
+    for b, h in ((0, 0), (cfg["B"] - 1, cfg["Hq"] - 1), (1, 7)):
+        rows = np.unique(np.concatenate([[0, 1, 127, 128, 255, 2048, cfg["Sq"] - 1],
+                                         rng.integers(0, cfg["Sq"], 24)]))
+        check_fp8_rows(out, lse, real, b, h, rows, ratios, causal=cfg["causal"])
+    check_rms_ratio(ratios)
 
 
 def test_fp8_refusals():

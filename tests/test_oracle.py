@@ -872,3 +872,64 @@ def test_planted_fp8_descale_by_q_head_is_caught(monkeypatch):
     with pytest.raises(AssertionError):
         test_fp8_descales_act_per_batch_and_kv_head()
     monkeypatch.setattr(oracle, "attn_fwd_fp8", orig)
+
+
+# ---------------------------------------------------------------------------
+# FP8: spacing of the E4M3 grid and the P-rounding error scale
+# ---------------------------------------------------------------------------
+
+def _e4m3_grid():
+    """Sorted non-negative finite E4M3 values, decoded from all 128 codes
+    with the sign bit clear."""
+    vals = oracle.e4m3_decode(np.arange(128, dtype=np.uint8))
+    return np.sort(vals[np.isfinite(vals)])
+
+
+def test_e4m3_spacing_matches_the_code_table():
+    grid = _e4m3_grid()
+    gaps = np.diff(grid)
+    np.testing.assert_array_equal(oracle.e4m3_spacing(grid[:-1]), gaps)
+    assert grid[-1] == 448.0 and grid[1] == 2.0 ** -9
+
+
+def _round_e4m3(x):
+    """Round non-negative x to the nearest E4M3 value (ties to the even
+    mantissa, i.e. the even code), by search in the decoded table."""
+    grid = _e4m3_grid()
+    i = np.clip(np.searchsorted(grid, x), 1, len(grid) - 1)
+    lo, hi = grid[i - 1], grid[i]
+    pick_hi = (x - lo > hi - x) | ((x - lo == hi - x) & (i % 2 == 0))
+    return np.where(pick_hi, hi, lo)
+
+
+@pytest.mark.parametrize("c", [1.0, 3.7, 200.0])
+def test_fp8_sigma_bounds_e4m3_rounded_probabilities(c):
+    """Quantising c * P to E4M3 (c = the factor a running maximum leaves on
+    the row's largest probability, 1 <= c <= 2^8) stays within 7 x 2 sigma
+    elementwise, and at c = 1 the errors have RMS ~ sigma: sigma is the
+    scale of the error, not a vacuous bound."""
+    rng = np.random.default_rng(60)
+    B, Sq, Sk, H, D = 1, 48, 700, 2, 16
+    q, k, v = _rand((B, Sq, H, D), rng), _rand((B, Sk, H, D), rng), _rand((B, Sk, H, D), rng)
+    kw = dict(scale=0.25, causal=True)
+    ratios = []
+    for h in range(H):
+        rows = np.arange(Sq)
+        o, lse, sig = oracle.fp8_p_rounding_sigma(q, k, v, 0, h, rows, **kw)
+        o_ref, lse_ref = oracle.attn_fwd_rows(q, k, v, 0, h, rows, **kw)
+        np.testing.assert_allclose(o, o_ref, atol=1e-13)
+        np.testing.assert_allclose(lse, lse_ref, atol=1e-13)
+        u = 0.25 * (q[0, :, h, :] @ k[0, :, h, :].T)
+        vis = oracle.visible(Sq, Sk, True)
+        u = np.where(vis, u, -np.inf)
+        P = np.where(vis, np.exp(u - u.max(axis=1, keepdims=True)), 0.0) * c
+        R = _round_e4m3(P)
+        oq = (R @ v[0, :, h, :]) / R.sum(axis=1, keepdims=True)
+        err = np.abs(oq - o_ref)
+        assert (err <= 14.0 * sig + 1e-12).all(), float((err / sig).max())
+        ratios.append(err / sig)
+    rms = float(np.sqrt(np.mean(np.concatenate(ratios) ** 2)))
+    if c == 1.0:
+        assert 0.5 <= rms <= 1.5, rms
+    else:
+        assert rms <= 2.0, rms
