@@ -10,7 +10,7 @@ import os
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfa.so")
 
-FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_BOUNDS = range(6)
 FA_FP16, FA_BF16 = 0, 1
 FA_MAX_SPLITS = 64
 
@@ -51,6 +51,7 @@ SIGNATURES = {
     "fa_selftest_bounded_wait": (_I, [_P, _I, ctypes.c_longlong, _P]),
     "fa_selftest_exp2_poly": (_I, [_P, _P, _I, _P]),
     "fa_last_launch_count": (_I, []),
+    "fa_build_flags": (_I, []),
     "fa_set_trace_events": (None, [_P, _P]),
 }
 

@@ -5,6 +5,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "fa.h"
 #include "fa_common.cuh"
 #include "fa_kernels.h"
@@ -20,7 +22,10 @@ namespace {
 __device__ int g_fa_status = 0;
 
 constexpr int kMaxDevices = 64;
-int* g_status_ptr[kMaxDevices] = {nullptr};
+// Device address of the status word per device, looked up once (with that
+// device current).  Atomic slots: concurrent first calls from several host
+// threads store the same address.
+std::atomic<int*> g_status_ptr[kMaxDevices];
 int g_fwd_kernel_choice = 0;
 int g_bwd_kernel_choice = 0;
 // Whether the automatic choice uses the tcgen05 forward kernel.
@@ -31,15 +36,24 @@ thread_local int g_last_launches = 0;
 int* status_ptr() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  if (!g_status_ptr[dev]) {
+  int* ptr = g_status_ptr[dev].load(std::memory_order_acquire);
+  if (!ptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_fa_status) != cudaSuccess) return nullptr;
-    g_status_ptr[dev] = static_cast<int*>(p);
+    ptr = static_cast<int*>(p);
+    g_status_ptr[dev].store(ptr, std::memory_order_release);
   }
-  return g_status_ptr[dev];
+  return ptr;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Largest element offset + 1 of a (B, S, H, D) tensor with (batch, token,
+// head) strides; 0 when it is empty.
+long long extent(long long B, long long S, long long H, int D, const long long st[3]) {
+  if (B <= 0 || S <= 0 || H <= 0) return 0;
+  return (B - 1) * st[0] + (S - 1) * st[1] + (H - 1) * st[2] + D;
+}
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 fa_status check_common(int B, int Sq, int Hq, int Hkv, int D, fa_dtype dt, float scale, float softcap) {
@@ -139,6 +153,7 @@ const char* fa_status_string(fa_status s) {
     case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
     case FA_ERR_CUDA: return "FA_ERR_CUDA";
     case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    case FA_ERR_BOUNDS: return "FA_ERR_BOUNDS";
   }
   return "FA_ERR_UNKNOWN";
 }
@@ -148,6 +163,14 @@ void fa_set_fwd_kernel(int which) { g_fwd_kernel_choice = which; }
 void fa_set_bwd_kernel(int which) { g_bwd_kernel_choice = which; }
 
 int fa_last_launch_count(void) { return g_last_launches; }
+
+int fa_build_flags(void) {
+#ifdef FA_DEBUG_BOUNDS
+  return FA_BUILD_DEBUG_BOUNDS;
+#else
+  return 0;
+#endif
+}
 
 // (batch, token, head) element strides of a packed (B, S, H, D) tensor
 static void contiguous_strides(long long st[3], int S, int H, int D) {
@@ -203,6 +226,8 @@ static fa_status fwd_impl(const void* q, const void* k, const void* v, void* out
   fill_cap(scale, softcap, &p.softcap, &p.cap_in, &p.cap_log2, &p.scale_log2);
   p.alibi = alibi;
   p.alibi_bstride = alibi_bstride;
+  p.ext_o = extent(B, Sq, Hq, D, p.st_o);
+  p.n_stat = (long long)B * Hq * Sq;
   p.status = status_ptr();
   if (!p.status) return FA_ERR_CUDA;
   int launches = 0;
@@ -272,6 +297,8 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, flo
   contiguous_strides(p.st_v, Sk, Hkv, D);
   contiguous_strides(p.st_o, Sq, Hq, D);
   p.descale_q = descale_q; p.descale_k = descale_k; p.descale_v = descale_v;
+  p.ext_o = extent(B, Sq, Hq, D, p.st_o);
+  p.n_stat = (long long)B * Hq * Sq;
   fold_window(causal, window_left, window_right, &p.wl, &p.wr);
   scale = resolve_scale(scale, D);
   fill_cap(scale, softcap, &p.softcap, &p.cap_in, &p.cap_log2, &p.scale_log2);
@@ -351,6 +378,13 @@ static fa_status bwd_impl(const void* dout, const void* q, const void* k, const 
   fill_cap(scale, softcap, &p.softcap, &p.cap_in, &p.cap_log2, &p.scale_log2);
   p.deterministic = deterministic ? 1 : 0;
   p.kernel_choice = g_bwd_kernel_choice;
+  p.ext_do = extent(B, Sq, Hq, D, p.st_do);
+  p.ext_o = extent(B, Sq, Hq, D, p.st_o);
+  p.ext_dq = extent(B, Sq, Hq, D, p.st_dq);
+  p.ext_dk = extent(B, Sk, Hkv, D, p.st_dk);
+  p.ext_dv = extent(B, Sk, Hkv, D, p.st_dv);
+  p.n_stat = (long long)B * Hq * Sq;
+  p.n_accum = (long long)B * Sq * Hq * D;
   p.alibi = alibi;
   p.alibi_bstride = alibi_bstride;
   // strided tensors and ALiBi run on the tcgen05 kernel only
@@ -427,6 +461,8 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* out, 
   // packed tensors: one batch of tokens (batch stride 0)
   for (long long* st : {p.st_q, p.st_o}) { st[0] = 0; st[1] = (long long)Hq * D; st[2] = D; }
   for (long long* st : {p.st_k, p.st_v}) { st[0] = 0; st[1] = (long long)Hkv * D; st[2] = D; }
+  p.ext_o = extent(1, total_q, Hq, D, p.st_o);
+  p.n_stat = (long long)Hq * total_q;
   fold_window(causal, window_left, window_right, &p.wl, &p.wr);
   scale = resolve_scale(scale, D);
   fill_cap(scale, softcap, &p.softcap, &p.cap_in, &p.cap_log2, &p.scale_log2);
@@ -486,6 +522,13 @@ fa_status fa_bwd_varlen(const void* dout, const void* q, const void* k, const vo
   for (long long* st : {p.st_do, p.st_q, p.st_o, p.st_dq}) { st[0] = 0; st[1] = (long long)Hq * D; st[2] = D; }
   for (long long* st : {p.st_k, p.st_v, p.st_dk, p.st_dv}) { st[0] = 0; st[1] = (long long)Hkv * D; st[2] = D; }
   p.rows_packed = 1;
+  p.ext_do = extent(1, total_q, Hq, D, p.st_do);
+  p.ext_o = extent(1, total_q, Hq, D, p.st_o);
+  p.ext_dq = extent(1, total_q, Hq, D, p.st_dq);
+  p.ext_dk = extent(1, total_k, Hkv, D, p.st_dk);
+  p.ext_dv = extent(1, total_k, Hkv, D, p.st_dv);
+  p.n_stat = (long long)Hq * total_q;
+  p.n_accum = (long long)total_q * Hq * D;
   fold_window(causal, window_left, window_right, &p.wl, &p.wr);
   scale = resolve_scale(scale, D);
   p.scale = scale;
@@ -503,12 +546,39 @@ fa_status fa_bwd_varlen(const void* dout, const void* q, const void* k, const vo
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+}  // extern "C"
+
+namespace fa {
+// Split count of the kvcache calls when the caller gives none: enough
+// (b, kv-head, split) work items for about seven waves of two CTAs per SM,
+// never more splits than pages of the longest sequence.
+int kvcache_auto_splits(int B, int Sq, int Hq, int Hkv, int page_size, int paged, int max_pages_per_seq,
+                        int num_pages_or_max_seqlen) {
+  if (B <= 0 || Sq <= 0 || Hkv <= 0 || Hq <= 0 || page_size <= 0) return 1;
+  const long long cap_tokens = paged ? (long long)max_pages_per_seq * page_size : num_pages_or_max_seqlen;
+  const long long max_units = (cap_tokens + page_size - 1) / page_size;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int nrt = (Sq * (Hq / Hkv) + 15) / 16;
+  const long long units = (long long)B * Hkv * nrt;
+  long long n = (14LL * sms + units - 1) / units;  // ~7 waves of 2 CTAs per SM
+  if (n > FA_MAX_SPLITS) n = FA_MAX_SPLITS;
+  if (n > max_units) n = max_units;
+  return n < 1 ? 1 : (int)n;
+}
+}  // namespace fa
+
+extern "C" {
+
 size_t fa_kvcache_workspace_size(int B, int Sq, int Hq, int D, int num_splits) {
   if (B < 0 || Sq < 0 || Hq <= 0 || (D != 64 && D != 128)) return 0;
   if (num_splits <= 0 || num_splits > FA_MAX_SPLITS) num_splits = FA_MAX_SPLITS;
   if (num_splits == 1) return 0;
   const size_t rows = (size_t)num_splits * B * Hq * Sq;
-  return round256(rows * D * sizeof(float)) + round256(rows * sizeof(float));
+  // partial outputs, partial LSEs, and one split counter per (b, kv-head,
+  // packed-row tile), at most B * Hq * Sq of them
+  return round256(rows * D * sizeof(float)) + round256(rows * sizeof(float)) +
+         round256((size_t)B * Hq * Sq * sizeof(int));
 }
 
 struct RotaryArgs {
@@ -549,24 +619,14 @@ static fa_status kvcache_impl(const void* q, void* k_cache, void* v_cache, const
   p.max_seqlen = paged ? 0 : num_pages_or_max_seqlen;
   p.out = out; p.lse = lse;
   p.B = B; p.Sq = Sq; p.Snew = Snew; p.Hq = Hq; p.Hkv = Hkv; p.D = D; p.G = Hq / Hkv;
+  p.n_out = (long long)B * Sq * Hq * D;
+  p.ext_cache = paged ? (long long)num_pages_or_max_seqlen * page_size * Hkv * D
+                      : (long long)B * num_pages_or_max_seqlen * Hkv * D;
   fold_window(causal, window_left, window_right, &p.wl, &p.wr);
   scale = resolve_scale(scale, D);
   fill_cap(scale, softcap, &p.softcap, &p.cap_in, &p.cap_log2, &p.scale_log2);
-  // Split count: explicit, else enough (b, kv-head, split) work items for about
-  // seven waves of two CTAs per SM, never more splits than pages of the
-  // longest sequence.
-  const int cap_tokens = paged ? max_pages_per_seq * page_size : num_pages_or_max_seqlen;
-  const int max_units = (cap_tokens + page_size - 1) / page_size;
-  if (num_splits <= 0) {
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int nrt = (Sq * p.G + 15) / 16;
-    const long long units = (long long)B * Hkv * nrt;
-    long long n = (14LL * sms + units - 1) / units;  // ~7 waves of 2 CTAs per SM
-    if (n > FA_MAX_SPLITS) n = FA_MAX_SPLITS;
-    if (n > max_units) n = max_units;
-    num_splits = n < 1 ? 1 : (int)n;
-  }
+  if (num_splits <= 0) num_splits = fa::kvcache_auto_splits(B, Sq, Hq, Hkv, page_size, paged, max_pages_per_seq,
+                                                           num_pages_or_max_seqlen);
   p.num_splits = num_splits;
   if (rot) {
     if (!rot->cos || !rot->sin || rot->dim <= 0 || rot->dim % 2 || rot->dim > D || rot->len <= 0)
@@ -584,11 +644,16 @@ static fa_status kvcache_impl(const void* q, void* k_cache, void* v_cache, const
   }
   if (num_splits > 1) {
     const size_t rows = (size_t)num_splits * B * Hq * Sq;
-    const size_t need = round256(rows * D * sizeof(float)) + round256(rows * sizeof(float));
+    const size_t need = fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits);
     if (!workspace || ws_bytes < need) return FA_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
-    p.o_part = static_cast<float*>(workspace);
-    p.lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round256(rows * D * sizeof(float)));
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p.o_part = reinterpret_cast<float*>(ws);
+    ws += round256(rows * D * sizeof(float));
+    p.lse_part = reinterpret_cast<float*>(ws);
+    ws += round256(rows * sizeof(float));
+    p.split_count = reinterpret_cast<int*>(ws);
+    p.n_part = (long long)rows;
   }
   p.status = status_ptr();
   if (!p.status) return FA_ERR_CUDA;

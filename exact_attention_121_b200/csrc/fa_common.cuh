@@ -18,6 +18,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 // Status word codes written by kernels (same values as fa_status).
 constexpr int kStatusTimeout = FA_ERR_TIMEOUT;
 constexpr int kStatusBadArg = FA_ERR_INVALID_ARG;
+constexpr int kStatusBounds = FA_ERR_BOUNDS;
 
 // Default time limit of every device-side wait.
 constexpr unsigned long long kWaitLimitNs = 10ull * 1000ull * 1000ull * 1000ull;
@@ -25,6 +26,20 @@ constexpr unsigned long long kWaitLimitNs = 10ull * 1000ull * 1000ull * 1000ull;
 __device__ __forceinline__ void report_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
+
+// Index checks of the bounds-checked build (compiled with -DFA_DEBUG_BOUNDS):
+// FA_IN_BOUNDS(cond, status) is `cond`, and a false `cond` records
+// FA_ERR_BOUNDS in the status word; callers skip the access it guards.  In
+// the normal build it is the constant `true` and costs nothing.
+#ifdef FA_DEBUG_BOUNDS
+__device__ __forceinline__ bool in_bounds_checked(bool ok, int* status) {
+  if (!ok) report_status(status, kStatusBounds);
+  return ok;
+}
+#define FA_IN_BOUNDS(cond, status) (::fa::in_bounds_checked((cond), (status)))
+#else
+#define FA_IN_BOUNDS(cond, status) (true)
+#endif
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
   unsigned long long t;

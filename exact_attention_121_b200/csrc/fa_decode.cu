@@ -509,10 +509,43 @@ cudaError_t launch_split(const DecodeParams& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// Write k_new / v_new (rotated with rotary tables) into the cache.
+template <typename T>
+cudaError_t launch_append(const DecodeParams& p, cudaStream_t s, int* launches) {
+  const int threads = 256;
+  if (p.rot_cos) {
+    const long long total = (long long)p.B * p.Snew * p.Hkv * p.D;
+    const int blocks = (int)((total + threads - 1) / threads < 4096 ? (total + threads - 1) / threads : 4096);
+    kvcache_append_rotary_kernel<T><<<blocks, threads, 0, s>>>(p);
+  } else {
+    const long long total = (long long)p.B * p.Snew * p.Hkv * (p.D / 8);
+    const int blocks = (int)((total + threads - 1) / threads < 4096 ? (total + threads - 1) / threads : 4096);
+    kvcache_append_kernel<T><<<blocks, threads, 0, s>>>(p);
+  }
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) ++*launches;
+  return e;
+}
+
+template <typename T>
+cudaError_t launch_combine(const DecodeParams& p, cudaStream_t s, int* launches) {
+  const long long rows = (long long)p.B * p.Hq * p.Sq;
+  if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;  // one block per row
+  static_assert(FA_MAX_SPLITS <= kCombineWarps * 32, "one thread per split for the LSE maximum");
+  if (p.D == 64)
+    decode_combine_kernel<T, 64><<<(unsigned)rows, kCombineWarps * 32, 0, s>>>(p);
+  else
+    decode_combine_kernel<T, 128><<<(unsigned)rows, kCombineWarps * 32, 0, s>>>(p);
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) ++*launches;
+  return e;
+}
+
 template <typename T>
 cudaError_t launch_decode_t(const DecodeParams& p_in, cudaStream_t s, int* launches) {
   cudaError_t e;
   DecodeParams p = p_in;
+  p.fuse_append = 0;
   if (p.rot_cos) {
     // rotate q into the scratch copy the attention kernels then read
     const long long total = (long long)p.B * p.Sq * p.Hq * p.D;
@@ -524,48 +557,44 @@ cudaError_t launch_decode_t(const DecodeParams& p_in, cudaStream_t s, int* launc
     ++*launches;
     p.q = p.q_rot;
   }
-  if (p.Snew > 0 && p.rot_cos) {
-    const long long total = (long long)p.B * p.Snew * p.Hkv * p.D;
-    const int threads = 256;
-    const int blocks = (int)((total + threads - 1) / threads < 4096 ? (total + threads - 1) / threads : 4096);
-    kvcache_append_rotary_kernel<T><<<blocks, threads, 0, s>>>(p);
-    e = cudaGetLastError();
+  bool appended = false;
+  if (decode_tma_supported(p)) {
+    // One kernel for the whole call: the TMA split kernel appends the new
+    // rows itself (not with rotary tables: those rows are rotated by the
+    // append kernel first) and merges its splits through the zeroed counters.
+    if (p.Snew > 0 && p.rot_cos) {
+      e = launch_append<T>(p, s, launches);
+      if (e != cudaSuccess) return e;
+      appended = true;
+    }
+    DecodeParams pf = p;
+    pf.fuse_append = p.Snew > 0 && !p.rot_cos;
+    if (p.num_splits > 1 && pf.split_count) {
+      const int nrt = (p.Sq * p.G + 15) / 16;
+      e = cudaMemsetAsync(pf.split_count, 0, (size_t)p.B * p.Hkv * nrt * sizeof(int), s);
+      if (e != cudaSuccess) return e;
+    }
+    e = launch_decode_split_tma(pf, Elem<T>::kBf16 ? FA_BF16 : FA_FP16, s);
+    if (e == cudaSuccess) {
+      ++*launches;
+      return (p.num_splits > 1 && !pf.split_count) ? launch_combine<T>(p, s, launches) : cudaSuccess;
+    }
+    if (e != cudaErrorNotSupported) return e;
+  }
+  // pages the TMA boxes cannot follow: append, the cp.async gather kernel,
+  // then the combine pass
+  if (p.Snew > 0 && !appended) {
+    e = launch_append<T>(p, s, launches);
     if (e != cudaSuccess) return e;
-    ++*launches;
-  } else if (p.Snew > 0) {
-    const long long total = (long long)p.B * p.Snew * p.Hkv * (p.D / 8);
-    const int threads = 256;
-    const int blocks = (int)((total + threads - 1) / threads < 4096 ? (total + threads - 1) / threads : 4096);
-    kvcache_append_kernel<T><<<blocks, threads, 0, s>>>(p);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    ++*launches;
   }
   const bool cap = p.softcap > 0.f;
-  e = cudaErrorNotSupported;
-  if (decode_tma_supported(p)) e = launch_decode_split_tma(p, Elem<T>::kBf16 ? FA_BF16 : FA_FP16, s);
-  if (e == cudaErrorNotSupported) {
-    // pages that are not a multiple of the TMA tile: the cp.async gather kernel
-    if (p.D == 64)
-      e = cap ? launch_split<T, 64, true>(p, s) : launch_split<T, 64, false>(p, s);
-    else
-      e = cap ? launch_split<T, 128, true>(p, s) : launch_split<T, 128, false>(p, s);
-  }
+  if (p.D == 64)
+    e = cap ? launch_split<T, 64, true>(p, s) : launch_split<T, 64, false>(p, s);
+  else
+    e = cap ? launch_split<T, 128, true>(p, s) : launch_split<T, 128, false>(p, s);
   if (e != cudaSuccess) return e;
   ++*launches;
-  if (p.num_splits > 1) {
-    const long long rows = (long long)p.B * p.Hq * p.Sq;
-    if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;  // one block per row
-    static_assert(FA_MAX_SPLITS <= kCombineWarps * 32, "one thread per split for the LSE maximum");
-    if (p.D == 64)
-      decode_combine_kernel<T, 64><<<(unsigned)rows, kCombineWarps * 32, 0, s>>>(p);
-    else
-      decode_combine_kernel<T, 128><<<(unsigned)rows, kCombineWarps * 32, 0, s>>>(p);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    ++*launches;
-  }
-  return cudaSuccess;
+  return p.num_splits > 1 ? launch_combine<T>(p, s, launches) : cudaSuccess;
 }
 
 }  // namespace

@@ -4,14 +4,24 @@
 //
 // The step is bound by HBM bandwidth, so the kernel is built around keeping
 // enough bytes in flight: one producer warp looks up the block table once per
-// 32-token tile and issues one TMA box per 64 head-dim columns of K and V into
-// a 6-stage shared-memory ring (96 KB per CTA, two CTAs per SM); three
-// consumer warps each own two stages, so every warp computes on one tile while
-// its next tile lands.  The q-heads of the GQA group (times the query rows)
-// are packed into the 16 rows of an mma.sync tile, so each K/V byte is read
-// from HBM once for the whole group.  Partial results per split go to the
-// workspace (or straight to the output when there is one split) exactly as in
-// the cp.async kernel, whose combine pass merges them.
+// TMA box (a 32-token tile is one box, or two / four boxes when pages hold 16
+// or 8 tokens) and issues one box per 64 head-dim columns of K and V into a
+// 6-stage shared-memory ring (96 KB per CTA, two CTAs per SM); three consumer
+// warps each own two stages, so every warp computes on one tile while its
+// next tile lands.  The q-heads of the GQA group (times the query rows) are
+// packed into the 16 rows of an mma.sync tile, so each K/V byte is read from
+// HBM once for the whole group.
+//
+// The whole call can run as this one kernel:
+//   * append (fuse_append): the CTAs of the first row tile write the new
+//     rows k_new / v_new into the cache, spread over the splits, and every
+//     CTA whose tile covers a new row takes that row from k_new / v_new in
+//     shared memory, so no CTA depends on another's cache write;
+//   * combine (split_count): each split writes its partial output and LSE to
+//     the workspace, then counts itself done on its (b, kv-head, row tile)
+//     counter; the CTA that finishes last merges the splits
+//     (LSE = ln sum_s e^{LSE_s}, O = sum_s e^{LSE_s - LSE} O_s) and clears
+//     the counter.
 #include <math.h>
 
 #include "fa_common.cuh"
@@ -41,7 +51,8 @@ struct DecCfg {
   static constexpr int OFF_ST = 16 * D * 2 > 1024 ? 16 * D * 2 : 1024;
   static constexpr int OFF_BAR = OFF_ST + kStages * STAGE;
   static constexpr int OFF_FLAG = OFF_BAR + 2 * kStages * 8;
-  static constexpr int SMEM = OFF_FLAG + kStages * 4 + 1024;
+  static constexpr int OFF_LAST = OFF_FLAG + kStages * 4;
+  static constexpr int SMEM = OFF_LAST + 4 + 1024;
 };
 
 // Byte offset of logical 16-byte chunk j of row r inside a TMA-swizzled tile
@@ -53,6 +64,21 @@ __device__ __forceinline__ uint32_t tma_sw(int r, int j) {
 
 __device__ __forceinline__ int cap_tokens(const DecodeParams& p) {
   return p.paged ? p.max_pages_per_seq * p.page_size : p.max_seqlen;
+}
+
+// Element offset of (sequence b, position pos, kv-head g) in the cache, or -1
+// when the position or its page is outside the cache.
+__device__ __forceinline__ long long cache_elem(const DecodeParams& p, int b, int pos, int g) {
+  if (pos < 0 || pos >= cap_tokens(p)) return -1;
+  long long row;
+  if (p.paged) {
+    const int page = __ldg(p.block_table + (size_t)b * p.max_pages_per_seq + pos / p.page_size);
+    if (page < 0 || page >= p.capacity_pages) return -1;
+    row = (long long)page * p.page_size + pos % p.page_size;
+  } else {
+    row = (long long)b * p.max_seqlen + pos;
+  }
+  return (row * p.Hkv + g) * p.D;
 }
 
 template <typename T, int D, bool kCap>
@@ -113,16 +139,23 @@ __global__ void __launch_bounds__(kThreadsD, 1)
           break;
         }
         const int t = t0 + tt * kTokT;
-        int c2, c3;
+        // boxes of R rows; each lies inside one page (R divides the page
+        // size and t0 starts a page); boxes past the split end are not loaded
+        const int R = p.box_rows;
+        const int nbox = min(kTokT / R, (t1 - t + R - 1) / R);
+        int c2[kTokT / 8], c3[kTokT / 8];
         bool ok = true;
-        if (p.paged) {
-          const int page = __ldg(p.block_table + (size_t)b * p.max_pages_per_seq + t / p.page_size);
-          ok = page >= 0 && page < p.capacity_pages;
-          c2 = t % p.page_size;
-          c3 = page;
-        } else {
-          c2 = t;
-          c3 = b;
+        for (int x = 0; x < nbox; ++x) {
+          const int tx = t + x * R;
+          if (p.paged) {
+            const int page = __ldg(p.block_table + (size_t)b * p.max_pages_per_seq + tx / p.page_size);
+            ok = ok && page >= 0 && page < p.capacity_pages;
+            c2[x] = tx % p.page_size;
+            c3[x] = page;
+          } else {
+            c2[x] = tx;
+            c3[x] = b;
+          }
         }
         flag[st] = ok ? 1 : 0;
         if (!ok) {
@@ -131,11 +164,12 @@ __global__ void __launch_bounds__(kThreadsD, 1)
           continue;
         }
         const uint32_t kst = sb + C::OFF_ST + st * C::STAGE;
-        mbar_expect_tx(full(st), C::STAGE);
-        for (int c = 0; c < C::NCH; ++c) {
-          tma_load_4d(kst + c * C::CHUNK, &tmK, c * 64, g, c2, c3, full(st));
-          tma_load_4d(kst + C::KT + c * C::CHUNK, &tmV, c * 64, g, c2, c3, full(st));
-        }
+        mbar_expect_tx(full(st), (uint32_t)(nbox * R * 128 * C::NCH * 2));
+        for (int x = 0; x < nbox; ++x)
+          for (int c = 0; c < C::NCH; ++c) {
+            tma_load_4d(kst + c * C::CHUNK + x * R * 128, &tmK, c * 64, g, c2[x], c3[x], full(st));
+            tma_load_4d(kst + C::KT + c * C::CHUNK + x * R * 128, &tmV, c * 64, g, c2[x], c3[x], full(st));
+          }
       }
     }
     return;  // the consumers never wait on this warp again
@@ -149,12 +183,36 @@ __global__ void __launch_bounds__(kThreadsD, 1)
     const bool okr = pr < rows;
     const int sq = okr ? pr / p.G : 0;
     const int h = g * p.G + (okr ? pr % p.G : 0);
-    const T* src = reinterpret_cast<const T*>(p.q) + (((size_t)b * p.Sq + sq) * p.Hq + h) * D + c * 8;
-    cp_async_16(smem_u32(sQ) + swz_offset<D>(r, c), src, okr ? 16 : 0);
+    const long long qi = (((long long)b * p.Sq + sq) * p.Hq + h) * D + c * 8;
+    const bool ld = okr && FA_IN_BOUNDS(qi >= 0 && qi + 8 <= p.n_out, p.status);
+    const T* src = reinterpret_cast<const T*>(p.q) + (ld ? qi : 0);
+    cp_async_16(smem_u32(sQ) + swz_offset<D>(r, c), src, ld ? 16 : 0);
   }
   cp_async_commit();
   cp_async_wait<0>();
   named_bar_sync(1, 32 * kConsumers);
+
+  if (p.fuse_append && rt == 0) {
+    // the cache write of this call's new rows for (b, g): split s takes rows
+    // s, s + num_splits, ...; positions outside the cache are reported and
+    // skipped (as the separate append kernel does)
+    const int base = __ldg(p.cache_seqlens + b);
+    for (int tn = split; tn < p.Snew; tn += p.num_splits) {
+      const long long dst = cache_elem(p, b, base + tn, g);
+      if (dst < 0) {
+        if (threadIdx.x == 0) report_status(p.status, kStatusBadArg);
+        continue;
+      }
+      if (!FA_IN_BOUNDS(dst + D <= p.ext_cache, p.status)) continue;
+      const size_t src = (((size_t)b * p.Snew + tn) * p.Hkv + g) * D;
+      for (int c = threadIdx.x; c < CH; c += 32 * kConsumers) {
+        *reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.k_cache) + dst + c * 8) =
+            *reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.k_new) + src + c * 8);
+        *reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.v_cache) + dst + c * 8) =
+            *reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.v_new) + src + c * 8);
+      }
+    }
+  }
 
   uint32_t qf[KSTEPS][4];
 #pragma unroll
@@ -187,11 +245,32 @@ __global__ void __launch_bounds__(kThreadsD, 1)
     if (flag[st]) {
       // rows past the split end may hold anything (even NaN): zero their V
       const int valid = t1 - tb;
+      bool patched = false;
       if (valid < kTokT) {
         for (int i = lane; i < (kTokT - valid) * CH; i += 32) {
           const int r = valid + i / CH, j = i % CH;
           *reinterpret_cast<uint4*>(kst + C::KT + tma_sw<kTokT>(r, j)) = make_uint4(0, 0, 0, 0);
         }
+        patched = true;
+      }
+      if (p.fuse_append) {
+        // this call's new rows (positions L - Snew .. L - 1) come from
+        // k_new / v_new: the cache write of another CTA may not have landed
+        const int n0 = max(tb, L - p.Snew), n1 = min(tb + kTokT, t1);
+        for (int i = lane; i < (n1 - n0) * CH; i += 32) {
+          const int r = n0 - tb + i / CH, j = i % CH;
+          const size_t src = (((size_t)b * p.Snew + (n0 + i / CH - (L - p.Snew))) * p.Hkv + g) * D + j * 8;
+          if (!FA_IN_BOUNDS(r >= 0 && r < kTokT && src + 8 <= (size_t)p.B * p.Snew * p.Hkv * D, p.status)) continue;
+          *reinterpret_cast<uint4*>(kst + tma_sw<kTokT>(r, j)) =
+              *reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.k_new) + src);
+          *reinterpret_cast<uint4*>(kst + C::KT + tma_sw<kTokT>(r, j)) =
+              *reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.v_new) + src);
+        }
+        patched = patched || n0 < n1;
+      }
+      if (patched) {
+        // the next TMA write into this stage must come after these stores
+        fence_proxy_async_smem();
         __syncwarp();
       }
       float s[NT_S][4];
@@ -338,7 +417,9 @@ __global__ void __launch_bounds__(kThreadsD, 1)
       for (int j = 0; j < 8; ++j) acc[j] += o[j] * fw[w];
     }
     if (p.num_splits == 1) {
-      T* out = reinterpret_cast<T*>(p.out) + (((size_t)b * p.Sq + sq) * p.Hq + h) * D + c0;
+      const long long oi = (((long long)b * p.Sq + sq) * p.Hq + h) * D + c0;
+      if (!FA_IN_BOUNDS(oi >= 0 && oi + 8 <= p.n_out, p.status)) continue;
+      T* out = reinterpret_cast<T*>(p.out) + oi;
       uint4 v;
       v.x = Elem<T>::pack(acc[0] * inv, acc[1] * inv);
       v.y = Elem<T>::pack(acc[2] * inv, acc[3] * inv);
@@ -348,12 +429,72 @@ __global__ void __launch_bounds__(kThreadsD, 1)
       if (p.lse && c0 == 0) p.lse[((size_t)b * p.Hq + h) * p.Sq + sq] = lse_nat;
     } else {
       const size_t row = (((size_t)split * p.B + b) * p.Hq + h) * p.Sq + sq;
+      if (!FA_IN_BOUNDS((long long)row < p.n_part, p.status)) continue;
       float* out = p.o_part + row * D + c0;
       *reinterpret_cast<float4*>(out) = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
       *reinterpret_cast<float4*>(out + 4) = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
       if (c0 == 0) p.lse_part[row] = lse_nat;
     }
   }
+  if (p.num_splits == 1 || !p.split_count) return;
+
+  // ---- the last split of (b, g, rt) to finish merges all splits' partials
+  volatile int* last = reinterpret_cast<volatile int*>(smem + C::OFF_LAST);
+  __threadfence();  // this split's partials are visible GPU-wide before it is counted
+  named_bar_sync(1, 32 * kConsumers);
+  if (threadIdx.x == 0) {
+    int* cnt = p.split_count + ((size_t)b * p.Hkv + g) * nrt + rt;
+    *last = atomicAdd(cnt, 1) == p.num_splits - 1;
+  }
+  named_bar_sync(1, 32 * kConsumers);
+  if (!*last) return;
+  __threadfence();
+  const size_t split_stride = (size_t)p.B * p.Hq * p.Sq;
+  for (int item = threadIdx.x; item < ITEMS; item += NT) {
+    const int r = item / (D / 8);
+    const int c0 = (item % (D / 8)) * 8;
+    const int pr = rt * 16 + r;
+    if (pr >= rows) continue;
+    const int sq = pr / p.G;
+    const int h = g * p.G + pr % p.G;
+    const size_t row0 = ((size_t)b * p.Hq + h) * p.Sq + sq;
+    if (!FA_IN_BOUNDS((long long)((p.num_splits - 1) * split_stride + row0) < p.n_part &&
+                          (long long)(row0 + 1) * D <= p.n_out,
+                      p.status))
+      continue;
+    float M = -INFINITY;
+    for (int sp = 0; sp < p.num_splits; ++sp) M = fmaxf(M, __ldcg(p.lse_part + sp * split_stride + row0));
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+    float W = 0.f;
+    if (M != -INFINITY) {
+      for (int sp = 0; sp < p.num_splits; ++sp) {
+        const size_t prow = sp * split_stride + row0;
+        const float w = fast_exp2((__ldcg(p.lse_part + prow) - M) * kLog2e);  // 0 for an empty split
+        if (w > 0.f) {
+          const float4 a = __ldcg(reinterpret_cast<const float4*>(p.o_part + prow * D + c0));
+          const float4 c = __ldcg(reinterpret_cast<const float4*>(p.o_part + prow * D + c0 + 4));
+          W += w;
+          acc[0] = fmaf(w, a.x, acc[0]); acc[1] = fmaf(w, a.y, acc[1]);
+          acc[2] = fmaf(w, a.z, acc[2]); acc[3] = fmaf(w, a.w, acc[3]);
+          acc[4] = fmaf(w, c.x, acc[4]); acc[5] = fmaf(w, c.y, acc[5]);
+          acc[6] = fmaf(w, c.z, acc[6]); acc[7] = fmaf(w, c.w, acc[7]);
+        }
+      }
+    }
+    const float inv = W > 0.f ? 1.f / W : 0.f;
+    T* out = reinterpret_cast<T*>(p.out) + (((size_t)b * p.Sq + sq) * p.Hq + h) * D + c0;
+    uint4 v;
+    v.x = Elem<T>::pack(acc[0] * inv, acc[1] * inv);
+    v.y = Elem<T>::pack(acc[2] * inv, acc[3] * inv);
+    v.z = Elem<T>::pack(acc[4] * inv, acc[5] * inv);
+    v.w = Elem<T>::pack(acc[6] * inv, acc[7] * inv);
+    *reinterpret_cast<uint4*>(out) = v;
+    if (p.lse && c0 == 0) p.lse[row0] = W > 0.f ? M + logf(W) : -INFINITY;
+  }
+  // the counter is zero again for the next call (the host also clears it)
+  if (threadIdx.x == 0) p.split_count[((size_t)b * p.Hkv + g) * nrt + rt] = 0;
 }
 
 template <typename T, int D, bool kCap>
@@ -372,19 +513,32 @@ cudaError_t launch_t(const DecodeParams& p, const CUtensorMap& mk, const CUtenso
 
 }  // namespace
 
-bool decode_tma_supported(const DecodeParams& p) {
-  return (p.D == 64 || p.D == 128) && (!p.paged || p.page_size % kTokT == 0) && tma_available();
+// Rows per TMA box: a whole 32-token tile, or 16 / 8 rows when pages hold a
+// multiple of 16 / 8 tokens but not of 32 (a box must stay inside one page);
+// 0 when neither fits (the cp.async kernel takes those pages).
+int decode_box_rows(const DecodeParams& p) {
+  if (!p.paged || p.page_size % kTokT == 0) return kTokT;
+  if (p.page_size % 16 == 0) return 16;
+  if (p.page_size % 8 == 0) return 8;
+  return 0;
 }
 
-cudaError_t launch_decode_split_tma(const DecodeParams& p, fa_dtype dt, cudaStream_t s) {
+bool decode_tma_supported(const DecodeParams& p) {
+  return (p.D == 64 || p.D == 128) && decode_box_rows(p) > 0 && tma_available();
+}
+
+cudaError_t launch_decode_split_tma(const DecodeParams& p_in, fa_dtype dt, cudaStream_t s) {
   CUtensorMap mk, mv;
+  DecodeParams p = p_in;
+  p.box_rows = decode_box_rows(p);
+  if (p.box_rows == 0) return cudaErrorNotSupported;
   const bool bf = dt == FA_BF16;
   // paged: (D, Hkv, page_size, num_pages); contiguous: (D, Hkv, max_seqlen, B)
   const int S = p.paged ? p.page_size : p.max_seqlen;
   const int N = p.paged ? p.capacity_pages : p.B;
   if (S <= 0 || N <= 0) return cudaErrorNotSupported;
-  if (!make_bshd_map(&mk, p.k_cache, bf, p.D, p.Hkv, S, N, kTokT) ||
-      !make_bshd_map(&mv, p.v_cache, bf, p.D, p.Hkv, S, N, kTokT))
+  if (!make_bshd_map(&mk, p.k_cache, bf, p.D, p.Hkv, S, N, p.box_rows) ||
+      !make_bshd_map(&mv, p.v_cache, bf, p.D, p.Hkv, S, N, p.box_rows))
     return cudaErrorNotSupported;
   const bool cap = p.softcap > 0.f;
   if (p.D == 64) {

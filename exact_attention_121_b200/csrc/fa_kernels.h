@@ -41,6 +41,9 @@ struct FwdParams {
   const float* descale_q;
   const float* descale_k;
   const float* descale_v;
+  // element extents (largest offset + 1) of out and of the LSE array; read
+  // only by the bounds-checked build
+  long long ext_o, n_stat;
 };
 
 struct BwdParams {
@@ -76,6 +79,10 @@ struct BwdParams {
   int rows_packed;       // dout, out and dq are packed (token, head) rows: plain indexing
   const float* alibi;    // ALiBi slopes as in FwdParams; null = off
   int alibi_bstride;
+  // element extents (largest offset + 1) of dout, out, dq, dk, dv, of the
+  // LSE / Delta arrays and of the dQ accumulator; read only by the
+  // bounds-checked build
+  long long ext_do, ext_o, ext_dq, ext_dk, ext_dv, n_stat, n_accum;
 };
 
 struct DecodeParams {
@@ -105,6 +112,18 @@ struct DecodeParams {
   const float* rot_sin;
   int rot_half, rot_len, rot_inter;
   void* q_rot;
+  // TMA split kernel only.  box_rows: cache rows per TMA box (32, or 16 / 8
+  // for pages smaller than or not a multiple of 32 tokens).  fuse_append: the
+  // split kernel writes k_new / v_new into the cache itself and takes the new
+  // rows from k_new / v_new (no separate append kernel).  split_count: one
+  // zeroed int32 per (b, kv-head, packed-row tile); the last split CTA of each
+  // combines the partials itself (no separate combine kernel); null = off.
+  int box_rows;
+  int fuse_append;
+  int* split_count;
+  // element counts of q / out (B*Sq*Hq*D), of the caches and of the split
+  // partial rows; read only by the bounds-checked build
+  long long n_out, ext_cache, n_part;
 };
 
 // Optional timing hooks around the dominant kernel of each call (events set
@@ -123,6 +142,9 @@ cudaError_t launch_bwd(const BwdParams& p, fa_dtype dt, cudaStream_t s, int* lau
 bool bwd_tc_supported(const BwdParams& p);
 cudaError_t launch_bwd_main_tc(const BwdParams& p, fa_dtype dt, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams& p, fa_dtype dt, cudaStream_t s, int* launches);
+// Split count the kvcache calls use when the caller passes num_splits <= 0.
+int kvcache_auto_splits(int B, int Sq, int Hq, int Hkv, int page_size, int paged, int max_pages_per_seq,
+                        int num_pages_or_max_seqlen);
 bool decode_tma_supported(const DecodeParams& p);
 cudaError_t launch_decode_split_tma(const DecodeParams& p, fa_dtype dt, cudaStream_t s);
 

@@ -59,7 +59,9 @@ typedef enum {
   FA_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment or Hq % Hkv != 0 */
   FA_ERR_UNSUPPORTED = 2, /* valid request the library does not implement (e.g. D=96) */
   FA_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
-  FA_ERR_TIMEOUT = 4      /* a bounded device wait ran out (device status word) */
+  FA_ERR_TIMEOUT = 4,     /* a bounded device wait ran out (device status word) */
+  FA_ERR_BOUNDS = 5       /* library built with FA_DEBUG_BOUNDS only: a kernel index fell
+                             outside its buffer; the access was skipped (device status word) */
 } fa_status;
 
 typedef enum { FA_FP16 = 0, FA_BF16 = 1 } fa_dtype;
@@ -243,9 +245,10 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, flo
 
 /*
  * Bytes of workspace fa_fwd_kvcache needs for `num_splits` KV splits: the
- * float32 partial outputs (splits, B, Hq, Sq, D) and partial LSEs
- * (splits, B, Hq, Sq).  num_splits <= 0 returns the size for FA_MAX_SPLITS.
- * Returns 0 when one split needs no workspace.
+ * float32 partial outputs (splits, B, Hq, Sq, D), the partial LSEs
+ * (splits, B, Hq, Sq) and B * Hq * Sq int32 split counters, each part
+ * rounded up to 256 bytes.  num_splits <= 0 returns the size for
+ * FA_MAX_SPLITS.  Returns 0 when one split needs no workspace.
  */
 size_t fa_kvcache_workspace_size(int B, int Sq, int Hq, int D, int num_splits);
 
@@ -271,7 +274,13 @@ size_t fa_kvcache_workspace_size(int B, int Sq, int Hq, int D, int num_splits);
  *   num_splits: KV range of each sequence split into this many page-aligned
  *     parts (<= 0: chosen from B, Hkv and the capacity); partials are merged
  *     by a log-sum-exp combine.  workspace >= fa_kvcache_workspace_size(B, Sq,
- *     Hq, D, num_splits) bytes, 256-byte aligned (may be NULL when that is 0).
+ *     Hq, D, num_splits) bytes, 256-byte aligned (may be NULL when that is 0);
+ *     its split counters are cleared by the call itself (an asynchronous
+ *     memset on `stream`), the rest needs no initial contents.
+ *   Kernels: with page_size a multiple of 8 tokens (or a contiguous cache)
+ *     and no rotary tables the whole call is one kernel: the split kernel
+ *     appends k_new / v_new itself and its last split per (b, kv-head) merges
+ *     the partials.  Other page sizes run append, split and combine kernels.
  */
 fa_status fa_fwd_kvcache(const void* q, void* k_cache, void* v_cache, const void* k_new,
                          const void* v_new, const int* cache_seqlens, const int* block_table,
@@ -324,21 +333,32 @@ fa_status fa_fwd_kvcache_rotary(const void* q, void* k_cache, void* v_cache, con
  * those callers only.
  *   Arguments: as fa_fwd_kvcache, minus workspace and ws_bytes.  The caller
  *   still owns and passes every input and output buffer.
- *   Scratch: the split-KV partials go to one file-scope device array of
- *   FA_STATIC_SCRATCH_BYTES (8 MiB) per GPU, part of the library's device
- *   image and held until the process exits.  That fits
- *   num_splits * B * Hq * Sq <= 16,256 partial rows at D=128 (32,263 at D=64);
- *   larger requests return FA_ERR_INVALID_ARG before anything is launched.
+ *   Scratch: the split-KV partials and split counters go to one file-scope
+ *   device array of FA_STATIC_SCRATCH_BYTES (8 MiB) per GPU, part of the
+ *   library's device image and held until the process exits.  A call fits
+ *   when fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits) <= 8 MiB: about
+ *   num_splits * B * Hq * Sq <= 16,200 partial rows at D=128 (32,200 at
+ *   D=64); larger requests return FA_ERR_INVALID_ARG before anything is
+ *   launched.
+ *   With num_splits <= 0 the call takes fa_fwd_kvcache's automatic split
+ *   count, lowered to the largest count whose partials fit the array.
  *   The call allocates nothing: no cudaMalloc, cudaFree or allocating library
  *   routine.
  *   Set-up: the first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current) and caches it; make that
- *   first call before any stream capture.
+ *   first call before any stream capture.  Under CUDA's lazy module loading
+ *   (the default) that lookup is also when the driver loads this part of the
+ *   library's device image, and with it the 8 MiB array: the device's free
+ *   memory drops once, at the set-up call, and never at a later call.  cudaDeviceReset unloads the
+ *   library's device image and with it the array: the cached address (and
+ *   that of the device status word) is then stale, so no call of this library
+ *   may follow a cudaDeviceReset in the same process.
  *   Sharing: every call on a device uses the same array, which keeps the last
- *   call's partials (nothing in it needs to start at zero: every partial row
- *   is written before it is read).  Calls whose executions overlap on the GPU
- *   (other streams, other host threads) race on the array and must be
- *   serialised by the caller.
+ *   call's partials.  What must start at zero (the split counters) is
+ *   cleared by each call before its kernel runs; every partial row is written
+ *   before it is read.  Calls whose executions overlap on the GPU (other
+ *   streams, other host threads) race on the array and must be serialised by
+ *   the caller.
  */
 fa_status fa_fwd_kvcache_noalloc(const void* q, void* k_cache, void* v_cache, const void* k_new,
                                  const void* v_new, const int* cache_seqlens, const int* block_table,
@@ -354,6 +374,18 @@ fa_status fa_fwd_kvcache_noalloc(const void* q, void* k_cache, void* v_cache, co
  * overflow).  Returns FA_ERR_CUDA if the synchronisation itself fails.
  */
 fa_status fa_last_device_status(fa_stream_t stream);
+
+/* Bit of fa_build_flags(): kernels compiled with -DFA_DEBUG_BOUNDS. */
+#define FA_BUILD_DEBUG_BOUNDS 1
+
+/*
+ * How this copy of the library was compiled: FA_BUILD_DEBUG_BOUNDS is set in
+ * the bounds-checked test build (libfa_debug.so), whose kernels check every
+ * buffer index they compute against the buffer's extent, record
+ * FA_ERR_BOUNDS in the device status word and skip the access on a miss; it
+ * is clear in the library proper (libfa.so).  No arguments, no errors.
+ */
+int fa_build_flags(void);
 
 /*
  * Which forward kernel fa_fwd runs: 0 = automatic, 1 = the warp-level

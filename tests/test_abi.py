@@ -76,6 +76,7 @@ def test_every_binding_matches_the_declared_parameter_types():
 def test_status_strings(lib):
     assert lib.fa_status_string(0) == b"FA_OK"
     assert lib.fa_status_string(4) == b"FA_ERR_TIMEOUT"
+    assert lib.fa_status_string(5) == b"FA_ERR_BOUNDS"
     assert lib.fa_status_string(99) == b"FA_ERR_UNKNOWN"
 
 
@@ -128,9 +129,12 @@ def test_bwd_workspace_is_linear_in_seqlen(lib, det):
 
 def test_kvcache_workspace(lib):
     assert lib.fa_kvcache_workspace_size(8, 1, 32, 128, 1) == 0
-    n4 = lib.fa_kvcache_workspace_size(8, 1, 32, 128, 4)
-    n16 = lib.fa_kvcache_workspace_size(8, 1, 32, 128, 16)
-    assert n4 >= 4 * 8 * 32 * 128 * 4 and n16 >= 4 * n4 - 1024
+    r256 = lambda x: (x + 255) // 256 * 256
+    rows = 8 * 1 * 32
+    for n in (2, 4, 16, 64):
+        # partial outputs, partial LSEs, one split counter per (b, q-head, query) at most
+        want = r256(n * rows * 128 * 4) + r256(n * rows * 4) + r256(rows * 4)
+        assert lib.fa_kvcache_workspace_size(8, 1, 32, 128, n) == want
     assert lib.fa_kvcache_workspace_size(8, 1, 32, 128, 0) == lib.fa_kvcache_workspace_size(8, 1, 32, 128, 64)
 
 
@@ -215,3 +219,7 @@ def test_kvcache_rotary_host_validation(lib):
     for splits in (1, 4, 0):
         assert lib.fa_kvcache_rotary_workspace_size(2, 1, 8, 128, splits) == \
             r256(2 * 1 * 8 * 128 * 2) + lib.fa_kvcache_workspace_size(2, 1, 8, 128, splits)
+
+
+def test_library_proper_is_not_the_bounds_checked_build(lib):
+    assert lib.fa_build_flags() == 0

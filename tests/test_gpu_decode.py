@@ -45,6 +45,9 @@ SMALL = [
     (3, 16, 4, 128, 64, 4, 200, 1, 1, "bf16", False, None),
     (2, 6, 2, 128, 8, 40, 300, 5, 5, "bf16", True, None),           # 15 packed rows per kv-head
     (1, 20, 1, 64, 16, 8, 100, 2, 1, "fp16", True, None),           # 40 packed rows: 3 row tiles
+    (2, 8, 2, 128, 48, 4, 180, 3, 3, "bf16", True, [46, 142]),      # 16-row boxes; new rows cross a page
+    (2, 8, 2, 64, 24, 6, 130, 2, 2, "fp16", True, [23, 100]),       # 8-row boxes; new rows cross a page
+    (2, 4, 2, 128, 12, 10, 100, 1, 1, "bf16", True, None),          # 12-token pages: cp.async kernel
 ]
 
 
@@ -62,6 +65,21 @@ def test_decode_small(case, splits):
     check_lse(lse, l_r)
     np.testing.assert_array_equal(f64(kc), kc_r)
     np.testing.assert_array_equal(f64(vc), vc_r)
+
+
+@pytest.mark.parametrize("page,launches", [(16, 1), (64, 1), (256, 1), (12, 3)])
+def test_decode_call_is_one_kernel(page, launches):
+    """With TMA-friendly pages the whole call (append, split-KV attention,
+    combine) is one kernel; other page sizes take append + split + combine."""
+    from exact_attention_121_b200 import _lib
+    d = inputs.kvcache_inputs(2, 8, 2, 128, page, 512 // page + 1, 500, Sq=1, Snew=1, dtype="bf16", seed=12)
+    out, lse, kc, vc, status = _run_case(d, 4)
+    assert status == 0
+    assert _lib.load().fa_last_launch_count() == launches
+    o_r, l_r, kc_r, vc_r = _oracle(d)
+    check_out(out, o_r, torch.bfloat16)
+    check_lse(lse, l_r)
+    np.testing.assert_array_equal(f64(kc), kc_r)
 
 
 @pytest.mark.parametrize("kw", [dict(window=(20, 0)), dict(softcap=3.0, scale=0.2), dict(causal=False)])
