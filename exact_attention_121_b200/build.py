@@ -3,6 +3,12 @@
 Usage: ``python -m exact_attention_121_b200.build`` (or call :func:`build`).
 Each .cu under csrc/ is compiled to an object in parallel, then linked into
 ``exact_attention_121_b200/libfa.so`` next to this file.
+
+``build(debug_bounds=True)`` (``--debug-bounds``) builds the bounds-checked
+variant instead, ``libfa_debug.so``: the same sources compiled with
+-DFA_DEBUG_BOUNDS, whose kernels check their buffer indices, record
+FA_ERR_BOUNDS in the device status word and skip an access that would fall
+outside its buffer.  It is a test build; the library proper is libfa.so.
 """
 
 import concurrent.futures as cf
@@ -17,6 +23,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libfa.so")
+BUILD_DEBUG = os.path.join(ROOT, "_build_debug")
+LIB_DEBUG = os.path.join(PKG, "libfa_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "--use_fast_math", "-Xcompiler", "-fPIC",
@@ -34,36 +42,38 @@ def _sources():
     return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cu"))
 
 
-def _compile(src, verbose=False):
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+def _compile(src, verbose=False, debug_bounds=False):
+    obj = os.path.join(BUILD_DEBUG if debug_bounds else BUILD, os.path.basename(src)[:-3] + ".o")
     deps = [src] + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))]
     deps.append(os.path.join(INCLUDE, "fa.h"))
     if os.path.exists(obj) and os.path.getmtime(obj) >= max(os.path.getmtime(d) for d in deps):
         return obj, ""
-    cmd = [nvcc()] + ARCH + FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-c", src, "-o", obj]
+    cmd = [nvcc()] + ARCH + FLAGS + (["-DFA_DEBUG_BOUNDS"] if debug_bounds else []) + \
+        (["-Xptxas", "-v"] if verbose else []) + ["-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")
     return obj, r.stderr
 
 
-def build(verbose=False, jobs=None):
-    os.makedirs(BUILD, exist_ok=True)
+def build(verbose=False, jobs=None, debug_bounds=False):
+    out_dir, lib = (BUILD_DEBUG, LIB_DEBUG) if debug_bounds else (BUILD, LIB)
+    os.makedirs(out_dir, exist_ok=True)
     srcs = _sources()
     with cf.ThreadPoolExecutor(max_workers=jobs or min(8, len(srcs))) as ex:
-        results = list(ex.map(lambda s: _compile(s, verbose), srcs))
+        results = list(ex.map(lambda s: _compile(s, verbose, debug_bounds), srcs))
     for obj, log in results:
         if log and (verbose or "spill" in log.lower() and "0 bytes spill" not in log):
             sys.stderr.write(log)
     objs = [o for o, _ in results]
     newest = max(os.path.getmtime(o) for o in objs)
-    if not os.path.exists(LIB) or os.path.getmtime(LIB) < newest:
-        cmd = [nvcc()] + ARCH + ["-shared", "-o", LIB] + objs + ["-lcudart"]
+    if not os.path.exists(lib) or os.path.getmtime(lib) < newest:
+        cmd = [nvcc()] + ARCH + ["-shared", "-o", lib] + objs + ["-lcudart"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(verbose="-v" in sys.argv))
+    print(build(verbose="-v" in sys.argv, debug_bounds="--debug-bounds" in sys.argv))

@@ -62,9 +62,10 @@ __global__ void bwd_preprocess_kernel(const BwdParams p, int n_sem) {
 #pragma unroll
     for (int u = 0; u < kPreSteps; ++u) {
       const long long r = base + u * kRowsPerStep + sub;
-      if (r < rows) {
-        const long long off_do = (kPacked ? r * D : row_offset(p, p.st_do, (unsigned)r)) + l * 8;
-        const long long off_o = (kPacked ? r * D : row_offset(p, p.st_o, (unsigned)r)) + l * 8;
+      const long long off_do = r < rows ? (kPacked ? r * D : row_offset(p, p.st_do, (unsigned)r)) + l * 8 : 0;
+      const long long off_o = r < rows ? (kPacked ? r * D : row_offset(p, p.st_o, (unsigned)r)) + l * 8 : 0;
+      if (r < rows && FA_IN_BOUNDS(off_do >= 0 && off_do + 8 <= p.ext_do && off_o >= 0 && off_o + 8 <= p.ext_o,
+                                   p.status)) {
         a[u] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.dout) + off_do));
         c[u] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.o) + off_o));
       } else {
@@ -84,20 +85,16 @@ __global__ void bwd_preprocess_kernel(const BwdParams p, int n_sem) {
       }
 #pragma unroll
       for (int o = kLanesPerRow / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (r < rows) {
+      if (r < rows && FA_IN_BOUNDS((r + 1) * D <= p.n_accum, p.status)) {
         float4* z = reinterpret_cast<float4*>(p.dq_accum + r * D + l * 8);
         z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
         z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (l == 0) {
           const int h = (int)(r % p.Hq);
           const long long tok = r / p.Hq;
-          if (p.cu_q) {
-            p.delta[(size_t)h * p.total_q + tok] = acc;  // (Hq, total_q)
-          } else {
-            const int i = (int)(tok % p.Sq);
-            const int b = (int)(tok / p.Sq);
-            p.delta[((size_t)b * p.Hq + h) * p.Sq + i] = acc;
-          }
+          const long long di = p.cu_q ? (long long)h * p.total_q + tok  // (Hq, total_q)
+                                      : ((long long)(tok / p.Sq) * p.Hq + h) * p.Sq + tok % p.Sq;
+          if (FA_IN_BOUNDS(di >= 0 && di < p.n_stat, p.status)) p.delta[di] = acc;
         }
       }
     }
@@ -407,6 +404,7 @@ __global__ void bwd_convert_kernel(const BwdParams p) {
     const long long n4 = (long long)rows * p.D / 4;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
          i += (long long)gridDim.x * blockDim.x) {
+      if (!FA_IN_BOUNDS(4 * i + 4 <= p.n_accum && 4 * i + 4 <= p.ext_dq, p.status)) continue;
       const float4 a = reinterpret_cast<const float4*>(p.dq_accum)[i];
       uint2 v;
       v.x = Elem<T>::pack(a.x * p.scale, a.y * p.scale);
@@ -418,11 +416,14 @@ __global__ void bwd_convert_kernel(const BwdParams p) {
   for (unsigned base = warp0 * rows_per_step; base < rows; base += nwarps * rows_per_step) {
     const unsigned r = base + sub;
     if (r >= rows) continue;
+    const long long dq_off = row_offset(p, p.st_dq, r) + l * 4;
+    if (!FA_IN_BOUNDS(((long long)r + 1) * p.D <= p.n_accum && dq_off >= 0 && dq_off + 4 <= p.ext_dq, p.status))
+      continue;
     const float4 a = reinterpret_cast<const float4*>(p.dq_accum + (size_t)r * p.D)[l];
     uint2 v;
     v.x = Elem<T>::pack(a.x * p.scale, a.y * p.scale);
     v.y = Elem<T>::pack(a.z * p.scale, a.w * p.scale);
-    *reinterpret_cast<uint2*>(dq + row_offset(p, p.st_dq, r) + l * 4) = v;
+    *reinterpret_cast<uint2*>(dq + dq_off) = v;
   }
 }
 

@@ -164,7 +164,11 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   if (p.wl >= 0) i_max = min(i_max, k1 - off + p.wl);
   const int qb_lo = i_min / kQ;
   const int n_qb = (k1 >= k0 && i_max >= i_min) ? (i_max / kQ - qb_lo + 1) : 0;
-  const int n_iter = n_qb * p.G;
+  // bounds-checked build: a CTA whose coordinates fall outside the tensors
+  // does no work (it has allocated TMEM already, so it still runs the
+  // common teardown)
+  const bool coords_ok = FA_IN_BOUNDS(hkv < p.Hkv && b < p.B && hkv * p.G + p.G <= p.Hq, p.status);
+  const int n_iter = coords_ok ? n_qb * p.G : 0;
   auto iter_q = [&](int it, int& h, int& q0) {
     h = hkv * p.G + it / n_qb;
     q0 = (qb_lo + it % n_qb) * kQ;
@@ -197,10 +201,12 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         float* r = rows + st * 2 * kQ;
         const float* L = p.lse + stat_base(p, seq, b, h);
         const float* Dl = p.delta + stat_base(p, seq, b, h);
+        const long long sbase = stat_base(p, seq, b, h);
         for (int t = lane; t < kQ; t += 32) {
           const int q = q0 + t;
           float l2 = INFINITY, dl = 0.f;
-          if (q < Sq) {  // rows past the sequence: P = 0, Delta = 0
+          // rows past the sequence: P = 0, Delta = 0
+          if (q < Sq && FA_IN_BOUNDS(sbase + q >= 0 && sbase + q < p.n_stat, p.status)) {
             const float l = L[q];
             l2 = (l == -INFINITY) ? INFINITY : l * kLog2e;  // stored negated below
             dl = Dl[q];
@@ -463,10 +469,15 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     } else {
       // ---- dV and dK rows of this warp's keys, head-dim half hh
       tc_fence_after();
-      T* dVr = reinterpret_cast<T*>(p.dv) + (long long)b * p.st_dv[0] + (long long)(seq.ktma + key) * p.st_dv[1] +
-               (long long)hkv * p.st_dv[2] + hh * (D / 2);
-      T* dKr = reinterpret_cast<T*>(p.dk) + (long long)b * p.st_dk[0] + (long long)(seq.ktma + key) * p.st_dk[1] +
-               (long long)hkv * p.st_dk[2] + hh * (D / 2);
+      const long long dv_off = (long long)b * p.st_dv[0] + (long long)(seq.ktma + key) * p.st_dv[1] +
+                               (long long)hkv * p.st_dv[2] + hh * (D / 2);
+      const long long dk_off = (long long)b * p.st_dk[0] + (long long)(seq.ktma + key) * p.st_dk[1] +
+                               (long long)hkv * p.st_dk[2] + hh * (D / 2);
+      T* dVr = reinterpret_cast<T*>(p.dv) + dv_off;
+      T* dKr = reinterpret_cast<T*>(p.dk) + dk_off;
+      const bool rows_ok = key_ok && FA_IN_BOUNDS(dv_off >= 0 && dv_off + D / 2 <= p.ext_dv && dk_off >= 0 &&
+                                                       dk_off + D / 2 <= p.ext_dk,
+                                                   p.status);
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const float mul = which ? p.scale : 1.f;
@@ -483,7 +494,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0u;
           }
-          if (key_ok) {
+          if (rows_ok) {
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
               uint4 o;
@@ -568,7 +579,10 @@ __global__ void __launch_bounds__(kThreadsB, 1)
             }
             fence_proxy_async_global();
           }
-          tma_reduce_add_4d(&tmDQ, 0, h, seq.qtma + q0, seq.tb, sb + C::OFF_DQ + i * C::DQ_TILE);
+          // a reduction may not start at a negative coordinate: skipped
+          // (and reported) by the bounds-checked build
+          if (FA_IN_BOUNDS(q0 >= 0 && h < p.Hq && seq.qtma + q0 >= 0, p.status))
+            tma_reduce_add_4d(&tmDQ, 0, h, seq.qtma + q0, seq.tb, sb + C::OFF_DQ + i * C::DQ_TILE);
           bulk_commit();
           if (sem) {
             // the additions are complete in global memory before the count moves

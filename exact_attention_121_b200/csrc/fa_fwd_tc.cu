@@ -91,6 +91,8 @@ struct TcCfg {
 };
 
 __device__ __forceinline__ float f32(uint32_t u) { return __uint_as_float(u); }
+// head dim 64 keeps P in its own TMEM columns beside O
+__host__ __device__ constexpr bool kSepPLayout(int D) { return D == 64; }
 
 // factor of (batch b, kv-head g) in a (B, Hkv) array; none given = 1
 __device__ __forceinline__ float descale_of(const float* d, int b, int g, int Hkv) {
@@ -105,6 +107,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = TcCfg<D, kFp8>;
   static_assert(!kFp8 || D == 128, "the 8-bit path is laid out for head dim 128");
+  // TMEM: S_A, S_B [0, 256), O_B ends at 384 + D (P at D = 64 inside O's 128 columns)
+  static_assert(384 + (kSepPLayout(D) ? 2 * D : D) <= 512, "tensor-memory columns");
+  static_assert(C::SMEM <= 227 * 1024, "shared memory per CTA");
   // Head dim 64 leaves TMEM room for P beside O (P_t at [256+128t+64, +64)),
   // so S_t can be refilled while P_t still feeds the PV product.
   constexpr bool kSepP = (D == 64);
@@ -129,6 +134,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   const SeqView seq = seq_view(p, b);
   const int Sq = seq.sq, Sk = seq.sk;
   if (q0 >= Sq) return;  // a shorter sequence of a packed batch: no rows here
+  // bounds-checked build: the CTA's head and batch coordinates (every
+  // thread takes the same branch, before any barrier)
+  if (!FA_IN_BOUNDS(h < p.Hq && g < p.Hkv && b < p.B, p.status)) return;
   const int off = Sk - Sq;
   const int qlast = min(q0 + 2 * kRows, Sq) - 1;
   int kmin = 0, kmax = Sk - 1;
@@ -198,6 +206,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         const int sk = j % C::NSK, uk = j / C::NSK;
         const int sv = j % C::NSV, uv = j / C::NSV;
         const int k0 = tile_k0(j);
+        (void)FA_IN_BOUNDS(k0 >= 0 && k0 < Sk, p.status);  // TMA fills outside the tensor; report only
         if (j >= C::NSK && !mbar_wait(bar(C::B_KE + sk), (uk - 1) & 1, abort_flag, kTcWaitNs)) {
           fail();
           break;
@@ -525,8 +534,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       // O / l (times the v factor of (b, g) for 8-bit inputs)
       const float ov = kFp8 ? descale_of(p.descale_v, b, g, p.Hkv) : 1.f;
       const float inv = l_q > 0.f ? ov / l_q : 0.f;
-      T* orow = reinterpret_cast<T*>(p.o) + (long long)b * p.st_o[0] + (long long)(seq.qtma + qi) * p.st_o[1] +
-                (long long)h * p.st_o[2];
+      const long long o_off =
+          (long long)b * p.st_o[0] + (long long)(seq.qtma + qi) * p.st_o[1] + (long long)h * p.st_o[2];
+      T* orow = reinterpret_cast<T*>(p.o) + o_off;
+      const bool row_ok = qi < Sq && FA_IN_BOUNDS(o_off >= 0 && o_off + D <= p.ext_o, p.status);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t u[32];
@@ -538,7 +549,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) u[i] = 0u;
         }
-        if (qi < Sq) {
+        if (row_ok) {
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4) {
             uint4 w;
@@ -550,8 +561,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           }
         }
       }
-      if (qi < Sq)
-        p.lse[stat_base(p, seq, b, h) + qi] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+      const long long li = stat_base(p, seq, b, h) + qi;
+      if (qi < Sq && FA_IN_BOUNDS(li >= 0 && li < p.n_stat, p.status))
+        p.lse[li] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
     }
   }
 
