@@ -115,7 +115,7 @@ def fa_fwd(q, k, v, out=None, lse=None, scale=None, causal=False, window=(-1, -1
 
 def fa_fwd_fp8(q, k, v, descale_q=None, descale_k=None, descale_v=None, out=None, lse=None, scale=None,
                causal=False, window=(-1, -1), softcap=0.0, stream=None):
-    """FP8 forward: q, k, v torch.float8_e4m3fn (B, S, H, D), head dim 128;
+    """FP8 forward: q, k, v torch.float8_e4m3fn (B, S, H, D), head dim 64 or 128;
     descales float32 (B, Hkv) or None.  Returns (out bf16, lse fp32)."""
     lib = _lib.load()
     B, Sq, Hq, D = q.shape

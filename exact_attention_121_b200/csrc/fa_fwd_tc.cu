@@ -62,8 +62,12 @@ constexpr unsigned long long kTcWaitNs = kWaitLimitNs;
 
 template <int D, bool kF8 = false>
 struct TcCfg {
-  static constexpr int CHUNK = kRows * 128;          // one 128-byte-wide, 128-row swizzled chunk (16 KB)
-  static constexpr int CHUNK_ELEMS = kF8 ? 128 : 64; // head-dim elements per chunk
+  // A row of a tile is one or two 128-byte swizzle atoms (16-bit elements),
+  // or D bytes of E4M3 codes: one 128-byte atom at head dim 128, one 64-byte
+  // atom at head dim 64.
+  static constexpr int ROWB = (kF8 && D == 64) ? 64 : 128;  // bytes per row of a chunk
+  static constexpr int CHUNK = kRows * ROWB;                // one swizzled 128-row chunk
+  static constexpr int CHUNK_ELEMS = kF8 ? D : 64;          // head-dim elements per chunk
   static constexpr int NCHUNK = D / CHUNK_ELEMS;
   static constexpr int TILE = CHUNK * NCHUNK;        // one 128-row tile
   static constexpr int NSK = (D == 128) ? 3 : 4;     // K stages
@@ -87,7 +91,11 @@ struct TcCfg {
   static constexpr int NBAR = B_DRAIN + 1;
   static constexpr int OFF_TMEM = OFF_BAR + 8 * NBAR;
   static constexpr int OFF_ABORT = OFF_TMEM + 4;
-  static constexpr int SMEM = OFF_ABORT + 4 + 1024;  // + alignment slack
+  // E4M3 at head dim 64: 16 KB of unused room after the barriers, so that
+  // operand reads cannot leave the CTA's shared memory whatever the rows'
+  // swizzle is taken to be
+  static constexpr int PAD = ROWB == 64 ? 16384 : 0;
+  static constexpr int SMEM = OFF_ABORT + 4 + PAD + 1024;  // + alignment slack
 };
 
 __device__ __forceinline__ float f32(uint32_t u) { return __uint_as_float(u); }
@@ -106,7 +114,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = TcCfg<D, kFp8>;
-  static_assert(!kFp8 || D == 128, "the 8-bit path is laid out for head dim 128");
+  // shared-memory operand descriptor of a chunk: 128-byte swizzle (8-row
+  // groups 1024 bytes apart), or 64-byte swizzle for E4M3 rows of head dim
+  // 64 (8-row groups 512 bytes apart)
+  constexpr bool kSw64 = C::ROWB == 64;
+  auto sdesc = [](uint32_t a, uint32_t lbo) -> uint64_t {
+    return kSw64 ? make_sdesc_sw64(a, lbo, 8 * 64) : make_sdesc_sw128(a, lbo, 8 * 128);
+  };
   // TMEM: S_A, S_B [0, 256), O_B ends at 384 + D (P at D = 64 inside O's 128 columns)
   static_assert(384 + (kSepPLayout(D) ? 2 * D : D) <= 512, "tensor-memory columns");
   static_assert(C::SMEM <= 227 * 1024, "shared memory per CTA");
@@ -144,6 +158,16 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   if (p.wr >= 0) kmax = min(kmax, qlast + off + p.wr);
   const int kt_begin = kmin / kRows;
   const int n_tiles = (kmax >= kmin) ? (kmax / kRows + 1 - kt_begin) : 0;
+  // Head dim 128: Q tile A (the CTA's first 128 rows) skips the trailing key
+  // tiles that a right bound (causal) masks for all of its rows; tile B
+  // takes them alone.  (Not with ALiBi, whose tile order is rotated; not at
+  // head dim 64, where the extra branches in the issue loop cost more than
+  // the skipped products save.)
+  int n_tiles_a = n_tiles;
+  if (p.wr >= 0 && !kAlibi && !kSepP) {
+    const int kmax_a = min(Sk - 1, min(q0 + kRows, Sq) - 1 + off + p.wr);
+    n_tiles_a = (kmax_a >= kmin) ? min(n_tiles, kmax_a / kRows + 1 - kt_begin) : 0;
+  }
   // Key-tile order.  Plain: ascending.  ALiBi: the tile at the diagonal of
   // the CTA's rows first, then the rest in ascending order from the far end,
   // so the running maximum is set at once and the (lower) bias of later
@@ -253,8 +277,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 #pragma unroll
         for (int kk = 0; kk < D / KS; ++kk) {
           const uint32_t koff = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          const uint64_t ad = make_sdesc_sw128(sb + C::OFF_Q + t * C::TILE + koff, 16, 1024);
-          const uint64_t bd = make_sdesc_sw128(sb + C::OFF_K + st * C::TILE + koff, 16, 1024);
+          const uint64_t ad = sdesc(sb + C::OFF_Q + t * C::TILE + koff, 16);
+          const uint64_t bd = sdesc(sb + C::OFF_K + st * C::TILE + koff, 16);
           if constexpr (kFp8)
             mma_ss_f8(tS[t], ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
           else
@@ -264,9 +288,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       auto issue_pv = [&](int t, int st, bool acc) {
 #pragma unroll
         for (int kk = 0; kk < kRows / KS; ++kk) {
-          // KS keys of V (MN-major: 128-byte rows of head-dim elements); P
-          // packs KS keys into 8 TMEM columns
-          const uint64_t bd = make_sdesc_sw128(sb + C::OFF_V + st * C::TILE + kk * KS * 128, C::CHUNK, 1024);
+          // KS keys of V (MN-major: rows of head-dim elements); P packs KS
+          // keys into 8 TMEM columns
+          const uint64_t bd = sdesc(sb + C::OFF_V + st * C::TILE + kk * KS * C::ROWB, C::CHUNK);
           if constexpr (kFp8)
             mma_ts_f8(tO[t], tP[t] + kk * 8, bd, idesc_pv, (acc || kk > 0) ? 1u : 0u);
           else
@@ -277,8 +301,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       ok = ok && mbar_wait(bar(C::B_KF + 0), 0, abort_flag, kTcWaitNs);
       if (ok) {
         tc_fence_after();
-        issue_qk(0, 0);
-        mma_commit(bar(C::B_S + 0));
+        if (n_tiles_a > 0) {
+          issue_qk(0, 0);
+          mma_commit(bar(C::B_S + 0));
+        }
         issue_qk(1, 0);
         mma_commit(bar(C::B_S + 1));
         mma_commit(bar(C::B_KE + 0));
@@ -324,18 +350,21 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         const int sv = j % C::NSV, uv = j / C::NSV;
         const int sk1 = (j + 1) % C::NSK, uk1 = (j + 1) / C::NSK;
         const bool more = j + 1 < n_tiles;
+        const bool a_now = j < n_tiles_a, a_more = j + 1 < n_tiles_a;
         ok = mbar_wait(bar(C::B_VF + sv), uv & 1, abort_flag, kTcWaitNs) &&
-             mbar_wait(bar(C::B_P + 0), j & 1, abort_flag, kTcWaitNs);
+             (!a_now || mbar_wait(bar(C::B_P + 0), j & 1, abort_flag, kTcWaitNs));
         if (!ok) break;
         tc_fence_after();
-        issue_pv(0, sv, j > 0);
+        if (a_now) issue_pv(0, sv, j > 0);
         if (more) {
           ok = mbar_wait(bar(C::B_KF + sk1), uk1 & 1, abort_flag, kTcWaitNs);
           if (!ok) break;
           tc_fence_after();
+        }
+        if (a_more) {
           issue_qk(0, sk1);
           mma_commit(bar(C::B_S + 0));
-        } else {
+        } else if (a_now) {
           mma_commit(bar(C::B_O + 0));
         }
         ok = mbar_wait(bar(C::B_P + 1), j & 1, abort_flag, kTcWaitNs);
@@ -376,7 +405,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     const float qk_f = kFp8 ? descale_of(p.descale_q, b, g, p.Hkv) * descale_of(p.descale_k, b, g, p.Hkv) : 1.f;
     const float scale_log2 = p.scale_log2 * qk_f, cap_in = p.cap_in * qk_f;
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
+    const int n_mine = t == 0 ? n_tiles_a : n_tiles;
+    for (int j = 0; j < n_mine; ++j) {
       // warp-uniform outcome: the TMEM accesses below are warp-collective
       if (!__all_sync(0xffffffffu, mbar_wait(bar(C::B_S + t), j & 1, abort_flag, kTcWaitNs))) {
         ok = false;
@@ -424,12 +454,16 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
       }
       if (!full) {
+        // Visible keys of this row in this tile as one range [lo, hi]
+        // relative to k0: two compares against constants per score.  (A
+        // per-key test of the three bounds made these tiles ~7x slower than
+        // unmasked ones: 15.5k against 2.1k cycles per tile.)
+        int lo = 0, hi = min(Sk - 1 - k0, kRows - 1);
+        if (p.wl >= 0) lo = max(lo, qpos - p.wl - k0);
+        if (p.wr >= 0) hi = min(hi, qpos + p.wr - k0);
 #pragma unroll
-        for (int i = 0; i < kRows; ++i) {
-          const int key = k0 + i;
-          const bool vis = key < Sk && (p.wl < 0 || key >= qpos - p.wl) && (p.wr < 0 || key <= qpos + p.wr);
-          if (!vis) s[i] = __float_as_uint(-INFINITY);
-        }
+        for (int i = 0; i < kRows; ++i)
+          if (i < lo || i > hi) s[i] = __float_as_uint(-INFINITY);
       }
       {
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -486,10 +520,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           }
           rq2 = f2_add(rq2, f2_pack(pr.x, pr.y));
         }
-        if constexpr (kFp8)
-          tmem_st8(tP + c * 8, *reinterpret_cast<uint32_t(*)[8]>(&pk[0]));
-        else if (!kSepP)
+        if constexpr (kFp8) {
+          if (!kSepP) tmem_st8(tP + c * 8, *reinterpret_cast<uint32_t(*)[8]>(&pk[0]));
+        } else if (!kSepP) {
           tmem_st16(tP + c * 16, pk);
+        }
       }
       if (kSepP) {
         // P_t and O_t are free once PV_t(j-1) has completed
@@ -499,7 +534,12 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_st16(tP + c * 16, pkall[c]);
+        for (int c = 0; c < 4; ++c) {
+          if constexpr (kFp8)
+            tmem_st8(tP + c * 8, *reinterpret_cast<uint32_t(*)[8]>(&pkall[c][0]));
+          else
+            tmem_st16(tP + c * 16, pkall[c]);
+        }
       }
       float rsa, rsb, rqa, rqb;
       f2_unpack(rs2, rsa, rsb);
@@ -525,7 +565,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       tc_fence_before();
       mbar_arrive(bar(C::B_P + t));
     }
-    if (ok && n_tiles > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_O + t), 0, abort_flag, kTcWaitNs));
+    if (ok && n_mine > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(C::B_O + t), 0, abort_flag, kTcWaitNs));
     if (!ok) {
       fail();
     } else {
@@ -541,7 +581,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t u[32];
-        if (n_tiles > 0) {
+        if (n_mine > 0) {
           tmem_ld32(tO + c * 32, u);
           tmem_wait_ld();
           reg_fence(u);
@@ -616,13 +656,19 @@ bool fwd_tc_supported(const FwdParams& p) {
 }
 
 cudaError_t launch_fwd_tc_fp8(const FwdParams& p, cudaStream_t s, int* launches) {
-  if (p.D != 128 || p.cu_q || p.alibi) return cudaErrorNotSupported;
+  if ((p.D != 128 && p.D != 64) || p.cu_q || p.alibi) return cudaErrorNotSupported;
   CUtensorMap mq, mk, mv;
   if (!make_bshd_map_u8(&mq, p.q, p.D, p.Hq, p.Sq, p.B, 128) || !make_bshd_map_u8(&mk, p.k, p.D, p.Hkv, p.Sk, p.B, 128) ||
       !make_bshd_map_u8(&mv, p.v, p.D, p.Hkv, p.Sk, p.B, 128))
     return cudaErrorNotSupported;
-  const cudaError_t e = p.softcap > 0.f ? launch_t<__nv_bfloat16, 128, true, false, true>(p, mq, mk, mv, s)
-                                        : launch_t<__nv_bfloat16, 128, false, false, true>(p, mq, mk, mv, s);
+  const bool cap = p.softcap > 0.f;
+  cudaError_t e;
+  if (p.D == 64)
+    e = cap ? launch_t<__nv_bfloat16, 64, true, false, true>(p, mq, mk, mv, s)
+            : launch_t<__nv_bfloat16, 64, false, false, true>(p, mq, mk, mv, s);
+  else
+    e = cap ? launch_t<__nv_bfloat16, 128, true, false, true>(p, mq, mk, mv, s)
+            : launch_t<__nv_bfloat16, 128, false, false, true>(p, mq, mk, mv, s);
   if (e == cudaSuccess) ++*launches;
   return e;
 }

@@ -21,8 +21,9 @@ bool make_bshd_map_strided(CUtensorMap* m, const void* base, bool bf16, int D, i
                            const long long st[3], int box_rows);
 
 // 4-D map (D, H, S, B) of packed 8-bit elements (E4M3 codes) with a box of
-// 128 head-dim elements (128 bytes) x 1 head x `box_rows` rows x 1 batch,
-// 128-byte swizzle, zero fill outside the tensor; D must be 128.
+// all D head-dim elements (D bytes) x 1 head x `box_rows` rows x 1 batch,
+// 128-byte swizzle (D = 128) or 64-byte swizzle (D = 64), zero fill outside
+// the tensor.
 bool make_bshd_map_u8(CUtensorMap* m, const void* base, int D, int H, int S, int B, int box_rows);
 
 // 4-D map (D, H, S, B) of fp32 elements with a box of all D elements x 1 head

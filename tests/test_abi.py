@@ -189,7 +189,7 @@ def test_fp8_host_validation(lib):
     p = ctypes.c_void_p(0x1000)
     fwd = lambda D=128, B=1, Sk=8, d=None: lib.fa_fwd_fp8(p, p, p, p, p, B, 8, Sk, 2, 2, D, d, None, None, 0.0, 0,
                                                           -1, -1, 0.0, None)
-    assert fwd(D=64) == _lib.FA_ERR_UNSUPPORTED                   # laid out for head dim 128
+    assert fwd(D=96) == _lib.FA_ERR_UNSUPPORTED                   # head dims 64 and 128 only
     assert fwd(d=ctypes.c_void_p(0x1002)) == _lib.FA_ERR_INVALID_ARG  # descale not 4-byte aligned
     assert fwd(B=0) == _lib.FA_OK                                 # nothing to do
     assert fwd(Sk=0) == _lib.FA_ERR_UNSUPPORTED

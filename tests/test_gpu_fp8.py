@@ -64,13 +64,17 @@ def check_rms_ratio(ratios):
     assert r <= RMS_RATIO_MAX, f"RMS of error / sigma {r:.2f}"
     return r
 
-# (B, Sq, Sk, Hq, Hkv, causal, window, softcap, with descales)
+# (B, Sq, Sk, Hq, Hkv, D, causal, window, softcap, with descales)
 CASES = [
-    (2, 300, 300, 4, 2, True, (-1, -1), 0.0, True),
-    (1, 200, 513, 4, 4, False, (-1, -1), 0.0, False),
-    (2, 129, 129, 8, 1, True, (40, 0), 0.0, True),
-    (1, 257, 257, 2, 2, False, (-1, -1), 20.0, True),
-    (1, 1024, 1024, 4, 2, False, (64, 64), 0.0, True),
+    (2, 300, 300, 4, 2, 128, True, (-1, -1), 0.0, True),
+    (1, 200, 513, 4, 4, 128, False, (-1, -1), 0.0, False),
+    (2, 129, 129, 8, 1, 128, True, (40, 0), 0.0, True),
+    (1, 257, 257, 2, 2, 128, False, (-1, -1), 20.0, True),
+    (1, 1024, 1024, 4, 2, 128, False, (64, 64), 0.0, True),
+    (2, 300, 300, 4, 2, 64, True, (-1, -1), 0.0, True),
+    (1, 200, 513, 4, 4, 64, False, (-1, -1), 0.0, False),
+    (1, 257, 257, 2, 2, 64, False, (-1, -1), 20.0, True),
+    (1, 700, 700, 4, 1, 64, True, (100, 0), 0.0, True),
 ]
 
 
@@ -78,11 +82,11 @@ def _codes(t):
     return t.view(torch.uint8).numpy()
 
 
-@pytest.mark.parametrize("case", CASES, ids=lambda c: "B%dS%dx%dH%d-%d%s%s" % (
-    c[0], c[1], c[2], c[3], c[4], "c" if c[5] else "", "w" if c[6] != (-1, -1) else ""))
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "B%dS%dx%dH%d-%dD%d%s%s" % (
+    c[0], c[1], c[2], c[3], c[4], c[5], "c" if c[6] else "", "w" if c[7] != (-1, -1) else ""))
 def test_fp8_forward_vs_oracle(case):
-    B, Sq, Sk, Hq, Hkv, causal, window, cap, desc = case
-    q, k, v, dq, dk, dv = inputs.fp8_inputs(B, Sq, Sk, Hq, Hkv, 128, seed=70)
+    B, Sq, Sk, Hq, Hkv, D, causal, window, cap, desc = case
+    q, k, v, dq, dk, dv = inputs.fp8_inputs(B, Sq, Sk, Hq, Hkv, D, seed=70)
     if not desc:
         dq = dk = dv = None
     dev = lambda t: None if t is None else t.cuda()
@@ -104,11 +108,12 @@ def test_fp8_forward_vs_oracle(case):
     check_rms_ratio(ratios)
 
 
-def test_fp8_exact_powers_of_two_match_to_bf16():
+@pytest.mark.parametrize("D", [128, 64])
+def test_fp8_exact_powers_of_two_match_to_bf16(D):
     # q one-hot in dim 0, k[:, :, :, 0] integers in [-4, 4]: raw scores are
     # those integers; scale ln 2 and dq * dk = 1 make P = 2^(score - max),
     # exact in E4M3, so O differs from the oracle by bf16 rounding only
-    B, S, H, D = 2, 384, 4, 128
+    B, S, H = 2, 384, 4
     g = torch.Generator().manual_seed(71)
     q = torch.zeros((B, S, H, D))
     q[..., 0] = 1.0
@@ -155,6 +160,6 @@ def test_fp8_refusals():
             api.fa_fwd_fp8(q.cuda(), k.cuda(), v.cuda())
         finally:
             api.fa_set_fwd_kernel(0)
-    q64, k64, v64, *_ = inputs.fp8_inputs(1, 16, 16, 2, 2, 64, seed=72)
-    with pytest.raises(_lib.FaError):  # head dim 64 is not laid out for 8 bits
-        api.fa_fwd_fp8(q64.cuda(), k64.cuda(), v64.cuda())
+    q96, k96, v96, *_ = inputs.fp8_inputs(1, 16, 16, 2, 2, 96, seed=72)
+    with pytest.raises(_lib.FaError):  # head dims other than 64 and 128
+        api.fa_fwd_fp8(q96.cuda(), k96.cuda(), v96.cuda())
