@@ -231,7 +231,7 @@ fa_status fa_bwd_alibi(const void* dout, const void* q, const void* k, const voi
  * Internally P is quantised to E4M3 for the P.V product and O is divided by
  * the sum of the quantised P, so each output row is a convex combination of
  * V rows whose weights are off by at most the E4M3 rounding of P.  Head dim
- * 128 and Sk >= 1 only (FA_ERR_UNSUPPORTED otherwise); misaligned pointers
+ * 64 or 128 and Sk >= 1 (FA_ERR_UNSUPPORTED otherwise); misaligned pointers
  * give FA_ERR_INVALID_ARG.  tcgen05 kernel only.
  */
 fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, float* lse,

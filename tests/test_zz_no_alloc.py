@@ -4,9 +4,16 @@ memory, a serving loop with a fixed footprint): its split-KV partials live in
 a fixed device array inside libfa.so instead of a caller workspace.
 
 Checked through the C ABI against fa_fwd_kvcache (the workspace entry point)
-on two calls in a row with different inputs and split counts, since the array
-keeps the previous call's contents.  Collected last so that a stop-at-first-
-failure run has already run every other test; it also passes alone.
+on calls in a row with different inputs and split counts (explicit, one, and
+the automatic choice), since the array keeps the previous call's contents.
+"Allocates nothing" is checked twice: PyTorch's allocator counter and the
+driver's free-memory figure (cudaMemGetInfo) are unchanged across a call.
+The first call on the device is the set-up call: it looks up the array's
+address, and with CUDA's lazy module loading (the default) that is when the
+driver loads this part of the library's device image, array included; the
+memory figures are compared on the calls after it.
+Collected last so that a stop-at-first-failure run has already run every
+other test; it also passes alone.
 """
 
 import ctypes
@@ -48,7 +55,11 @@ def _reference(d, num_splits):
 
 def test_noalloc_matches_workspace_entry_point_on_two_calls():
     lib = _lib.load()
-    for seed, splits in ((31, 4), (32, 7)):
+    # set-up call (array address lookup, device image of the entry point)
+    d0 = _device_case(30)
+    assert _noalloc(lib, d0, 4, torch.empty_like(d0["q"]), torch.empty(4, 32, 1, device="cuda")) == _lib.FA_OK
+    torch.cuda.synchronize()
+    for seed, splits in ((31, 4), (32, 7), (34, 0), (35, 1)):
         d = _device_case(seed)
         ref_out, ref_lse = _reference(d, splits)
         out = torch.empty_like(d["q"])
@@ -60,14 +71,17 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
         gc.disable()
         try:
             before = torch.cuda.memory_allocated()
+            free_before = torch.cuda.mem_get_info()[0]
             code = _noalloc(lib, d, splits, out, lse)
             torch.cuda.synchronize()
+            free_after = torch.cuda.mem_get_info()[0]
             after = torch.cuda.memory_allocated()
         finally:
             gc.enable()
         assert code == _lib.FA_OK, api.fa_status_string(code)
         assert api.fa_last_device_status() == 0
         assert after == before
+        assert free_after == free_before, (free_before, free_after)
         check_out(out, f64(ref_out), torch.bfloat16)
         check_lse(lse, f64(ref_lse))
 
@@ -88,3 +102,20 @@ def test_noalloc_refuses_requests_beyond_the_array():
     assert _noalloc(lib, big, 64, out2, lse2) == _lib.FA_ERR_INVALID_ARG
     torch.cuda.synchronize()
     assert api.fa_last_device_status() == 0
+
+
+def test_noalloc_automatic_splits_fit_the_array():
+    """A shape whose automatic split count would need more partial rows than
+    the array holds (16 sequences x 32 heads x 16 queries) runs with the
+    largest count that fits instead of being refused."""
+    lib = _lib.load()
+    d = inputs.kvcache_inputs(16, 32, 8, 128, 64, 4, 200, Sq=16, Snew=16, dtype="bf16", seed=36)
+    d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+    ref_out, ref_lse = _reference(d, 0)
+    out = torch.empty_like(d["q"])
+    lse = torch.empty_like(ref_lse)
+    assert _noalloc(lib, d, 0, out, lse) == _lib.FA_OK
+    torch.cuda.synchronize()
+    assert api.fa_last_device_status() == 0
+    check_out(out, f64(ref_out), torch.bfloat16)
+    check_lse(lse, f64(ref_lse))
