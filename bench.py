@@ -8,10 +8,16 @@ A step is one pass of the whole hot path over one batch of synthetic inputs:
     window (1024,0), softcap 30): forward + backward, once with atomic and
     once with deterministic (ordered) dQ accumulation;
   * the paged KV-cache decode (B=8, Hq=32, Hkv=8, D=128, lengths U[1,32768],
-    page 256): append + split-KV attention + combine.
+    page 256): append + split-KV attention + combine, with the automatic
+    split count and with 1, 4 and 16 splits.
 ``value`` is algorithmic attention TFLOP/s of the whole step (4*D flops per
 visible (query, key) pair forward, 10*D backward; decode flops counted the
-same way) with inputs resident in HBM.  Every tensor of a sweep point, the GQA
+same way) with inputs resident in HBM.  ``per_config`` gives, from CUDA
+events around every API call of the timed steps, each point's forward and
+forward+backward TFLOP/s as fractions of the measured bf16 tensor rates and
+each decode call's GB/s as a fraction of the measured HBM copy rate;
+``per_config_summary`` the worst head-dim-128 point at S >= 4096 and the
+worst decode call.  Every tensor of a sweep point, the GQA
 workload and the KV cache is larger than L2 (126 MB per step working set far
 exceeds it), so L2 is not flushed.  Multi-GPU: every rank runs its own replica
 of the step (the work units are independent), value sums all ranks' flops

@@ -282,7 +282,6 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, flo
   if (Sk < 0) return FA_ERR_INVALID_ARG;
   for (const float* d : {descale_q, descale_k, descale_v})
     if (reinterpret_cast<uintptr_t>(d) & 3u) return FA_ERR_INVALID_ARG;
-  if (D != 128) return FA_ERR_UNSUPPORTED;
   if (B == 0 || Sq == 0) return FA_OK;
   if (Sk == 0) return FA_ERR_UNSUPPORTED;
   if (!q || !k || !v || !out || !lse) return FA_ERR_INVALID_ARG;
@@ -575,10 +574,7 @@ size_t fa_kvcache_workspace_size(int B, int Sq, int Hq, int D, int num_splits) {
   if (num_splits <= 0 || num_splits > FA_MAX_SPLITS) num_splits = FA_MAX_SPLITS;
   if (num_splits == 1) return 0;
   const size_t rows = (size_t)num_splits * B * Hq * Sq;
-  // partial outputs, partial LSEs, and one split counter per (b, kv-head,
-  // packed-row tile), at most B * Hq * Sq of them
-  return round256(rows * D * sizeof(float)) + round256(rows * sizeof(float)) +
-         round256((size_t)B * Hq * Sq * sizeof(int));
+  return round256(rows * D * sizeof(float)) + round256(rows * sizeof(float));
 }
 
 struct RotaryArgs {
@@ -651,8 +647,6 @@ static fa_status kvcache_impl(const void* q, void* k_cache, void* v_cache, const
     p.o_part = reinterpret_cast<float*>(ws);
     ws += round256(rows * D * sizeof(float));
     p.lse_part = reinterpret_cast<float*>(ws);
-    ws += round256(rows * sizeof(float));
-    p.split_count = reinterpret_cast<int*>(ws);
     p.n_part = (long long)rows;
   }
   p.status = status_ptr();

@@ -437,6 +437,9 @@ __global__ void __launch_bounds__(kCombineWarps * 32) decode_combine_kernel(cons
   using Vec = typename std::conditional<PER_LANE == 4, float4, float2>::type;
   __shared__ float s_acc[kCombineWarps][D];
   __shared__ float s_w[kCombineWarps], s_m[kCombineWarps];
+  // launched as a programmatic dependent of the split kernel: wait until
+  // that grid has completed and its partials are visible
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const long long row = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t split_stride = (size_t)p.B * p.Hq * p.Sq;
@@ -527,16 +530,27 @@ cudaError_t launch_append(const DecodeParams& p, cudaStream_t s, int* launches) 
   return e;
 }
 
+// The combine pass as a programmatic dependent launch: its blocks may be
+// scheduled while the split kernel's last CTAs still run (the TMA split
+// kernel signals this at its start) and wait in griddepcontrol.wait until
+// that grid has completed and its partials are visible.
 template <typename T>
 cudaError_t launch_combine(const DecodeParams& p, cudaStream_t s, int* launches) {
   const long long rows = (long long)p.B * p.Hq * p.Sq;
   if (rows > 0x7fffffffLL) return cudaErrorInvalidValue;  // one block per row
   static_assert(FA_MAX_SPLITS <= kCombineWarps * 32, "one thread per split for the LSE maximum");
-  if (p.D == 64)
-    decode_combine_kernel<T, 64><<<(unsigned)rows, kCombineWarps * 32, 0, s>>>(p);
-  else
-    decode_combine_kernel<T, 128><<<(unsigned)rows, kCombineWarps * 32, 0, s>>>(p);
-  const cudaError_t e = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)rows);
+  cfg.blockDim = dim3(kCombineWarps * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = p.D == 64 ? cudaLaunchKernelEx(&cfg, decode_combine_kernel<T, 64>, p)
+                                  : cudaLaunchKernelEx(&cfg, decode_combine_kernel<T, 128>, p);
   if (e == cudaSuccess) ++*launches;
   return e;
 }
@@ -559,9 +573,9 @@ cudaError_t launch_decode_t(const DecodeParams& p_in, cudaStream_t s, int* launc
   }
   bool appended = false;
   if (decode_tma_supported(p)) {
-    // One kernel for the whole call: the TMA split kernel appends the new
-    // rows itself (not with rotary tables: those rows are rotated by the
-    // append kernel first) and merges its splits through the zeroed counters.
+    // The TMA split kernel appends the new rows itself (not with rotary
+    // tables: those rows are rotated by the append kernel first); the
+    // combine follows as its programmatic dependent.
     if (p.Snew > 0 && p.rot_cos) {
       e = launch_append<T>(p, s, launches);
       if (e != cudaSuccess) return e;
@@ -569,15 +583,10 @@ cudaError_t launch_decode_t(const DecodeParams& p_in, cudaStream_t s, int* launc
     }
     DecodeParams pf = p;
     pf.fuse_append = p.Snew > 0 && !p.rot_cos;
-    if (p.num_splits > 1 && pf.split_count) {
-      const int nrt = (p.Sq * p.G + 15) / 16;
-      e = cudaMemsetAsync(pf.split_count, 0, (size_t)p.B * p.Hkv * nrt * sizeof(int), s);
-      if (e != cudaSuccess) return e;
-    }
     e = launch_decode_split_tma(pf, Elem<T>::kBf16 ? FA_BF16 : FA_FP16, s);
     if (e == cudaSuccess) {
       ++*launches;
-      return (p.num_splits > 1 && !pf.split_count) ? launch_combine<T>(p, s, launches) : cudaSuccess;
+      return p.num_splits > 1 ? launch_combine<T>(p, s, launches) : cudaSuccess;
     }
     if (e != cudaErrorNotSupported) return e;
   }

@@ -12,16 +12,15 @@
 // packed into the 16 rows of an mma.sync tile, so each K/V byte is read from
 // HBM once for the whole group.
 //
-// The whole call can run as this one kernel:
+// The append and the launch gap of the combine are folded in:
 //   * append (fuse_append): the CTAs of the first row tile write the new
 //     rows k_new / v_new into the cache, spread over the splits, and every
 //     CTA whose tile covers a new row takes that row from k_new / v_new in
 //     shared memory, so no CTA depends on another's cache write;
-//   * combine (split_count): each split writes its partial output and LSE to
-//     the workspace, then counts itself done on its (b, kv-head, row tile)
-//     counter; the CTA that finishes last merges the splits
-//     (LSE = ln sum_s e^{LSE_s}, O = sum_s e^{LSE_s - LSE} O_s) and clears
-//     the counter.
+//   * combine: the partials go to the workspace; the combine kernel that
+//     merges them is launched as a programmatic dependent of this kernel
+//     (each CTA signals it at its start), so it is scheduled during this
+//     kernel's tail and only waits for the grid to complete.
 #include <math.h>
 
 #include "fa_common.cuh"
@@ -51,8 +50,7 @@ struct DecCfg {
   static constexpr int OFF_ST = 16 * D * 2 > 1024 ? 16 * D * 2 : 1024;
   static constexpr int OFF_BAR = OFF_ST + kStages * STAGE;
   static constexpr int OFF_FLAG = OFF_BAR + 2 * kStages * 8;
-  static constexpr int OFF_LAST = OFF_FLAG + kStages * 4;
-  static constexpr int SMEM = OFF_LAST + 4 + 1024;
+  static constexpr int SMEM = OFF_FLAG + kStages * 4 + 1024;
 };
 
 // Byte offset of logical 16-byte chunk j of row r inside a TMA-swizzled tile
@@ -97,6 +95,9 @@ __global__ void __launch_bounds__(kThreadsD, 1)
   auto empty = [&](int st) -> uint32_t { return sb + C::OFF_BAR + 8 * (kStages + st); };
   volatile int* flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAG);
 
+  // the combine kernel (a programmatic dependent launch) may be scheduled
+  // once every CTA of this grid has started; it waits for the grid to finish
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x;
   const int nrt = (p.Sq * p.G + 15) / 16;
@@ -139,22 +140,47 @@ __global__ void __launch_bounds__(kThreadsD, 1)
           break;
         }
         const int t = t0 + tt * kTokT;
-        // boxes of R rows; each lies inside one page (R divides the page
-        // size and t0 starts a page); boxes past the split end are not loaded
+        const uint32_t kst = sb + C::OFF_ST + st * C::STAGE;
+        if (p.box_rows == kTokT) {
+          // one box per tile: the tile lies inside one page
+          int c2 = t, c3 = b;
+          bool ok = true;
+          if (p.paged) {
+            const int page = __ldg(p.block_table + (size_t)b * p.max_pages_per_seq + t / p.page_size);
+            ok = page >= 0 && page < p.capacity_pages;
+            c2 = t % p.page_size;
+            c3 = page;
+          }
+          flag[st] = ok ? 1 : 0;
+          if (!ok) {
+            report_status(p.status, kStatusBadArg);
+            mbar_arrive(full(st));
+            continue;
+          }
+          mbar_expect_tx(full(st), C::STAGE);
+          for (int c = 0; c < C::NCH; ++c) {
+            tma_load_4d(kst + c * C::CHUNK, &tmK, c * 64, g, c2, c3, full(st));
+            tma_load_4d(kst + C::KT + c * C::CHUNK, &tmV, c * 64, g, c2, c3, full(st));
+          }
+          continue;
+        }
+        // boxes of R = 16 or 8 rows; each lies inside one page (R divides the
+        // page size and t0 starts a page); boxes past the split end are not
+        // loaded
         const int R = p.box_rows;
         const int nbox = min(kTokT / R, (t1 - t + R - 1) / R);
-        int c2[kTokT / 8], c3[kTokT / 8];
+        int c2[kTokT / 8], c3[kTokT / 8];  // unrolled: registers
         bool ok = true;
-        for (int x = 0; x < nbox; ++x) {
+#pragma unroll
+        for (int x = 0; x < kTokT / 8; ++x) {
           const int tx = t + x * R;
-          if (p.paged) {
+          c2[x] = tx;
+          c3[x] = b;
+          if (x < nbox && p.paged) {
             const int page = __ldg(p.block_table + (size_t)b * p.max_pages_per_seq + tx / p.page_size);
             ok = ok && page >= 0 && page < p.capacity_pages;
             c2[x] = tx % p.page_size;
             c3[x] = page;
-          } else {
-            c2[x] = tx;
-            c3[x] = b;
           }
         }
         flag[st] = ok ? 1 : 0;
@@ -163,13 +189,15 @@ __global__ void __launch_bounds__(kThreadsD, 1)
           mbar_arrive(full(st));
           continue;
         }
-        const uint32_t kst = sb + C::OFF_ST + st * C::STAGE;
         mbar_expect_tx(full(st), (uint32_t)(nbox * R * 128 * C::NCH * 2));
-        for (int x = 0; x < nbox; ++x)
-          for (int c = 0; c < C::NCH; ++c) {
-            tma_load_4d(kst + c * C::CHUNK + x * R * 128, &tmK, c * 64, g, c2[x], c3[x], full(st));
-            tma_load_4d(kst + C::KT + c * C::CHUNK + x * R * 128, &tmV, c * 64, g, c2[x], c3[x], full(st));
-          }
+#pragma unroll
+        for (int x = 0; x < kTokT / 8; ++x)
+          if (x < nbox)
+#pragma unroll
+            for (int c = 0; c < C::NCH; ++c) {
+              tma_load_4d(kst + c * C::CHUNK + x * R * 128, &tmK, c * 64, g, c2[x], c3[x], full(st));
+              tma_load_4d(kst + C::KT + c * C::CHUNK + x * R * 128, &tmV, c * 64, g, c2[x], c3[x], full(st));
+            }
       }
     }
     return;  // the consumers never wait on this warp again
@@ -436,65 +464,6 @@ __global__ void __launch_bounds__(kThreadsD, 1)
       if (c0 == 0) p.lse_part[row] = lse_nat;
     }
   }
-  if (p.num_splits == 1 || !p.split_count) return;
-
-  // ---- the last split of (b, g, rt) to finish merges all splits' partials
-  volatile int* last = reinterpret_cast<volatile int*>(smem + C::OFF_LAST);
-  __threadfence();  // this split's partials are visible GPU-wide before it is counted
-  named_bar_sync(1, 32 * kConsumers);
-  if (threadIdx.x == 0) {
-    int* cnt = p.split_count + ((size_t)b * p.Hkv + g) * nrt + rt;
-    *last = atomicAdd(cnt, 1) == p.num_splits - 1;
-  }
-  named_bar_sync(1, 32 * kConsumers);
-  if (!*last) return;
-  __threadfence();
-  const size_t split_stride = (size_t)p.B * p.Hq * p.Sq;
-  for (int item = threadIdx.x; item < ITEMS; item += NT) {
-    const int r = item / (D / 8);
-    const int c0 = (item % (D / 8)) * 8;
-    const int pr = rt * 16 + r;
-    if (pr >= rows) continue;
-    const int sq = pr / p.G;
-    const int h = g * p.G + pr % p.G;
-    const size_t row0 = ((size_t)b * p.Hq + h) * p.Sq + sq;
-    if (!FA_IN_BOUNDS((long long)((p.num_splits - 1) * split_stride + row0) < p.n_part &&
-                          (long long)(row0 + 1) * D <= p.n_out,
-                      p.status))
-      continue;
-    float M = -INFINITY;
-    for (int sp = 0; sp < p.num_splits; ++sp) M = fmaxf(M, __ldcg(p.lse_part + sp * split_stride + row0));
-    float acc[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-    float W = 0.f;
-    if (M != -INFINITY) {
-      for (int sp = 0; sp < p.num_splits; ++sp) {
-        const size_t prow = sp * split_stride + row0;
-        const float w = fast_exp2((__ldcg(p.lse_part + prow) - M) * kLog2e);  // 0 for an empty split
-        if (w > 0.f) {
-          const float4 a = __ldcg(reinterpret_cast<const float4*>(p.o_part + prow * D + c0));
-          const float4 c = __ldcg(reinterpret_cast<const float4*>(p.o_part + prow * D + c0 + 4));
-          W += w;
-          acc[0] = fmaf(w, a.x, acc[0]); acc[1] = fmaf(w, a.y, acc[1]);
-          acc[2] = fmaf(w, a.z, acc[2]); acc[3] = fmaf(w, a.w, acc[3]);
-          acc[4] = fmaf(w, c.x, acc[4]); acc[5] = fmaf(w, c.y, acc[5]);
-          acc[6] = fmaf(w, c.z, acc[6]); acc[7] = fmaf(w, c.w, acc[7]);
-        }
-      }
-    }
-    const float inv = W > 0.f ? 1.f / W : 0.f;
-    T* out = reinterpret_cast<T*>(p.out) + (((size_t)b * p.Sq + sq) * p.Hq + h) * D + c0;
-    uint4 v;
-    v.x = Elem<T>::pack(acc[0] * inv, acc[1] * inv);
-    v.y = Elem<T>::pack(acc[2] * inv, acc[3] * inv);
-    v.z = Elem<T>::pack(acc[4] * inv, acc[5] * inv);
-    v.w = Elem<T>::pack(acc[6] * inv, acc[7] * inv);
-    *reinterpret_cast<uint4*>(out) = v;
-    if (p.lse && c0 == 0) p.lse[row0] = W > 0.f ? M + logf(W) : -INFINITY;
-  }
-  // the counter is zero again for the next call (the host also clears it)
-  if (threadIdx.x == 0) p.split_count[((size_t)b * p.Hkv + g) * nrt + rt] = 0;
 }
 
 template <typename T, int D, bool kCap>

@@ -115,12 +115,9 @@ struct DecodeParams {
   // TMA split kernel only.  box_rows: cache rows per TMA box (32, or 16 / 8
   // for pages smaller than or not a multiple of 32 tokens).  fuse_append: the
   // split kernel writes k_new / v_new into the cache itself and takes the new
-  // rows from k_new / v_new (no separate append kernel).  split_count: one
-  // zeroed int32 per (b, kv-head, packed-row tile); the last split CTA of each
-  // combines the partials itself (no separate combine kernel); null = off.
+  // rows from k_new / v_new (no separate append kernel).
   int box_rows;
   int fuse_append;
-  int* split_count;
   // element counts of q / out (B*Sq*Hq*D), of the caches and of the split
   // partial rows; read only by the bounds-checked build
   long long n_out, ext_cache, n_part;

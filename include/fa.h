@@ -245,10 +245,10 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, flo
 
 /*
  * Bytes of workspace fa_fwd_kvcache needs for `num_splits` KV splits: the
- * float32 partial outputs (splits, B, Hq, Sq, D), the partial LSEs
- * (splits, B, Hq, Sq) and B * Hq * Sq int32 split counters, each part
- * rounded up to 256 bytes.  num_splits <= 0 returns the size for
- * FA_MAX_SPLITS.  Returns 0 when one split needs no workspace.
+ * float32 partial outputs (splits, B, Hq, Sq, D) and partial LSEs
+ * (splits, B, Hq, Sq), each rounded up to 256 bytes.  num_splits <= 0
+ * returns the size for FA_MAX_SPLITS.  Returns 0 when one split needs no
+ * workspace.
  */
 size_t fa_kvcache_workspace_size(int B, int Sq, int Hq, int D, int num_splits);
 
@@ -275,12 +275,12 @@ size_t fa_kvcache_workspace_size(int B, int Sq, int Hq, int D, int num_splits);
  *     parts (<= 0: chosen from B, Hkv and the capacity); partials are merged
  *     by a log-sum-exp combine.  workspace >= fa_kvcache_workspace_size(B, Sq,
  *     Hq, D, num_splits) bytes, 256-byte aligned (may be NULL when that is 0);
- *     its split counters are cleared by the call itself (an asynchronous
- *     memset on `stream`), the rest needs no initial contents.
+ *     its contents need not be initialised.
  *   Kernels: with page_size a multiple of 8 tokens (or a contiguous cache)
- *     and no rotary tables the whole call is one kernel: the split kernel
- *     appends k_new / v_new itself and its last split per (b, kv-head) merges
- *     the partials.  Other page sizes run append, split and combine kernels.
+ *     and no rotary tables the split kernel appends k_new / v_new itself, and
+ *     the combine kernel (num_splits > 1) is launched as its programmatic
+ *     dependent (scheduled during its tail).  Other page sizes run separate
+ *     append, split and combine kernels.
  */
 fa_status fa_fwd_kvcache(const void* q, void* k_cache, void* v_cache, const void* k_new,
                          const void* v_new, const int* cache_seqlens, const int* block_table,
@@ -333,11 +333,11 @@ fa_status fa_fwd_kvcache_rotary(const void* q, void* k_cache, void* v_cache, con
  * those callers only.
  *   Arguments: as fa_fwd_kvcache, minus workspace and ws_bytes.  The caller
  *   still owns and passes every input and output buffer.
- *   Scratch: the split-KV partials and split counters go to one file-scope
- *   device array of FA_STATIC_SCRATCH_BYTES (8 MiB) per GPU, part of the
- *   library's device image and held until the process exits.  A call fits
- *   when fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits) <= 8 MiB: about
- *   num_splits * B * Hq * Sq <= 16,200 partial rows at D=128 (32,200 at
+ *   Scratch: the split-KV partials go to one file-scope device array of
+ *   FA_STATIC_SCRATCH_BYTES (8 MiB) per GPU, part of the library's device
+ *   image and held until the process exits.  A call fits when
+ *   fa_kvcache_workspace_size(B, Sq, Hq, D, num_splits) <= 8 MiB:
+ *   num_splits * B * Hq * Sq <= 16,256 partial rows at D=128 (32,263 at
  *   D=64); larger requests return FA_ERR_INVALID_ARG before anything is
  *   launched.
  *   With num_splits <= 0 the call takes fa_fwd_kvcache's automatic split
@@ -354,11 +354,10 @@ fa_status fa_fwd_kvcache_rotary(const void* q, void* k_cache, void* v_cache, con
  *   that of the device status word) is then stale, so no call of this library
  *   may follow a cudaDeviceReset in the same process.
  *   Sharing: every call on a device uses the same array, which keeps the last
- *   call's partials.  What must start at zero (the split counters) is
- *   cleared by each call before its kernel runs; every partial row is written
- *   before it is read.  Calls whose executions overlap on the GPU (other
- *   streams, other host threads) race on the array and must be serialised by
- *   the caller.
+ *   call's partials (nothing in it needs to start at zero: every partial row
+ *   is written before it is read).  Calls whose executions overlap on the GPU
+ *   (other streams, other host threads) race on the array and must be
+ *   serialised by the caller.
  */
 fa_status fa_fwd_kvcache_noalloc(const void* q, void* k_cache, void* v_cache, const void* k_new,
                                  const void* v_new, const int* cache_seqlens, const int* block_table,

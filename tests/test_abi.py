@@ -132,8 +132,8 @@ def test_kvcache_workspace(lib):
     r256 = lambda x: (x + 255) // 256 * 256
     rows = 8 * 1 * 32
     for n in (2, 4, 16, 64):
-        # partial outputs, partial LSEs, one split counter per (b, q-head, query) at most
-        want = r256(n * rows * 128 * 4) + r256(n * rows * 4) + r256(rows * 4)
+        # partial outputs and partial LSEs of every split
+        want = r256(n * rows * 128 * 4) + r256(n * rows * 4)
         assert lib.fa_kvcache_workspace_size(8, 1, 32, 128, n) == want
     assert lib.fa_kvcache_workspace_size(8, 1, 32, 128, 0) == lib.fa_kvcache_workspace_size(8, 1, 32, 128, 64)
 

@@ -67,10 +67,11 @@ def test_decode_small(case, splits):
     np.testing.assert_array_equal(f64(vc), vc_r)
 
 
-@pytest.mark.parametrize("page,launches", [(16, 1), (64, 1), (256, 1), (12, 3)])
-def test_decode_call_is_one_kernel(page, launches):
-    """With TMA-friendly pages the whole call (append, split-KV attention,
-    combine) is one kernel; other page sizes take append + split + combine."""
+@pytest.mark.parametrize("page,launches", [(16, 2), (64, 2), (256, 2), (12, 3)])
+def test_decode_call_launches(page, launches):
+    """With TMA-friendly pages the split kernel appends the new rows itself
+    (split + combine: two kernels); other page sizes take separate append,
+    split and combine kernels."""
     from exact_attention_121_b200 import _lib
     d = inputs.kvcache_inputs(2, 8, 2, 128, page, 512 // page + 1, 500, Sq=1, Snew=1, dtype="bf16", seed=12)
     out, lse, kc, vc, status = _run_case(d, 4)
