@@ -49,13 +49,13 @@ ROOFLINE_UNIT = {"fwd": "H16D128S4096n", "bwd": "H16D128S4096n", "fwd8": "fp8-H1
 # roofline peak is the measured bf16 figure times this ratio
 FP8_OVER_BF16 = 2.0
 # DRAM bytes (read + write) per launch from one ncu capture of that launch
-# (profiles/*_H16D128S4096n.md, profiles/decode_tma_kernel_paged_B8.md).  An
-# entry must be removed whenever its kernel changes.
+# (profiles/fwd_tc_kernel_H16D128S4096n.md, profiles/bwd_tc_kernel_H16D128S4096n.md,
+# profiles/decode_tma_kernel_paged_B8.md).  An entry must be removed whenever
+# its kernel changes.
 TRAFFIC_PER_LAUNCH = {
-    ("fwd", "H16D128S4096n"): 201.704960e6 + 53.250816e6,
-    ("bwd", "H16D128S4096n"): 415.648512e6 + 231.981824e6,
-    ("fwd8", "fp8-H16D128S4096n"): 100.751104e6 + 37.022720e6,
-    ("decode", "decode"): 521.946368e6 + 7.995904e6,
+    ("fwd", "H16D128S4096n"): 201.663744e6 + 54.419200e6,
+    ("bwd", "H16D128S4096n"): 414.194688e6 + 234.748928e6,
+    ("decode", "decode"): 521.964288e6 + 8.303616e6,
 }
 
 
