@@ -392,9 +392,13 @@ class Tracer:
     recorded on the same stream).  A call span runs from arm() to the next
     arm() or disarm()."""
 
-    def __init__(self, lib, enabled=False):
+    def __init__(self, lib, enabled=False, kernel_classes=("fwd", "bwd", "fwd8", "decode")):
         self.lib = lib
         self.enabled = enabled
+        # classes whose dominant kernel gets its own event pair; the others
+        # get the call span only (an event recorded between the decode split
+        # kernel and its dependent combine kernel would serialise them)
+        self.kernel_classes = kernel_classes
         self.pending = []
         self.pending_calls = []
         self.totals = {}
@@ -422,6 +426,8 @@ class Tracer:
         c = torch.cuda.Event(enable_timing=True)
         c.record()
         self._open = (cls, unit.name(), c, work)
+        if cls not in self.kernel_classes:
+            return
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         b.record()
@@ -710,14 +716,23 @@ def main():
     flops_step = sum(u.flops() for u in units)
     peaks, peak_src = load_peaks()
 
-    # device-resident timing with per-kernel trace events
-    tracer = Tracer(lib, enabled=True)
+    # device-resident timing with per-call events and, except for decode,
+    # per-kernel trace events
+    tracer = Tracer(lib, enabled=True, kernel_classes=("fwd", "bwd", "fwd8"))
     gidx = os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local] if "CUDA_VISIBLE_DEVICES" in os.environ else str(local)
     clocks = ClockSampler(gidx)
     clocks.start()
     ms, launches = time_steps(units, args.steps, args.warmup, tracer, barrier=barrier)
     clk = clocks.stop()
     totals = tracer.collect()
+    dec_units = [u for u in units if u.kind == "decode"]
+    if dec_units:
+        # the decode split kernel alone, in a short separate pass
+        ktr = Tracer(lib, enabled=True)
+        time_steps(dec_units, 3, 1, ktr)
+        for cls, v in ktr.collect().items():
+            totals[cls] = v
+        tracer.per_unit.update({k: v for k, v in ktr.per_unit.items() if k[0] == "decode"})
     points, points_summary = per_config(tracer, peaks)
     ms_max = max_over_ranks(ms, pg, dev)
     value = whole_job_tflops(world, flops_step, args.steps, ms_max)

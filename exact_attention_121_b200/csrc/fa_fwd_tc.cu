@@ -455,15 +455,18 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
       if (!full) {
         // Visible keys of this row in this tile as one range [lo, hi]
-        // relative to k0: two compares against constants per score.  (A
-        // per-key test of the three bounds made these tiles ~7x slower than
-        // unmasked ones: 15.5k against 2.1k cycles per tile.)
+        // relative to k0.  (A per-key test of the three bounds made these
+        // tiles ~7x slower than unmasked ones: 15.5k against 2.1k cycles.)
         int lo = 0, hi = min(Sk - 1 - k0, kRows - 1);
         if (p.wl >= 0) lo = max(lo, qpos - p.wl - k0);
         if (p.wr >= 0) hi = min(hi, qpos + p.wr - k0);
+        // one unsigned compare per score: i is visible iff i - lo <= hi - lo
+        // (an empty range moves lo past the tile)
+        if (hi < lo) lo = hi = kRows;
+        const unsigned span = (unsigned)(hi - lo);
 #pragma unroll
         for (int i = 0; i < kRows; ++i)
-          if (i < lo || i > hi) s[i] = __float_as_uint(-INFINITY);
+          if ((unsigned)(i - lo) > span) s[i] = __float_as_uint(-INFINITY);
       }
       {
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
