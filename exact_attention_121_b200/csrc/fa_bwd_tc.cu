@@ -188,6 +188,30 @@ __global__ void __launch_bounds__(kThreadsB, 1)
           tma_load_4d(sb + C::OFF_V + c * C::KV_CHUNK, &tmV, c * 64, hkv, seq.ktma + k0, seq.tb, bar(C::B_KV));
         }
       }
+      // LSE and Delta of a block's 64 rows (two per lane), read into
+      // registers one block ahead so that their global-memory latency
+      // overlaps the wait for the stage instead of delaying the Q/dO copies
+      constexpr int kRowsPerLane = kQ / 32;
+      float nl_next[kRowsPerLane], dl_next[kRowsPerLane];
+      auto fetch_rows = [&](int it) {
+        int h, q0;
+        iter_q(it, h, q0);
+        const long long sbase = stat_base(p, seq, b, h);
+#pragma unroll
+        for (int j = 0; j < kRowsPerLane; ++j) {
+          const int q = q0 + lane + 32 * j;
+          float l2 = INFINITY, dl = 0.f;
+          // rows past the sequence: P = 0, Delta = 0
+          if (q < Sq && FA_IN_BOUNDS(sbase + q >= 0 && sbase + q < p.n_stat, p.status)) {
+            const float l = p.lse[sbase + q];
+            l2 = (l == -INFINITY) ? INFINITY : l * kLog2e;
+            dl = p.delta[sbase + q];
+          }
+          nl_next[j] = -l2;  // x - LSE*log2e becomes one fma: s * scale_log2 + (-LSE*log2e)
+          dl_next[j] = dl;
+        }
+      };
+      fetch_rows(0);
       int issued = 0;
       for (int it = 0; it < n_iter; ++it) {
         const int st = it % C::NQS, u = it / C::NQS;
@@ -199,20 +223,10 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         int h, q0;
         iter_q(it, h, q0);
         float* r = rows + st * 2 * kQ;
-        const float* L = p.lse + stat_base(p, seq, b, h);
-        const float* Dl = p.delta + stat_base(p, seq, b, h);
-        const long long sbase = stat_base(p, seq, b, h);
-        for (int t = lane; t < kQ; t += 32) {
-          const int q = q0 + t;
-          float l2 = INFINITY, dl = 0.f;
-          // rows past the sequence: P = 0, Delta = 0
-          if (q < Sq && FA_IN_BOUNDS(sbase + q >= 0 && sbase + q < p.n_stat, p.status)) {
-            const float l = L[q];
-            l2 = (l == -INFINITY) ? INFINITY : l * kLog2e;  // stored negated below
-            dl = Dl[q];
-          }
-          r[t] = -l2;  // x - LSE*log2e becomes one fma: s * scale_log2 + (-LSE*log2e)
-          r[kQ + t] = dl;
+#pragma unroll
+        for (int j = 0; j < kRowsPerLane; ++j) {
+          r[lane + 32 * j] = nl_next[j];
+          r[kQ + lane + 32 * j] = dl_next[j];
         }
         __syncwarp();
         if (lane == 0) {
@@ -225,6 +239,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
           }
         }
         issued = it + 1;
+        if (it + 1 < n_iter) fetch_rows(it + 1);
       }
       if (*abort_flag && lane == 0) {
         volatile int never = 0;

@@ -132,6 +132,14 @@ def seqlen_sweep_configs():
     return out
 
 
+def long_context_configs():
+    """One 32k-token sequence at hidden 2048: (H=16, D=128) causal and
+    (H=32, D=64) non-causal, twice the longest sweep point."""
+    return [dict(B=1, Sq=32768, Sk=32768, Hq=H, Hkv=H, D=D, dtype="bf16", causal=causal,
+                 window=(-1, -1), softcap=0.0, scale=1.0 / math.sqrt(D), seed=seed, amp=1.0)
+            for H, D, causal, seed in ((16, 128, True, 401), (32, 64, False, 402))]
+
+
 def gqa_local_config():
     """B=2, S=4096, Hq=32, Hkv=8, D=128, bf16, causal, window (1024,0), softcap 30, x2."""
     return dict(B=2, Sq=4096, Sk=4096, Hq=32, Hkv=8, D=128, dtype="bf16", causal=True,

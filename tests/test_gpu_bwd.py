@@ -166,3 +166,31 @@ def test_bwd_seqlen_sweep_sampled(cfg):
     for det, (_, dk, dv) in grads.items():
         check_grad(dk[b, cols, g], dk_r, f"dK b{b} g{g} det={det}")
         check_grad(dv[b, cols, g], dv_r, f"dV b{b} g{g} det={det}")
+
+
+@pytest.mark.parametrize("cfg", inputs.long_context_configs(),
+                         ids=lambda c: "H%dD%dS%d%s" % (c["Hq"], c["D"], c["Sq"], "c" if c["causal"] else "n"))
+def test_bwd_long_context_sampled(cfg):
+    """32k tokens in one sequence, atomic dQ: dQ of sampled query rows of
+    the first and last head and dK/dV of sampled key rows of the last kv-head
+    (every query row of that head evaluated by the oracle)."""
+    q, k, v, do = inputs.attention_inputs(cfg["B"], cfg["Sq"], cfg["Sk"], cfg["Hq"], cfg["Hkv"], cfg["D"],
+                                          cfg["dtype"], seed=cfg["seed"])
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    kw = dict(scale=cfg["scale"], causal=cfg["causal"])
+    out, lse = api.fa_fwd(qd, kd, vd, **kw)
+    dq, dk, dv = (t.cpu() for t in api.fa_bwd(dod, qd, kd, vd, out, lse, **kw))
+    torch.cuda.synchronize()
+    assert api.fa_last_device_status() == 0
+    Q, K, V, DO = (t.to(torch.float64).numpy() for t in (q, k, v, do))
+    rng = np.random.default_rng(cfg["seed"])
+    S, Hq = cfg["Sq"], cfg["Hq"]
+    for h in (0, Hq - 1):
+        rows = _sample(S, rng, 16)
+        dq_r, _, _ = oracle.attn_bwd_rows(DO, Q, K, V, 0, h, rows, cfg["scale"], cfg["causal"])
+        check_grad(dq[0, rows, h], dq_r, f"dQ h{h}")
+    g = cfg["Hkv"] - 1
+    cols = _sample(S, rng, 8)
+    dk_r, dv_r = oracle.attn_bwd_cols(DO, Q, K, V, 0, g, cols, cfg["scale"], cfg["causal"])
+    check_grad(dk[0, cols, g], dk_r, f"dK g{g}")
+    check_grad(dv[0, cols, g], dv_r, f"dV g{g}")

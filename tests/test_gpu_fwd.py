@@ -94,6 +94,22 @@ def test_fwd_seqlen_sweep_sampled(cfg):
     assert np.isfinite(out).all()
 
 
+@pytest.mark.parametrize("cfg", inputs.long_context_configs(),
+                         ids=lambda c: "H%dD%dS%d%s" % (c["Hq"], c["D"], c["Sq"], "c" if c["causal"] else "n"))
+def test_fwd_long_context_sampled(cfg):
+    """32k tokens in one sequence: the LSE and O of sampled rows of the first
+    and last head, the rows near the end seeing every key."""
+    q, k, v, _ = inputs.attention_inputs(cfg["B"], cfg["Sq"], cfg["Sk"], cfg["Hq"], cfg["Hkv"], cfg["D"],
+                                         cfg["dtype"], seed=cfg["seed"], with_dout=False)
+    out, lse = api.fa_fwd(q.cuda(), k.cuda(), v.cuda(), scale=cfg["scale"], causal=cfg["causal"])
+    torch.cuda.synchronize()
+    assert api.fa_last_device_status() == 0
+    out, lse = f64(out), f64(lse)
+    qn, kn, vn = q.float().numpy(), k.float().numpy(), v.float().numpy()
+    _check_sampled(cfg, qn, kn, vn, out, lse, heads=[0, cfg["Hq"] - 1], batches=[0], seed=cfg["seed"])
+    assert np.isfinite(out).all()
+
+
 def test_fwd_gqa_local_sampled():
     cfg = inputs.gqa_local_config()
     q, k, v, _ = inputs.attention_inputs(cfg["B"], cfg["Sq"], cfg["Sk"], cfg["Hq"], cfg["Hkv"], cfg["D"],
