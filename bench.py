@@ -54,7 +54,7 @@ FP8_OVER_BF16 = 2.0
 # its kernel changes.
 TRAFFIC_PER_LAUNCH = {
     ("fwd", "H16D128S4096n"): 201.726976e6 + 55.111680e6,
-    ("bwd", "H16D128S4096n"): 414.194688e6 + 234.748928e6,
+    ("bwd", "H16D128S4096n"): 412.014080e6 + 230.850816e6,
     ("decode", "decode"): 521.964288e6 + 8.303616e6,
 }
 
