@@ -262,25 +262,25 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       auto issue_s = [&](int it) {
         const int x = it & 1, st = it % C::NQS;
         const uint32_t tb = tmem + x * 128;
-        const uint32_t q_st = sb + C::OFF_Q + st * C::Q_TILE;
+        const uint64_t a0 = make_sdesc_sw128(sb + C::OFF_K, 16, 1024);
+        const uint64_t b0 = make_sdesc_sw128(sb + C::OFF_Q + st * C::Q_TILE, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t okv = (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32;
           const uint32_t oq = (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32;
-          mma_ss(tb, make_sdesc_sw128(sb + C::OFF_K + okv, 16, 1024), make_sdesc_sw128(q_st + oq, 16, 1024),
-                 idesc_s, kk > 0 ? 1u : 0u);
+          mma_ss(tb, desc_advance(a0, okv), desc_advance(b0, oq), idesc_s, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_dp = [&](int it) {
         const int x = it & 1, st = it % C::NQS;
         const uint32_t tb = tmem + x * 128;
-        const uint32_t do_st = sb + C::OFF_DO + st * C::Q_TILE;
+        const uint64_t a0 = make_sdesc_sw128(sb + C::OFF_V, 16, 1024);
+        const uint64_t b0 = make_sdesc_sw128(sb + C::OFF_DO + st * C::Q_TILE, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t okv = (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32;
           const uint32_t oq = (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32;
-          mma_ss(tb + 64, make_sdesc_sw128(sb + C::OFF_V + okv, 16, 1024), make_sdesc_sw128(do_st + oq, 16, 1024),
-                 idesc_s, kk > 0 ? 1u : 0u);
+          mma_ss(tb + 64, desc_advance(a0, okv), desc_advance(b0, oq), idesc_s, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_grads = [&](int it) {
@@ -289,22 +289,24 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         const uint32_t q_st = sb + C::OFF_Q + st * C::Q_TILE, do_st = sb + C::OFF_DO + st * C::Q_TILE;
         const uint32_t ds = sb + C::OFF_DS + (it % C::NDS) * C::DS_TILE;
         const bool acc = it > 0;
+        const uint64_t bv = make_sdesc_sw128(do_st, C::Q_CHUNK, 1024);
+        const uint64_t bk = make_sdesc_sw128(q_st, C::Q_CHUNK, 1024);
 #pragma unroll
         for (int kk = 0; kk < kQ / 16; ++kk)
           // 16-query k-step kk of P^T sits at column 32*(kk/2) + 8*(kk%2)
-          mma_ts(tdV, tb + (kk >> 1) * 32 + (kk & 1) * 8, make_sdesc_sw128(do_st + kk * 16 * 128, C::Q_CHUNK, 1024),
-                 idesc_kv,
+          mma_ts(tdV, tb + (kk >> 1) * 32 + (kk & 1) * 8, desc_advance(bv, kk * 16 * 128), idesc_kv,
                  (acc || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < kQ / 16; ++kk)
-          mma_ts(tdK, tb + 64 + (kk >> 1) * 32 + (kk & 1) * 8,
-                 make_sdesc_sw128(q_st + kk * 16 * 128, C::Q_CHUNK, 1024), idesc_kv,
+          mma_ts(tdK, tb + 64 + (kk >> 1) * 32 + (kk & 1) * 8, desc_advance(bk, kk * 16 * 128), idesc_kv,
                  (acc || kk > 0) ? 1u : 0u);
         if (kPair) return;
+        const uint64_t aq = make_sdesc_sw128(sb + C::OFF_K, C::NCH > 1 ? C::KV_CHUNK : 0, 1024);
+        const uint64_t bq = make_sdesc_sw128(ds, C::KV_CHUNK, 1024);
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk)
-          mma_ss(tb + 64, make_sdesc_sw128(sb + C::OFF_K + kk * 16 * 128, C::NCH > 1 ? C::KV_CHUNK : 0, 1024),
-                 make_sdesc_sw128(ds + kk * 16 * 128, C::KV_CHUNK, 1024), idesc_dq, kk > 0 ? 1u : 0u);
+          mma_ss(tb + 64, desc_advance(aq, kk * 16 * 128), desc_advance(bq, kk * 16 * 128), idesc_dq,
+                 kk > 0 ? 1u : 0u);
       };
       // Head dim 64: dQ^T of blocks (it0, it0 + n - 1), n = 2 (or 1 for a
       // last unpaired block) into [384, 384 + 64n): M = 128 head dims, where
@@ -314,10 +316,12 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       auto issue_dq_pair = [&](int it0, int n) {
         const uint32_t ds = sb + C::OFF_DS + (it0 % C::NDS) * C::DS_TILE;
         const uint32_t idesc = n == 2 ? idesc_dq2 : idesc_dq;
+        const uint64_t aq = make_sdesc_sw128(sb + C::OFF_K, 0, 1024);
+        const uint64_t bq = make_sdesc_sw128(ds, C::DS_TILE, 1024);
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk)
-          mma_ss(tmem + 384, make_sdesc_sw128(sb + C::OFF_K + kk * 16 * 128, 0, 1024),
-                 make_sdesc_sw128(ds + kk * 16 * 128, C::DS_TILE, 1024), idesc, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + 384, desc_advance(aq, kk * 16 * 128), desc_advance(bq, kk * 16 * 128), idesc,
+                 kk > 0 ? 1u : 0u);
       };
       bool ok = mbar_wait(bar(C::B_KV), 0, abort_flag, kWaitNs) && mbar_wait(bar(C::B_QF), 0, abort_flag, kWaitNs);
       if (ok) {

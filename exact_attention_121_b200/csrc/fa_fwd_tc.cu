@@ -274,11 +274,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       const uint32_t tO[2] = {tmem + 256, tmem + 384};
       const uint32_t tP[2] = {kSepP ? tmem + 256 + D : tS[0], kSepP ? tmem + 384 + D : tS[1]};
       auto issue_qk = [&](int t, int st) {
+        const uint64_t a0 = sdesc(sb + C::OFF_Q + t * C::TILE, 16);
+        const uint64_t b0 = sdesc(sb + C::OFF_K + st * C::TILE, 16);
 #pragma unroll
         for (int kk = 0; kk < D / KS; ++kk) {
           const uint32_t koff = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          const uint64_t ad = sdesc(sb + C::OFF_Q + t * C::TILE + koff, 16);
-          const uint64_t bd = sdesc(sb + C::OFF_K + st * C::TILE + koff, 16);
+          const uint64_t ad = desc_advance(a0, koff);
+          const uint64_t bd = desc_advance(b0, koff);
           if constexpr (kFp8)
             mma_ss_f8(tS[t], ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
           else
@@ -286,11 +288,12 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
       };
       auto issue_pv = [&](int t, int st, bool acc) {
+        const uint64_t b0 = sdesc(sb + C::OFF_V + st * C::TILE, C::CHUNK);
 #pragma unroll
         for (int kk = 0; kk < kRows / KS; ++kk) {
           // KS keys of V (MN-major: rows of head-dim elements); P packs KS
           // keys into 8 TMEM columns
-          const uint64_t bd = sdesc(sb + C::OFF_V + st * C::TILE + kk * KS * C::ROWB, C::CHUNK);
+          const uint64_t bd = desc_advance(b0, kk * KS * C::ROWB);
           if constexpr (kFp8)
             mma_ts_f8(tO[t], tP[t] + kk * 8, bd, idesc_pv, (acc || kk > 0) ? 1u : 0u);
           else

@@ -217,6 +217,15 @@ __device__ __forceinline__ uint64_t make_sdesc_sw64(uint32_t saddr, uint32_t lbo
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (4ull << 61);
 }
 
+// The descriptor of the same tile `bytes` further on (a multiple of 16): the
+// start-address field holds address >> 4 in the low bits, and every address
+// of the shared-memory window fits it, so the advance is one add.  Building
+// a tile's descriptor once and advancing it per k-step keeps the issuing
+// thread's work per MMA small.
+__device__ __forceinline__ uint64_t desc_advance(uint64_t desc, uint32_t bytes) {
+  return desc + (uint64_t)(bytes >> 4);
+}
+
 // D[tmem] (+)= A[smem] * B[smem]
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accumulate) {
