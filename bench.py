@@ -53,8 +53,8 @@ FP8_OVER_BF16 = 2.0
 # profiles/decode_tma_kernel_paged_B8.md).  An entry must be removed whenever
 # its kernel changes.
 TRAFFIC_PER_LAUNCH = {
-    ("fwd", "H16D128S4096n"): 201.726976e6 + 55.111680e6,
-    ("bwd", "H16D128S4096n"): 412.014080e6 + 230.850816e6,
+    ("fwd", "H16D128S4096n"): 201.473280e6 + 51.724032e6,
+    ("bwd", "H16D128S4096n"): 422.807296e6 + 244.183296e6,
     ("decode", "decode"): 521.964288e6 + 8.303616e6,
 }
 
