@@ -119,3 +119,30 @@ def test_noalloc_automatic_splits_fit_the_array():
     assert api.fa_last_device_status() == 0
     check_out(out, f64(ref_out), torch.bfloat16)
     check_lse(lse, f64(ref_lse))
+
+
+def test_noalloc_matches_the_oracle():
+    """O, LSE and the appended cache rows of the allocation-free call against
+    the float64 oracle (append, then attend), at an explicit and at the
+    automatic split count, for fp16 and bf16."""
+    import oracle
+    import numpy as np
+
+    lib = _lib.load()
+    for seed, splits, dtype in ((37, 3, "bf16"), (38, 0, "fp16")):
+        host = inputs.kvcache_inputs(4, 32, 8, 128, 64, 6, 380, Sq=1, Snew=1, dtype=dtype, seed=seed)
+        d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in host.items()}
+        out = torch.empty_like(d["q"])
+        lse = torch.empty(4, 32, 1, device="cuda")
+        assert _noalloc(lib, d, splits, out, lse) == _lib.FA_OK
+        torch.cuda.synchronize()
+        assert api.fa_last_device_status() == 0
+        o_ref, l_ref, kc_ref, vc_ref = oracle.attn_with_kvcache(
+            host["q"].double().numpy(), host["k_cache"].double().numpy(), host["v_cache"].double().numpy(),
+            host["k_new"].double().numpy(), host["v_new"].double().numpy(), host["cache_seqlens"].numpy(),
+            host["block_table"].numpy(), host["page_size"], causal=True)
+        check_out(out, o_ref, host["q"].dtype)
+        check_lse(lse, l_ref)
+        # the appended rows are exact copies of k_new / v_new
+        assert np.array_equal(d["k_cache"].double().cpu().numpy(), kc_ref)
+        assert np.array_equal(d["v_cache"].double().cpu().numpy(), vc_ref)
