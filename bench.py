@@ -55,7 +55,7 @@ FP8_OVER_BF16 = 2.0
 TRAFFIC_PER_LAUNCH = {
     ("fwd", "H16D128S4096n"): 201.473280e6 + 51.724032e6,
     ("bwd", "H16D128S4096n"): 422.807296e6 + 244.183296e6,
-    ("decode", "decode"): 521.964288e6 + 8.303616e6,
+    ("decode", "decode"): 521.979136e6 + 5.864960e6,
 }
 
 
