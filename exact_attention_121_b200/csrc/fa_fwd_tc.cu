@@ -127,6 +127,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   // Head dim 64 leaves TMEM room for P beside O (P_t at [256+128t+64, +64)),
   // so S_t can be refilled while P_t still feeds the PV product.
   constexpr bool kSepP = (D == 64);
+  // the K-stage-free signal comes from tile B's S commit (one commit fewer
+  // per key tile) where the stage count makes that safe: an odd count of at
+  // least 3, and the single-P loop, whose tile B commit follows both QK^T
+  constexpr bool kKeFromS = !kSepP && (C::NSK % 2 == 1) && C::NSK >= 3;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -231,7 +235,15 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         const int sv = j % C::NSV, uv = j / C::NSV;
         const int k0 = tile_k0(j);
         (void)FA_IN_BOUNDS(k0 >= 0 && k0 < Sk, p.status);  // TMA fills outside the tensor; report only
-        if (j >= C::NSK && !mbar_wait(bar(C::B_KE + sk), (uk - 1) & 1, abort_flag, kTcWaitNs)) {
+        // K stage free: both QK^T products of tile j - NSK done.  Head dim
+        // 128 reads it from tile B's S barrier (its product is issued after
+        // tile A's; phase = tile): with NSK = 3 stages that barrier is never
+        // two phases past tile j - NSK here, since tile j's K is not issued.
+        const bool free_k =
+            j < C::NSK ||
+            (!kKeFromS ? mbar_wait(bar(C::B_KE + sk), (uk - 1) & 1, abort_flag, kTcWaitNs)
+                       : mbar_wait(bar(C::B_S + 1), (j - C::NSK) & 1, abort_flag, kTcWaitNs));
+        if (!free_k) {
           fail();
           break;
         }
@@ -310,7 +322,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
         issue_qk(1, 0);
         mma_commit(bar(C::B_S + 1));
-        mma_commit(bar(C::B_KE + 0));
+        if (!kKeFromS) mma_commit(bar(C::B_KE + 0));
       }
       // Separate-P order: QK_t(j+1) as soon as the softmax has read S_t(j),
       // PV_t(j) once it has written P_t(j).
@@ -378,7 +390,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         if (more) {
           issue_qk(1, sk1);
           mma_commit(bar(C::B_S + 1));
-          mma_commit(bar(C::B_KE + sk1));
+          if (!kKeFromS) mma_commit(bar(C::B_KE + sk1));
         } else {
           mma_commit(bar(C::B_O + 1));
         }
