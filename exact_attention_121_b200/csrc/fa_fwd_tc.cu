@@ -70,8 +70,10 @@ struct TcCfg {
   static constexpr int CHUNK_ELEMS = kF8 ? D : 64;          // head-dim elements per chunk
   static constexpr int NCHUNK = D / CHUNK_ELEMS;
   static constexpr int TILE = CHUNK * NCHUNK;        // one 128-row tile
-  static constexpr int NSK = (D == 128) ? 3 : 4;     // K stages
-  static constexpr int NSV = (D == 128) ? 2 : 4;     // V stages
+  // odd stage counts at head dim 64: the loader can then take "stage free"
+  // from the S and PV barriers (see the kernel)
+  static constexpr int NSK = (D == 128) ? 3 : 5;     // K stages
+  static constexpr int NSV = (D == 128) ? 2 : 5;     // V stages
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = 2 * TILE;
   static constexpr int OFF_V = OFF_K + NSK * TILE;
@@ -127,10 +129,15 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   // Head dim 64 leaves TMEM room for P beside O (P_t at [256+128t+64, +64)),
   // so S_t can be refilled while P_t still feeds the PV product.
   constexpr bool kSepP = (D == 64);
-  // the K-stage-free signal comes from tile B's S commit (one commit fewer
-  // per key tile) where the stage count makes that safe: an odd count of at
-  // least 3, and the single-P loop, whose tile B commit follows both QK^T
-  constexpr bool kKeFromS = !kSepP && (C::NSK % 2 == 1) && C::NSK >= 3;
+  // "Stage free" signals without commits of their own (one tcgen05 commit
+  // fewer each per key tile): K from tile B's S commit, which follows both
+  // QK^T of a tile; V (separate-P loop) from tile B's PV commit, which
+  // follows both P.V.  A barrier whose phase is the tile cannot be two
+  // phases past the tile the loader waits for when the stage count is odd:
+  // the tile being loaded has not been issued, so its products cannot
+  // complete.
+  constexpr bool kKeFromS = (C::NSK % 2 == 1) && C::NSK >= 3;
+  constexpr bool kVeFromPv = kSepP && (C::NSV % 2 == 1) && C::NSV >= 3;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -235,10 +242,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         const int sv = j % C::NSV, uv = j / C::NSV;
         const int k0 = tile_k0(j);
         (void)FA_IN_BOUNDS(k0 >= 0 && k0 < Sk, p.status);  // TMA fills outside the tensor; report only
-        // K stage free: both QK^T products of tile j - NSK done.  Head dim
-        // 128 reads it from tile B's S barrier (its product is issued after
-        // tile A's; phase = tile): with NSK = 3 stages that barrier is never
-        // two phases past tile j - NSK here, since tile j's K is not issued.
+        // K stage free: both QK^T products of tile j - NSK done
         const bool free_k =
             j < C::NSK ||
             (!kKeFromS ? mbar_wait(bar(C::B_KE + sk), (uk - 1) & 1, abort_flag, kTcWaitNs)
@@ -251,7 +255,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         for (int c = 0; c < C::NCHUNK; ++c)
           tma_load_4d(sb + C::OFF_K + sk * C::TILE + c * C::CHUNK, &tmK, c * C::CHUNK_ELEMS, g, seq.ktma + k0,
                       seq.tb, bar(C::B_KF + sk));
-        if (j >= C::NSV && !mbar_wait(bar(C::B_VE + sv), (uv - 1) & 1, abort_flag, kTcWaitNs)) {
+        const bool free_v =
+            j < C::NSV ||
+            (!kVeFromPv ? mbar_wait(bar(C::B_VE + sv), (uv - 1) & 1, abort_flag, kTcWaitNs)
+                        : mbar_wait(bar(C::B_PV + 1), (j - C::NSV) & 1, abort_flag, kTcWaitNs));
+        if (!free_v) {
           fail();
           issued = -(j + 1);  // K of tile j is in flight, V is not
           break;
@@ -351,14 +359,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           tc_fence_after();
           issue_qk(1, sk1);
           mma_commit(bar(C::B_S + 1));
-          mma_commit(bar(C::B_KE + sk1));
+          if (!kKeFromS) mma_commit(bar(C::B_KE + sk1));
         }
         ok = mbar_wait(bar(C::B_P + 1), j & 1, abort_flag, kTcWaitNs);
         if (!ok) break;
         tc_fence_after();
         issue_pv(1, sv, j > 0);
         mma_commit(bar(C::B_PV + 1));
-        mma_commit(bar(C::B_VE + sv));
+        if (!kVeFromPv) mma_commit(bar(C::B_VE + sv));
         if (!more) mma_commit(bar(C::B_O + 1));
       }
       for (int j = 0; !kSepP && ok && j < n_tiles; ++j) {
