@@ -55,7 +55,7 @@ FP8_OVER_BF16 = 2.0
 # profiles/decode_tma_kernel_paged_B8.md).  An entry must be removed whenever
 # its kernel changes.
 TRAFFIC_PER_LAUNCH = {
-    ("fwd", "H16D128S4096n"): 201.473280e6 + 51.724032e6,
+    ("fwd", "H16D128S4096n"): 201.659904e6 + 51.587840e6,
     ("bwd", "H16D128S4096n"): 422.807296e6 + 244.183296e6,
     ("decode", "decode"): 521.979136e6 + 5.864960e6,
 }
