@@ -75,6 +75,8 @@ CASES = [
     (1, 200, 513, 4, 4, 64, False, (-1, -1), 0.0, False),
     (1, 257, 257, 2, 2, 64, False, (-1, -1), 20.0, True),
     (1, 700, 700, 4, 1, 64, True, (100, 0), 0.0, True),
+    # more key tiles than the 5 K/V stages of head dim 64, ragged tail
+    (1, 256, 1300, 2, 2, 64, False, (-1, -1), 0.0, True),
 ]
 
 

@@ -33,6 +33,12 @@ SMALL = [
     (3, 190, 190, 6, 3, 128, "fp16", True, (50, 0), 10.0, None, 2.0),
     (1, 512, 512, 4, 1, 128, "bf16", True, (-1, -1), 30.0, 0.3, 2.0),
     (2, 384, 384, 2, 2, 64, "bf16", False, (-1, -1), 0.0, None, 1.0),
+    # more key tiles than K/V stages (5 at head dim 64, 3 and 2 at 128), ragged
+    # tails: every stage is reused and every stage-free wait runs
+    (1, 300, 1317, 2, 1, 64, "bf16", False, (-1, -1), 0.0, None, 1.0),
+    (1, 1100, 1100, 2, 2, 64, "fp16", True, (-1, -1), 0.0, None, 1.0),
+    (1, 260, 777, 2, 2, 128, "bf16", False, (-1, -1), 0.0, None, 1.0),
+    (1, 900, 900, 2, 1, 128, "bf16", True, (-1, -1), 0.0, None, 1.0),
 ]
 
 
