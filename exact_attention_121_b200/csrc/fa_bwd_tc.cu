@@ -76,8 +76,9 @@ struct BwdTcCfg {
   static constexpr int OFF_DQ = OFF_DS + NDS * DS_TILE; // NDQ tiles
   static constexpr int OFF_ROW = OFF_DQ + NDQ * DQ_TILE;  // [stage][LSE*log2e 64 | Delta 64]
   static constexpr int OFF_BAR = OFF_ROW + NQS * 2 * kQ * 4;
-  enum { B_KV = 0, B_QF = 1, B_QE = 4, B_SDP = 7, B_PDS = 9, B_DQF = 11, B_TMF = 13, B_FIN = 15, B_DRAIN = 16,
-         B_DQT_FULL = 17, B_DQT_FREE = 18, NBAR = 19 };
+  enum { B_KV = 0, B_QF = 1, B_QE = B_QF + NQS, B_SDP = B_QE + NQS, B_PDS = B_SDP + 2, B_DQF = B_PDS + 2,
+         B_TMF = B_DQF + 2, B_FIN = B_TMF + 2, B_DRAIN = B_FIN + 1, B_DQT_FULL = B_DRAIN + 1,
+         B_DQT_FREE = B_DQT_FULL + 1, NBAR = B_DQT_FREE + 1 };
   static constexpr int OFF_TMEM = OFF_BAR + 8 * NBAR;
   static constexpr int OFF_ABORT = OFF_TMEM + 4;
   static constexpr int OFF_ITEM = OFF_ABORT + 4;  // claimed work item (deterministic mode)
@@ -94,6 +95,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   using C = BwdTcCfg<D_>;
   constexpr int D = C::D;
   constexpr bool kPair = C::PAIR;
+  static_assert(C::SMEM <= 227 * 1024, "shared memory per CTA");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
